@@ -1,0 +1,87 @@
+"""Planted mistakes in the oracle (on the CPU) must each fail at least one pin.
+
+Every mutation below is a plausible slip in writing the oracle: a dropped
+term, a wrong rounding mode, a transposed operand, a missing factor.  The
+test patches the oracle function, runs the pins that should catch it, and
+requires that at least one of them fails.
+"""
+import numpy as np
+import pytest
+
+import tests.test_oracle_pins as pins
+from oracle import ref
+
+
+def _trunc_bf16(v):
+    u = np.asarray(v, np.float32).view(np.uint32)
+    return (u >> 16).astype(np.uint16)
+
+
+def _e4m3_half_away(v):
+    v = np.asarray(v, np.float32).astype(np.float64)
+    a = np.abs(v)
+    _, E = np.frexp(np.where(a > 0, a, 1.0))
+    q = np.ldexp(1.0, np.maximum(E.astype(np.int64) - 1, -6) - 3)
+    r = np.minimum(np.floor(a / q + 0.5) * q, 448.0)
+    return ref._orig_e4m3((np.sign(v) * r).astype(np.float32))
+
+
+def _e4m3_no_sat(v):
+    v = np.asarray(v, np.float32)
+    out = ref._orig_e4m3(v)
+    return np.where(np.abs(v) > 448, np.uint8(0x7F), out).astype(np.uint8)
+
+
+MUTATIONS = {
+    # name: (oracle attribute, mutated version, pins expected to catch it)
+    "bf16_truncates": ("bf16_bits_from_f32", lambda orig: _trunc_bf16,
+                       ["test_bf16_matches_torch_and_ml_dtypes"]),
+    "e4m3_half_away": ("e4m3_bits_from_f32", lambda orig: _e4m3_half_away,
+                       ["test_e4m3_hand_cases", "test_e4m3_random_fp32"]),
+    "e4m3_no_saturation": ("e4m3_bits_from_f32", lambda orig: _e4m3_no_sat,
+                           ["test_e4m3_hand_cases", "test_worked_example_golden"]),
+    "up_proj_operand_swapped": ("up_proj", lambda orig: (lambda x, W1: ref.bf16_to_f64(x) @ ref.bf16_to_f64(W1).T[:, ::-1]),
+                                ["test_up_proj_bruteforce"]),
+    "relu_dropped": ("relu2_post", lambda orig: (lambda pre: ref.bf16_bits_from_f32((ref.f32(pre) * ref.f32(pre)).astype(np.float32))),
+                     ["test_relu2_invariants"]),
+    "square_dropped": ("relu2_post", lambda orig: (lambda pre: ref.bf16_bits_from_f32(np.maximum(ref.f32(pre), np.float32(0)))),
+                       ["test_relu2_invariants", "test_worked_example_golden"]),
+    "margin_dropped": ("scale_update", lambda orig: (lambda st, A: orig(dict(st, margin=np.float32(1.0)), A) | {"margin": st["margin"]}),
+                       ["test_scale_exact_values"]),
+    "scale_inv_not_reciprocal": ("scale_update", lambda orig: (lambda st, A: (lambda o: o | {"scale_inv": o["scale"]})(orig(st, A))),
+                                 ["test_scale_exact_values", "test_worked_example_golden", "test_scale_keeps_previous_on_degenerate_amax"]),
+    "w2_cache_not_transposed": ("w2_cache", lambda orig: (lambda W2: (lambda r: (r[0].T.copy(), r[1], r[2]))(orig(W2))),
+                                ["test_w2_cache_matches_library", "test_worked_example_golden"]),
+    "dpre_factor_two_dropped": ("bwd_dpre", lambda orig: (lambda post, dOut, W2: ref.bf16_bits_from_f32(ref.f32(np.sqrt(ref.bf16_to_f64(post)) * (ref.bf16_to_f64(dOut) @ ref.bf16_to_f64(W2).T)))),
+                                ["test_backward_vs_torch_autograd"]),
+    "dpre_uses_post_not_sqrt": ("bwd_dpre", lambda orig: (lambda post, dOut, W2: ref.bf16_bits_from_f32(ref.f32(2 * ref.bf16_to_f64(post) * (ref.bf16_to_f64(dOut) @ ref.bf16_to_f64(W2).T)))),
+                                ["test_backward_vs_torch_autograd"]),
+    "dw2_scaled": ("bwd_dw2", lambda orig: (lambda post, dOut: ref.f32(ref.bf16_to_f64(post).T @ (ref.bf16_to_f64(dOut) * 0.5))),
+                   ["test_backward_vs_torch_autograd", "test_backward_gemms_bruteforce"]),
+    "dx_wrong_operand": ("bwd_dx", lambda orig: (lambda dPre, W1: ref.bf16_bits_from_f32(ref.f32(ref.bf16_to_f64(dPre) @ ref.bf16_to_f64(W1)[::-1]))),
+                         ["test_backward_gemms_bruteforce"]),
+    "rmsnorm_bwd_sign": ("rmsnorm_bwd", lambda orig: (lambda r, dx: -orig(r, dx)),
+                         ["test_rmsnorm_constant_rows_and_autograd"]),
+    "amax_drops_last_block": ("partial_amax", lambda orig: (lambda post, rows, cols: orig(post, rows, cols)[:-1]),
+                              ["test_amax_partials_equal_brute_max"]),
+}
+
+PARAMS = {"test_e4m3_exhaustive_over_bf16": dict(s=3.7),
+          "test_scale_update_closed_form": dict(A=3.0, margin=2.0),
+          "test_scale_keeps_previous_on_degenerate_amax": dict(A=0.0)}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    attr, make, catchers = MUTATIONS[name]
+    orig = getattr(ref, attr)
+    monkeypatch.setattr(ref, "_orig_e4m3", ref.e4m3_bits_from_f32, raising=False)
+    monkeypatch.setattr(ref, attr, make(orig))
+    failed = []
+    for pin in catchers:
+        fn = getattr(pins, pin)
+        try:
+            fn(**PARAMS.get(pin, {}))
+        except Exception:
+            failed.append(pin)
+    assert failed, f"mutation {name} passed the pins {catchers}"
