@@ -1,0 +1,448 @@
+#!/usr/bin/env python
+"""Benchmark of the fused FP8 ReLU^2 MLP block (fwd + bwd) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload step16k]
+                    [--impl ours|reference]
+
+One step = one pass of the whole block over one batch of synthetic tokens:
+fused up-projection (BF16 post + FP8 copy + partial amax), FP8
+down-projection, the BF16 backward (dPre through sqrt(post), dX, dW1, dW2),
+the partial-amax reduction with the delayed-scale update, and the W2 FP8
+cache refresh.  Inputs are resident in HBM when the timed region starts; L2
+is flushed (a 256 MiB write) between timed steps, outside the step's events.
+The per-kernel CUDA events are recorded on the launching stream inside the
+timed steps.  ``e2e`` repeats the measurement through the same public API
+with the step's inputs copied in from pinned host memory and its results
+(out, dX) copied back, inside the timed region.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch
+(weak scaling, data-parallel replicas, no collective on the data path); the
+time is the max over ranks.  Rank 0 prints one JSON line.
+
+``--impl reference`` times the CPU oracle on the host cores on a bounded
+sample of the same workload (rank 0 only; other ranks exit 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ReLU² MLP fwd+bwd tokens/s and % of FP8/BF16 roofline at d=768,h=3072"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="step16k", choices=["step16k", "train49k", "heavytail"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# peaks
+# ---------------------------------------------------------------------------
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def measure_fp8_peak(torch, bf16_peak):
+    """Burst e4m3 GEMM throughput (8192^3, torch._scaled_mm) for the FP8
+    roofline; falls back to 2x the BF16 peak (the nominal dense ratio)."""
+    try:
+        n = 8192
+        a = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device="cuda")
+        for _ in range(3):
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        best = 1e30
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+            e0.record()
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1) * 1e-3)
+        del a, b
+        return 2 * n ** 3 / best / 1e12, "measured (torch._scaled_mm e4m3 8192^3, best of 10)"
+    except Exception as ex:  # pragma: no cover
+        return 2 * bf16_peak, f"2x bf16 peak (nominal ratio; scaled_mm failed: {type(ex).__name__})"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML polled from a thread)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for k, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per kernel (per launch at M tokens)
+# ---------------------------------------------------------------------------
+
+def kernel_work(M, d, h):
+    """FLOPs (by precision) and minimum HBM bytes of each kernel of a step."""
+    F = 2 * M * d * h
+    return {
+        "up_fused": dict(bf16=F, fp8=0, bytes=2 * M * d + 2 * h * d + 2 * M * h + M * h),
+        "down_fp8": dict(bf16=0, fp8=F, bytes=M * h + d * h + 2 * M * d),
+        "bwd_dpre": dict(bf16=F, fp8=0, bytes=2 * M * d + 2 * h * d + 2 * M * h + 2 * M * h),
+        "bwd_dx": dict(bf16=F, fp8=0, bytes=2 * M * h + 2 * h * d + 2 * M * d),
+        "bwd_dw": dict(bf16=2 * F, fp8=0, bytes=2 * M * h + 2 * M * d + 2 * M * h + 2 * M * d + 8 * h * d),
+        "amax_scale": dict(bf16=0, fp8=0, bytes=4 * (4 * -(-M // 128)) * -(-h // 256)),
+        "w2_cache": dict(bf16=0, fp8=0, bytes=2 * (2 * h * d) + d * h),
+    }
+
+
+def src_digest():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "fp8_relu_mlp_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return {}
+    d = json.load(open(p))
+    if d.get("src_digest") != src_digest():
+        return {}
+    return d.get("workloads", {}).get(workload, {})
+
+
+# ---------------------------------------------------------------------------
+# oracle on the host cores
+# ---------------------------------------------------------------------------
+
+def oracle_step_timer(W, tokens, seed=0):
+    """Returns (fn running one oracle step on `tokens` tokens of the workload,
+    threads used)."""
+    import numpy as np
+    from fp8_relu_mlp_b200 import synth
+    from oracle import ref
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        threads = 1
+    P = synth.make_problem(tokens, W.d, W.h, seed=seed)
+    st = {"s": ref.scale_state_init(W.margin, 1.0)}
+
+    def step():
+        W2q_t, s_w, s_wi = ref.w2_cache(P["W2"])
+        f = ref.forward(P["x"], P["W1"], W2q_t, s_wi, st["s"]["scale"], st["s"]["scale_inv"])
+        ref.backward(P["x"], P["W1"], P["W2"], f["post"], P["dOut"])
+        st["s"] = ref.scale_update(st["s"], f["amax"])
+        return np
+    return step, threads
+
+
+def cpu_baseline(W, seconds, tokens=512):
+    step, threads = oracle_step_timer(W, tokens)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        step()
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or reps >= 50:
+            break
+    return {"value": tokens * reps / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{reps} oracle steps of {tokens} tokens of the {W.name} workload "
+                      f"(d={W.d}, h={W.h}; fwd+bwd+scale+W2 cache), {el:.1f} s"}
+
+
+def run_reference(a, W, world, rank):
+    if rank != 0:
+        return
+    tokens = 256
+    step, threads = oracle_step_timer(W, tokens)
+    for _ in range(a.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        step()
+    el = time.perf_counter() - t0
+    v = tokens * a.steps / el
+    sample = f"{a.steps} oracle steps of {tokens} tokens each (bounded sample of {W.name}: M={W.M}, d={W.d}, h={W.h})"
+    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": a.gpus, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": el / a.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64 (bf16/e4m3 rounding emulated)", "data": "synthetic",
+            "config": config_of(W), "impl": "reference",
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(W):
+    return {"workload": f"{W.name}: {W.description}", "M_per_gpu": W.M, "d": W.d, "h": W.h,
+            "x_dist": W.x_dist, "l2": "flushed (256 MiB write) between timed steps"}
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+
+def run_ours(a, W, world, rank, local_rank):
+    import numpy as np
+    import torch
+    from fp8_relu_mlp_b200 import _abi as A
+    from fp8_relu_mlp_b200 import synth
+    from fp8_relu_mlp_b200.block import MLPBlock
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    M, d, h = W.M, W.d, W.h
+    peaks = load_peaks()
+    fp8_peak, fp8_src = measure_fp8_peak(torch, peaks["bf16_tflops"])
+
+    blk = MLPBlock(M, d, h, device=dev, margin=W.margin)
+    P = synth.make_problem(M, d, h, seed=rank, x_dist=W.x_dist)
+    blk.x.copy_(MLPBlock.bits_to_bf16(P["x"], dev))
+    blk.W1.copy_(MLPBlock.bits_to_bf16(P["W1"], dev))
+    blk.W2.copy_(MLPBlock.bits_to_bf16(P["W2"], dev))
+    blk.dOut.copy_(MLPBlock.bits_to_bf16(P["dOut"], dev))
+    blk.refresh_w2_cache()
+    blk.calibrate()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    names = ["up_fused", "down_fp8", "bwd_dpre", "bwd_dx", "bwd_dw", "amax_scale", "w2_cache"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        A.fp8mlp_up_proj_fused(M, d, h, blk.x, blk.W1, blk.state, blk.post, blk.post_fp8, blk.partial_amax)
+        mark(1)
+        A.fp8mlp_down_proj_fp8(M, d, h, blk.post_fp8, blk.W2q_t, blk.w2_scale_inv, blk.state, blk.out)
+        mark(2)
+        A.fp8mlp_bwd_dpre(M, d, h, blk.dOut, blk.W2, blk.post, blk.dPre)
+        mark(3)
+        A.fp8mlp_bwd_dx(M, d, h, blk.dPre, blk.W1, blk.dX)
+        mark(4)
+        A.fp8mlp_bwd_dw(M, d, h, blk.x, blk.dPre, blk.post, blk.dOut, blk.dW1, blk.dW2)
+        mark(5)
+        blk.update_scale()
+        mark(6)
+        blk.refresh_w2_cache()
+        mark(7)
+
+    for _ in range(max(a.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    A.fp8mlp_clear_device_status()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(a.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = A.fp8mlp_kernel_launch_count()
+    with ClockSampler(local_rank) as clk:
+        for i in range(a.steps):
+            flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize()
+    launches = A.fp8mlp_kernel_launch_count() - n0
+    if dist:
+        dist.barrier()
+    status = A.fp8mlp_get_device_status()
+    per_kernel = {n: [] for n in names}
+    step_ms = []
+    for ev in evs:
+        for k, n in enumerate(names):
+            per_kernel[n].append(ev[k].elapsed_time(ev[k + 1]))
+        step_ms.append(ev[0].elapsed_time(ev[7]))
+    total_s = sum(step_ms) * 1e-3
+    if dist:
+        t = torch.tensor([total_s], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_s = float(t.item())
+    value = M * world * a.steps / total_s
+
+    # roofline of the dominant kernel and of the whole step
+    work = kernel_work(M, d, h)
+    avg = {n: statistics.mean(v) * 1e-3 for n, v in per_kernel.items()}
+    dom = max(avg, key=lambda n: avg[n])
+    wd = work[dom]
+    peak_dom = fp8_peak if wd["fp8"] else peaks["bf16_tflops"]
+    achieved = (wd["bf16"] + wd["fp8"]) / avg[dom] / 1e12
+    traffic = load_traffic(W.name).get(dom)
+    roof_t = 0.0
+    for n, w in work.items():
+        roof_t += max(w["bf16"] / (peaks["bf16_tflops"] * 1e12) + w["fp8"] / (fp8_peak * 1e12),
+                      w["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    fwd_s = avg["up_fused"] + avg["down_fp8"]
+    fwd_roof = (work["up_fused"]["bf16"] / (peaks["bf16_tflops"] * 1e12) +
+                work["down_fp8"]["fp8"] / (fp8_peak * 1e12))
+
+    e2e = None
+    if not a.no_e2e:
+        e2e = measure_e2e(a, blk, P, torch, dev, stream, M, world, dist)
+
+    line = None
+    if rank == 0:
+        clocks = clk.summary()
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": total_s / a.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16+e4m3 (fp32 accumulate)",
+            "data": "synthetic (seeded; shapes of the 768-dim GPT-2-small / nanochat MLP)",
+            "config": dict(config_of(W), parallelism=f"dp{world} replicas" if world > 1 else "single GPU"),
+            "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak_dom,
+                         "unit": "TFLOP/s", "frac": achieved / peak_dom, "traffic": traffic,
+                         "peak_source": (fp8_src if wd["fp8"] else
+                                         f"bf16_tflops burst of {peaks['source']} peaks")},
+            "step_roofline": {"roofline_ms": roof_t * 1e3, "measured_ms": total_s / a.steps * 1e3,
+                              "frac": roof_t / (total_s / a.steps),
+                              "fwd_ms": fwd_s * 1e3, "fwd_roofline_ms": fwd_roof * 1e3,
+                              "fwd_frac": fwd_roof / fwd_s, "fwd_tokens_per_s": M / fwd_s,
+                              "peaks": {"bf16_tflops": peaks["bf16_tflops"], "fp8_tflops": fp8_peak,
+                                        "hbm_gbs": peaks["hbm_gbs"]}},
+            "kernels_ms": {n: statistics.mean(v) for n, v in per_kernel.items()},
+            "clocks": clocks, "gpu_launches": int(launches), "device_status": status,
+        }
+        if e2e:
+            line["e2e"] = e2e
+        if not a.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(W, a.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return line
+
+
+def measure_e2e(a, blk, P, torch, dev, stream, M, world, dist):
+    """Same step through the public API with host buffers: the step's inputs
+    (x, dOut) come from pinned host memory and its results (out, dX) go back
+    to pinned host memory inside the timed region."""
+    import numpy as np
+    xh = torch.from_numpy(P["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    gh = torch.from_numpy(P["dOut"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    oh = torch.empty_like(blk.out, device="cpu").pin_memory()
+    dxh = torch.empty_like(blk.dX, device="cpu").pin_memory()
+
+    def step():
+        blk.x.copy_(xh, non_blocking=True)
+        blk.dOut.copy_(gh, non_blocking=True)
+        blk.forward()
+        blk.backward()
+        blk.update_scale()
+        blk.refresh_w2_cache()
+        oh.copy_(blk.out, non_blocking=True)
+        dxh.copy_(blk.dX, non_blocking=True)
+
+    for _ in range(max(a.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    e0.record(stream)
+    for _ in range(a.steps):
+        step()
+    e1.record(stream)
+    e1.synchronize()
+    t = e0.elapsed_time(e1) * 1e-3
+    if dist:
+        tt = torch.tensor([t], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t = float(tt.item())
+    return {"value": M * world * a.steps / t, "unit": "tokens/s",
+            "h2d_bytes_per_step": int(xh.numel() * 2 + gh.numel() * 2),
+            "d2h_bytes_per_step": int(oh.numel() * 2 + dxh.numel() * 2)}
+
+
+def main():
+    a = parse()
+    from fp8_relu_mlp_b200 import synth
+    W = synth.WORKLOADS[a.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if a.impl == "reference":
+        run_reference(a, W, world, rank)
+        return 0
+    run_ours(a, W, world, rank, local_rank)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,92 @@
+"""One fused FP8 ReLU^2 MLP block: device buffers plus the call sequence.
+
+Torch is used only to allocate device memory and to name the stream; every
+step runs in libfp8mlp's kernels through the C ABI (:mod:`._abi`).
+
+Training step at step t ("A Retrospective on Our World Records", Modded-NanoGPT
+Main Track):
+    forward      fused up-projection (post, FP8 copy under s_t, partial amax)
+                 + FP8 down-projection against the transposed W2 cache
+    backward     dPre = 2 sqrt(post) dPost, then dX, dW1, dW2 (BF16)
+    scale        reduce the partial amax -> s_{t+1}
+    (optimizer)  caller updates W1 / W2
+    W2 cache     refreshed after the update
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _abi as A
+
+
+class MLPBlock:
+    def __init__(self, M: int, d: int, h: int, device="cuda", margin: float = 2.0, initial_scale: float = 1.0,
+                 with_backward: bool = True, stream=None):
+        self.M, self.d, self.h = M, d, h
+        self.device = torch.device(device)
+        self.stream = stream
+        dev = self.device
+        bf, u8, f32 = torch.bfloat16, torch.uint8, torch.float32
+        self.x = torch.zeros(M, d, dtype=bf, device=dev)
+        self.W1 = torch.zeros(h, d, dtype=bf, device=dev)
+        self.W2 = torch.zeros(h, d, dtype=bf, device=dev)
+        self.W2q_t = torch.zeros(d, h, dtype=u8, device=dev)
+        self.w2_scale_inv = torch.ones(4, dtype=f32, device=dev)
+        self.state = torch.zeros(8, dtype=f32, device=dev)  # fp8mlp_scale_state (32 bytes)
+        self.post = torch.empty(M, h, dtype=bf, device=dev)
+        self.post_fp8 = torch.empty(M, h, dtype=u8, device=dev)
+        rb, cb, _, _ = A.fp8mlp_partial_amax_shape(M, h)
+        self.partial_amax = torch.zeros(rb, cb, dtype=f32, device=dev)
+        self.out = torch.empty(M, d, dtype=bf, device=dev)
+        self.workspace = torch.zeros(max(256, A.fp8mlp_workspace_size(M, d, h)), dtype=u8, device=dev)
+        if with_backward:
+            self.dOut = torch.zeros(M, d, dtype=bf, device=dev)
+            self.dPre = torch.empty(M, h, dtype=bf, device=dev)
+            self.dX = torch.empty(M, d, dtype=bf, device=dev)
+            self.dW1 = torch.empty(h, d, dtype=f32, device=dev)
+            self.dW2 = torch.empty(h, d, dtype=f32, device=dev)
+        A.fp8mlp_scale_state_init(self.state, margin, initial_scale, self.stream)
+
+    # ------------------------------------------------------------------ calls
+    def refresh_w2_cache(self):
+        A.fp8mlp_w2_fp8_cache_refresh(self.h, self.d, self.W2, self.W2q_t, self.w2_scale_inv, self.workspace,
+                                      self.stream)
+
+    def calibrate(self):
+        """Step 0: post and partial amax only, then the first scale."""
+        A.fp8mlp_mlp_fwd(self.M, self.d, self.h, self.x, self.W1, None, None, None, self.state, self.post, None,
+                         self.partial_amax, None, None, A.FWD_CALIBRATE, self.stream)
+        self.update_scale()
+
+    def forward(self, eval_bf16: bool = False, pre_debug=None):
+        flags = A.FWD_EVAL_BF16 if eval_bf16 else 0
+        A.fp8mlp_mlp_fwd(self.M, self.d, self.h, self.x, self.W1, self.W2q_t, self.w2_scale_inv, self.W2,
+                         self.state, self.post, None if eval_bf16 else self.post_fp8, self.partial_amax, self.out,
+                         pre_debug, flags, self.stream)
+
+    def update_scale(self):
+        A.fp8mlp_amax_reduce_update_scale(self.partial_amax, self.partial_amax.numel(), self.state, self.stream)
+
+    def backward(self):
+        A.fp8mlp_mlp_bwd(self.M, self.d, self.h, self.x, self.W1, self.W2, self.post, self.dOut, self.dPre,
+                         self.dX, self.dW1, self.dW2, self.stream)
+
+    def train_step(self):
+        """forward at s_t, backward, s_{t+1}; the caller's optimizer then
+        updates W1/W2 and calls refresh_w2_cache()."""
+        self.forward()
+        self.backward()
+        self.update_scale()
+
+    # --------------------------------------------------------------- helpers
+    def read_state(self) -> dict:
+        s = self.state.cpu()
+        i = s.view(torch.int32)
+        return dict(amax_prev=float(s[0]), scale=float(s[1]), scale_inv=float(s[2]), margin=float(s[3]),
+                    step=int(i[4]), flags=int(i[5]))
+
+    @staticmethod
+    def bits_to_bf16(a, device):
+        """numpy uint16 BF16 bit patterns -> torch bf16 device tensor."""
+        import numpy as np
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)

@@ -1,0 +1,523 @@
+// C-ABI entry points: argument checks on the host, tensor-map encoding, and
+// the launches.  See include/fp8mlp.h for the contract of each call.
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "internal.h"
+
+#define FP8MLP_VERSION_STRING "fp8mlp 0.1.0 (sm_100a)"
+
+namespace fp8mlp {
+namespace {
+
+thread_local std::string g_detail;
+std::atomic<unsigned long long> g_launches{0};
+std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
+std::atomic<int> g_debug_flags{0};
+
+int fail(int code, const std::string& what) {
+  g_detail = what;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  g_detail = std::string(where) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
+  return FP8MLP_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define REQUIRE_PTR(p)                                                                     \
+  do {                                                                                     \
+    if ((p) == nullptr) return fail(FP8MLP_ERR_INVALID_ARG, #p " is NULL");                \
+    if (!aligned16(p)) return fail(FP8MLP_ERR_INVALID_ARG, #p " is not 16-byte aligned"); \
+  } while (0)
+
+int check_dims(int M, int d, int h) {
+  if (M < 0) return fail(FP8MLP_ERR_INVALID_ARG, "M < 0");
+  if (d < 16 || h < 16) return fail(FP8MLP_ERR_UNSUPPORTED_SHAPE, "d and h must be >= 16");
+  if (d % 16 != 0 || h % 16 != 0) return fail(FP8MLP_ERR_UNSUPPORTED_SHAPE, "d and h must be multiples of 16");
+  return FP8MLP_OK;
+}
+
+// ---- device info --------------------------------------------------------
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+bool g_dev_ok[kMaxDevices] = {};
+
+// ---- tensor maps ---------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D row-major tensor [outer, inner] of `esize`-byte elements, dense rows.
+int map2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t inner, uint64_t outer,
+          uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz, const char* what) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(FP8MLP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * static_cast<uint64_t>(esize)};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[160];
+    snprintf(buf, sizeof(buf), "tensor map for %s failed (CUresult %d)", what, static_cast<int>(r));
+    return fail(FP8MLP_ERR_CUDA, buf);
+  }
+  return FP8MLP_OK;
+}
+
+constexpr CUtensorMapDataType BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+constexpr CUtensorMapDataType U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+constexpr CUtensorMapDataType F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+constexpr CUtensorMapSwizzle SW128 = CU_TENSOR_MAP_SWIZZLE_128B;
+constexpr CUtensorMapSwizzle SW64 = CU_TENSOR_MAP_SWIZZLE_64B;
+constexpr CUtensorMapSwizzle SW32 = CU_TENSOR_MAP_SWIZZLE_32B;
+
+// operand maps: K-major [rows, K] or MN-major [K, cols]
+int map_kmajor(CUtensorMap* m, const void* p, CUtensorMapDataType dt, int esize, int rows, int K, int box_rows,
+               const char* what) {
+  return map2d(m, p, dt, esize, K, rows, 128 / esize, box_rows, SW128, what);
+}
+int map_mnmajor(CUtensorMap* m, const void* p, int K, int cols, const char* what) {
+  return map2d(m, p, BF16, 2, cols, K, 64, 64, SW128, what);
+}
+// 32x32 output/aux tiles of an [rows, cols] tensor
+int map_tile32(CUtensorMap* m, const void* p, CUtensorMapDataType dt, int esize, int rows, int cols,
+               const char* what) {
+  const CUtensorMapSwizzle swz = esize == 4 ? SW128 : (esize == 2 ? SW64 : SW32);
+  return map2d(m, p, dt, esize, cols, rows, 32, 32, swz, what);
+}
+
+#define TRY(x)                           \
+  do {                                   \
+    const int rc_ = (x);                 \
+    if (rc_ != FP8MLP_OK) return rc_;    \
+  } while (0)
+
+int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+void fill_common(GemmParams& p, const DeviceInfo* di, int M, int N, int K, int groups) {
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.tiles_m = cdiv(M, kGemmBM);
+  p.tiles_n = cdiv(N, kGemmBN);
+  p.num_groups = groups;
+  p.status = di->status;
+  p.timeout_ns = g_timeout_ns.load();
+  p.debug_flags = g_debug_flags.load();
+}
+
+int launch(GemmKind k, const GemmParams& p, const DeviceInfo* di, cudaStream_t s, const char* what) {
+  const cudaError_t e = launch_gemm(k, p, p.tiles_m * p.tiles_n * p.num_groups, di->num_sms, s);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return FP8MLP_OK;
+}
+
+}  // namespace
+
+void count_launches(unsigned long long n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+int current_device(DeviceInfo** info) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(FP8MLP_ERR_NO_DEVICE, std::string("no CUDA device: ") + cudaGetErrorString(e));
+  }
+  if (dev < 0 || dev >= kMaxDevices) return fail(FP8MLP_ERR_NO_DEVICE, "device index out of range");
+  if (!g_dev_ok[dev]) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(FP8MLP_ERR_NO_DEVICE, "cannot query the current device");
+    }
+    if (major != 10 || minor != 0) {
+      char buf[96];
+      snprintf(buf, sizeof(buf), "device %d has compute capability %d.%d; sm_100a (10.0) is required", dev, major,
+               minor);
+      return fail(FP8MLP_ERR_NO_DEVICE, buf);
+    }
+    unsigned int* st = nullptr;
+    e = status_word_address(&st);
+    if (e != cudaSuccess) return cuda_fail(e, "status word");
+    g_dev[dev].device = dev;
+    g_dev[dev].num_sms = sms;
+    g_dev[dev].status = st;
+    g_dev_ok[dev] = true;
+  }
+  *info = &g_dev[dev];
+  return FP8MLP_OK;
+}
+
+}  // namespace fp8mlp
+
+using namespace fp8mlp;
+
+extern "C" {
+
+int fp8mlp_partial_amax_shape(int M, int h, int* row_blocks, int* col_blocks, int* block_rows, int* block_cols) {
+  if (M < 0 || h < 0) return fail(FP8MLP_ERR_INVALID_ARG, "negative size");
+  if (row_blocks) *row_blocks = 4 * cdiv(M, kGemmBM);
+  if (col_blocks) *col_blocks = cdiv(h, kGemmBN);
+  if (block_rows) *block_rows = kGemmBM / 4;
+  if (block_cols) *block_cols = kGemmBN;
+  return FP8MLP_OK;
+}
+
+size_t fp8mlp_workspace_size(int M, int d, int h) {
+  (void)M;
+  (void)d;
+  (void)h;
+  return 256;
+}
+
+int fp8mlp_up_proj_fused(int M, int d, int h, const uint16_t* x, const uint16_t* W1, const fp8mlp_scale_state* st,
+                         uint16_t* post, uint8_t* post_fp8, float* partial_amax, float* pre_debug, int flags,
+                         fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, d, h));
+  if (flags & ~(FP8MLP_FWD_EVAL_BF16 | FP8MLP_FWD_CALIBRATE)) return fail(FP8MLP_ERR_INVALID_ARG, "unknown flags");
+  const bool write_q = (flags & (FP8MLP_FWD_EVAL_BF16 | FP8MLP_FWD_CALIBRATE)) == 0;
+  if (M == 0) return FP8MLP_OK;
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(W1);
+  REQUIRE_PTR(post);
+  if (partial_amax == nullptr) return fail(FP8MLP_ERR_INVALID_ARG, "partial_amax is NULL");
+  if (reinterpret_cast<uintptr_t>(partial_amax) & 3u) return fail(FP8MLP_ERR_INVALID_ARG, "partial_amax misaligned");
+  if (write_q) {
+    REQUIRE_PTR(post_fp8);
+    REQUIRE_PTR(st);
+  }
+  if (pre_debug != nullptr && (reinterpret_cast<uintptr_t>(pre_debug) & 3u))
+    return fail(FP8MLP_ERR_INVALID_ARG, "pre_debug misaligned");
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  GemmParams p{};
+  TRY(map_kmajor(&p.tmA[0], x, BF16, 2, M, d, kGemmBM, "x"));
+  TRY(map_kmajor(&p.tmB[0], W1, BF16, 2, h, d, kGemmBN, "W1"));
+  TRY(map_tile32(&p.tmOut[0], post, BF16, 2, M, h, "post"));
+  if (write_q) TRY(map_tile32(&p.tmOut2, post_fp8, U8, 1, M, h, "post_fp8"));
+  fill_common(p, di, M, h, d, 1);
+  p.write_q = write_q ? 1 : 0;
+  p.partial_amax = partial_amax;
+  p.pre_debug = pre_debug;
+  p.st = st;
+  return launch(GemmKind::Up, p, di, stream, "up_proj_fused launch");
+}
+
+int fp8mlp_down_proj_fp8(int M, int d, int h, const uint8_t* post_fp8, const uint8_t* W2q_t,
+                         const float* w2_scale_inv, const fp8mlp_scale_state* st, uint16_t* out,
+                         fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, d, h));
+  if (M == 0) return FP8MLP_OK;
+  REQUIRE_PTR(post_fp8);
+  REQUIRE_PTR(W2q_t);
+  REQUIRE_PTR(out);
+  REQUIRE_PTR(st);
+  if (w2_scale_inv == nullptr) return fail(FP8MLP_ERR_INVALID_ARG, "w2_scale_inv is NULL");
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  GemmParams p{};
+  TRY(map_kmajor(&p.tmA[0], post_fp8, U8, 1, M, h, kGemmBM, "post_fp8"));
+  TRY(map_kmajor(&p.tmB[0], W2q_t, U8, 1, d, h, kGemmBN, "W2q_t"));
+  TRY(map_tile32(&p.tmOut[0], out, BF16, 2, M, d, "out"));
+  fill_common(p, di, M, d, h, 1);
+  p.st = st;
+  p.w2_scale_inv = w2_scale_inv;
+  return launch(GemmKind::Down8, p, di, stream, "down_proj_fp8 launch");
+}
+
+int fp8mlp_down_proj_bf16(int M, int d, int h, const uint16_t* post, const uint16_t* W2, uint16_t* out,
+                          fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, d, h));
+  if (M == 0) return FP8MLP_OK;
+  REQUIRE_PTR(post);
+  REQUIRE_PTR(W2);
+  REQUIRE_PTR(out);
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  GemmParams p{};
+  TRY(map_kmajor(&p.tmA[0], post, BF16, 2, M, h, kGemmBM, "post"));
+  TRY(map_mnmajor(&p.tmB[0], W2, h, d, "W2"));
+  TRY(map_tile32(&p.tmOut[0], out, BF16, 2, M, d, "out"));
+  fill_common(p, di, M, d, h, 1);
+  return launch(GemmKind::Bf16MnB, p, di, stream, "down_proj_bf16 launch");
+}
+
+int fp8mlp_mlp_fwd(int M, int d, int h, const uint16_t* x, const uint16_t* W1, const uint8_t* W2q_t,
+                   const float* w2_scale_inv, const uint16_t* W2, const fp8mlp_scale_state* st, uint16_t* post,
+                   uint8_t* post_fp8, float* partial_amax, uint16_t* out, float* pre_debug, int flags,
+                   fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, d, h));
+  if ((flags & FP8MLP_FWD_EVAL_BF16) && (flags & FP8MLP_FWD_CALIBRATE))
+    return fail(FP8MLP_ERR_INVALID_ARG, "EVAL_BF16 and CALIBRATE are exclusive");
+  if (M == 0) return FP8MLP_OK;
+  // check the down-projection's arguments before anything is enqueued
+  if (flags & FP8MLP_FWD_EVAL_BF16) {
+    REQUIRE_PTR(W2);
+    REQUIRE_PTR(out);
+  } else if (!(flags & FP8MLP_FWD_CALIBRATE)) {
+    REQUIRE_PTR(W2q_t);
+    REQUIRE_PTR(out);
+    if (w2_scale_inv == nullptr) return fail(FP8MLP_ERR_INVALID_ARG, "w2_scale_inv is NULL");
+  }
+  TRY(fp8mlp_up_proj_fused(M, d, h, x, W1, st, post, post_fp8, partial_amax, pre_debug, flags, stream));
+  if (flags & FP8MLP_FWD_CALIBRATE) return FP8MLP_OK;
+  if (flags & FP8MLP_FWD_EVAL_BF16) return fp8mlp_down_proj_bf16(M, d, h, post, W2, out, stream);
+  return fp8mlp_down_proj_fp8(M, d, h, post_fp8, W2q_t, w2_scale_inv, st, out, stream);
+}
+
+int fp8mlp_scale_state_init(fp8mlp_scale_state* st, float margin, float initial_scale, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  REQUIRE_PTR(st);
+  if (!(margin > 0.f) || !std::isfinite(margin)) return fail(FP8MLP_ERR_INVALID_ARG, "margin must be finite and > 0");
+  if (!(initial_scale > 0.f) || !std::isfinite(initial_scale))
+    return fail(FP8MLP_ERR_INVALID_ARG, "initial_scale must be finite and > 0");
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  const cudaError_t e = launch_state_init(st, margin, initial_scale, stream);
+  return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "scale_state_init launch");
+}
+
+int fp8mlp_amax_reduce_update_scale(const float* partial_amax, int n, fp8mlp_scale_state* st,
+                                    fp8mlp_stream_t stream) {
+  g_detail.clear();
+  if (n < 0) return fail(FP8MLP_ERR_INVALID_ARG, "n < 0");
+  REQUIRE_PTR(st);
+  if (n > 0 && partial_amax == nullptr) return fail(FP8MLP_ERR_INVALID_ARG, "partial_amax is NULL");
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  const cudaError_t e = launch_amax_scale(partial_amax, n, st, di->status, stream);
+  return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "amax_reduce_update_scale launch");
+}
+
+int fp8mlp_w2_fp8_cache_refresh(int h, int d, const uint16_t* W2, uint8_t* W2q_t, float* w2_scale_inv,
+                                void* workspace, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(0, d, h));
+  REQUIRE_PTR(W2);
+  REQUIRE_PTR(W2q_t);
+  REQUIRE_PTR(workspace);
+  if (w2_scale_inv == nullptr) return fail(FP8MLP_ERR_INVALID_ARG, "w2_scale_inv is NULL");
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  const cudaError_t e = launch_w2_cache(h, d, W2, W2q_t, w2_scale_inv, static_cast<unsigned int*>(workspace),
+                                        di->status, di->num_sms, stream);
+  return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "w2_fp8_cache_refresh launch");
+}
+
+int fp8mlp_bwd_dpre(int M, int d, int h, const uint16_t* dOut, const uint16_t* W2, const uint16_t* post,
+                    uint16_t* dPre, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, d, h));
+  if (M == 0) return FP8MLP_OK;
+  REQUIRE_PTR(dOut);
+  REQUIRE_PTR(W2);
+  REQUIRE_PTR(post);
+  REQUIRE_PTR(dPre);
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  GemmParams p{};
+  TRY(map_kmajor(&p.tmA[0], dOut, BF16, 2, M, d, kGemmBM, "dOut"));
+  TRY(map_kmajor(&p.tmB[0], W2, BF16, 2, h, d, kGemmBN, "W2"));
+  TRY(map_tile32(&p.tmOut[0], dPre, BF16, 2, M, h, "dPre"));
+  TRY(map_tile32(&p.tmAux, post, BF16, 2, M, h, "post"));
+  fill_common(p, di, M, h, d, 1);
+  return launch(GemmKind::DPre, p, di, stream, "bwd_dpre launch");
+}
+
+int fp8mlp_bwd_dx(int M, int d, int h, const uint16_t* dPre, const uint16_t* W1, uint16_t* dX,
+                  fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, d, h));
+  if (M == 0) return FP8MLP_OK;
+  REQUIRE_PTR(dPre);
+  REQUIRE_PTR(W1);
+  REQUIRE_PTR(dX);
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  GemmParams p{};
+  TRY(map_kmajor(&p.tmA[0], dPre, BF16, 2, M, h, kGemmBM, "dPre"));
+  TRY(map_mnmajor(&p.tmB[0], W1, h, d, "W1"));
+  TRY(map_tile32(&p.tmOut[0], dX, BF16, 2, M, d, "dX"));
+  fill_common(p, di, M, d, h, 1);
+  return launch(GemmKind::Bf16MnB, p, di, stream, "bwd_dx launch");
+}
+
+int fp8mlp_bwd_dw(int M, int d, int h, const uint16_t* x, const uint16_t* dPre, const uint16_t* post,
+                  const uint16_t* dOut, float* dW1, float* dW2, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, d, h));
+  REQUIRE_PTR(dW1);
+  REQUIRE_PTR(dW2);
+  if (M == 0) {
+    // an empty batch contributes zero gradient
+    DeviceInfo* di = nullptr;
+    TRY(current_device(&di));
+    cudaError_t e = cudaMemsetAsync(dW1, 0, sizeof(float) * h * d, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dW2, 0, sizeof(float) * h * d, stream);
+    return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "bwd_dw memset");
+  }
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(dPre);
+  REQUIRE_PTR(post);
+  REQUIRE_PTR(dOut);
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  GemmParams p{};
+  // group 0: dW1[i,j] = sum_m dPre[m,i] x[m,j];  group 1: dW2[i,j] = sum_m post[m,i] dOut[m,j]
+  TRY(map_mnmajor(&p.tmA[0], dPre, M, h, "dPre"));
+  TRY(map_mnmajor(&p.tmB[0], x, M, d, "x"));
+  TRY(map_tile32(&p.tmOut[0], dW1, F32, 4, h, d, "dW1"));
+  TRY(map_mnmajor(&p.tmA[1], post, M, h, "post"));
+  TRY(map_mnmajor(&p.tmB[1], dOut, M, d, "dOut"));
+  TRY(map_tile32(&p.tmOut[1], dW2, F32, 4, h, d, "dW2"));
+  fill_common(p, di, h, d, M, 2);
+  return launch(GemmKind::DW, p, di, stream, "bwd_dw launch");
+}
+
+int fp8mlp_mlp_bwd(int M, int d, int h, const uint16_t* x, const uint16_t* W1, const uint16_t* W2,
+                   const uint16_t* post, const uint16_t* dOut, uint16_t* dPre, uint16_t* dX, float* dW1,
+                   float* dW2, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, d, h));
+  if (M > 0) {
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(W1);
+    REQUIRE_PTR(W2);
+    REQUIRE_PTR(post);
+    REQUIRE_PTR(dOut);
+    REQUIRE_PTR(dPre);
+    REQUIRE_PTR(dX);
+  }
+  REQUIRE_PTR(dW1);
+  REQUIRE_PTR(dW2);
+  TRY(fp8mlp_bwd_dpre(M, d, h, dOut, W2, post, dPre, stream));
+  TRY(fp8mlp_bwd_dx(M, d, h, dPre, W1, dX, stream));
+  return fp8mlp_bwd_dw(M, d, h, x, dPre, post, dOut, dW1, dW2, stream);
+}
+
+int fp8mlp_rmsnorm_fwd(int M, int d, const uint16_t* r, uint16_t* x, float* rstd, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, d, 16));
+  if (M == 0) return FP8MLP_OK;
+  REQUIRE_PTR(r);
+  REQUIRE_PTR(x);
+  if (rstd == nullptr || (reinterpret_cast<uintptr_t>(rstd) & 3u)) return fail(FP8MLP_ERR_INVALID_ARG, "rstd");
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  const cudaError_t e = launch_rmsnorm_fwd(M, d, r, x, rstd, di->num_sms, stream);
+  return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "rmsnorm_fwd launch");
+}
+
+int fp8mlp_rmsnorm_bwd(int M, int d, const uint16_t* r, const float* rstd, const uint16_t* dx,
+                       const uint16_t* dr_in, uint16_t* dr_out, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, d, 16));
+  if (M == 0) return FP8MLP_OK;
+  REQUIRE_PTR(r);
+  REQUIRE_PTR(dx);
+  REQUIRE_PTR(dr_in);
+  REQUIRE_PTR(dr_out);
+  if (rstd == nullptr || (reinterpret_cast<uintptr_t>(rstd) & 3u)) return fail(FP8MLP_ERR_INVALID_ARG, "rstd");
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  const cudaError_t e = launch_rmsnorm_bwd(M, d, r, rstd, dx, dr_in, dr_out, di->num_sms, stream);
+  return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "rmsnorm_bwd launch");
+}
+
+int fp8mlp_residual_add(int M, int d, const uint16_t* r, const uint16_t* out, uint16_t* r_next,
+                        fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, d, 16));
+  if (M == 0) return FP8MLP_OK;
+  REQUIRE_PTR(r);
+  REQUIRE_PTR(out);
+  REQUIRE_PTR(r_next);
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  const cudaError_t e = launch_residual_add(M, d, r, out, r_next, di->num_sms, stream);
+  return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "residual_add launch");
+}
+
+int fp8mlp_get_device_status(unsigned int* status, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  if (status == nullptr) return fail(FP8MLP_ERR_INVALID_ARG, "status is NULL");
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  cudaError_t e = cudaMemcpyAsync(status, di->status, sizeof(unsigned int), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "get_device_status");
+}
+
+int fp8mlp_clear_device_status(fp8mlp_stream_t stream) {
+  g_detail.clear();
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  const cudaError_t e = cudaMemsetAsync(di->status, 0, sizeof(unsigned int), stream);
+  return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "clear_device_status");
+}
+
+int fp8mlp_set_wait_timeout_ns(unsigned long long ns) {
+  if (ns == 0) return fail(FP8MLP_ERR_INVALID_ARG, "timeout must be > 0");
+  g_timeout_ns.store(ns);
+  return FP8MLP_OK;
+}
+
+int fp8mlp_set_debug_flags(int flags) {
+  if (flags & ~FP8MLP_DEBUG_STALL_PRODUCER) return fail(FP8MLP_ERR_INVALID_ARG, "unknown debug flags");
+  g_debug_flags.store(flags);
+  return FP8MLP_OK;
+}
+
+const char* fp8mlp_error_string(int code) {
+  switch (code) {
+    case FP8MLP_OK:
+      return "ok";
+    case FP8MLP_ERR_INVALID_ARG:
+      return "invalid argument";
+    case FP8MLP_ERR_UNSUPPORTED_SHAPE:
+      return "unsupported shape";
+    case FP8MLP_ERR_CUDA:
+      return "CUDA error";
+    case FP8MLP_ERR_TIMEOUT:
+      return "device wait timed out";
+    case FP8MLP_ERR_NO_DEVICE:
+      return "no sm_100a device";
+    default:
+      return "unknown error code";
+  }
+}
+
+const char* fp8mlp_last_error_detail(void) { return g_detail.c_str(); }
+
+const char* fp8mlp_version(void) { return FP8MLP_VERSION_STRING; }
+
+unsigned long long fp8mlp_kernel_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,427 @@
+// Warp-specialised, persistent tcgen05 GEMM with fused epilogues.
+//
+//   D[m, n] = sum_k A[m, k] * B[n, k]      (fp32 accumulate in TMEM)
+//
+// One CTA per SM (192 threads):
+//   warp 0      TMA producer: streams A/B k-blocks into a STAGES-deep smem ring
+//   warp 1      allocates 512 TMEM columns (two 256-column accumulators) and
+//               issues the UMMAs from one thread
+//   warps 2..5  epilogue: TMEM -> registers -> fused math -> swizzled smem ->
+//               TMA store, 32 columns at a time; warp w owns TMEM lanes
+//               32*(w%4) .. +31, i.e. tile rows 32*(w%4) .. +31
+// The two accumulators let the epilogue of tile i overlap the mainloop of
+// tile i+1.  Operands are BF16 (kind::f16) or e4m3 (kind::f8f6f4), each
+// K-major or MN-major, staged with 128-byte swizzle.  TMA zero-fills rows and
+// columns past the tensor edges and clips stores, so any M, N, K work.
+#pragma once
+
+#include "fp8mlp.h"
+#include "sm100.cuh"
+
+namespace fp8mlp {
+
+enum class Epi : int {
+  UpFused = 0,     // post = bf16(relu(acc)^2), q = e4m3(post*s), partial amax
+  DownScaled = 1,  // out = bf16(acc * s^-1 * s_w^-1)
+  StoreBf16 = 2,   // out = bf16(acc)
+  DPre = 3,        // dPre = bf16(2 sqrt(post) * acc), post read by TMA
+  StoreF32 = 4,    // out = acc (fp32)
+};
+
+struct alignas(64) GemmParams {
+  CUtensorMap tmA[2];
+  CUtensorMap tmB[2];
+  CUtensorMap tmOut[2];
+  CUtensorMap tmOut2;  // UpFused: post_fp8
+  CUtensorMap tmAux;   // DPre: post
+  int M, N, K;
+  int tiles_m, tiles_n;
+  int num_groups;
+  int write_q;
+  int pad0;
+  float* partial_amax;
+  float* pre_debug;
+  const fp8mlp_scale_state* st;
+  const float* w2_scale_inv;
+  unsigned int* status;
+  unsigned long long timeout_ns;
+  int debug_flags;
+};
+
+template <int BN_, int STAGES_, bool FP8_, bool A_MN_, bool B_MN_, Epi EPI_>
+struct GemmCfg {
+  static constexpr int BM = 128;
+  static constexpr int BN = BN_;
+  static constexpr int STAGES = STAGES_;
+  static constexpr bool FP8 = FP8_;
+  static constexpr bool A_MN = A_MN_;
+  static constexpr bool B_MN = B_MN_;
+  static constexpr Epi EPI = EPI_;
+  static_assert(!(FP8 && (A_MN || B_MN)), "MN-major operands are BF16 only here");
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
+  static constexpr int ELEM = FP8 ? 1 : 2;
+  static constexpr int BK = 128 / ELEM;     // K elements per stage (one 128-byte swizzle row)
+  static constexpr int UMMA_K = 32 / ELEM;  // K per UMMA instruction (32 bytes)
+  static constexpr int A_BYTES = BM * BK * ELEM;
+  static constexpr int B_BYTES = BN * BK * ELEM;
+  // descriptor strides: K-major: 8-row groups 1024 B apart (LBO unused);
+  // MN-major: 64-element MN atoms BK*128 B apart (LBO), 8-k-row groups 1024 B apart
+  static constexpr uint32_t A_LBO = A_MN ? BK * 128 : 16;
+  static constexpr uint32_t B_LBO = B_MN ? BK * 128 : 16;
+  static constexpr uint32_t SBO = 1024;
+  static constexpr uint32_t A_KSTEP = A_MN ? UMMA_K * 128 : UMMA_K * ELEM;
+  static constexpr uint32_t B_KSTEP = B_MN ? UMMA_K * 128 : UMMA_K * ELEM;
+  static constexpr uint32_t IDESC =
+      dev::instr_desc(FP8 ? dev::FMT_E4M3 : dev::FMT_BF16, FP8 ? dev::FMT_E4M3 : dev::FMT_BF16, A_MN, B_MN, BM, BN);
+  static constexpr int ECOLS = 32;
+  static constexpr int NCHUNK = BN / ECOLS;
+  static constexpr int OUT_BUF = 32 * ECOLS * (EPI == Epi::StoreF32 ? 4 : 2);
+  static constexpr int OUT2_BUF = EPI == Epi::UpFused ? 32 * ECOLS : 0;
+  static constexpr int AUX_BUF = EPI == Epi::DPre ? 32 * ECOLS * 2 : 0;
+  static constexpr int SLOT = OUT_BUF + OUT2_BUF + AUX_BUF;  // multiple of 1024
+  static_assert(SLOT % 1024 == 0, "slot alignment");
+  static constexpr int TMEM_COLS = 512;
+  static_assert(2 * BN <= TMEM_COLS, "two accumulators");
+  static constexpr int NUM_BARS = 2 * STAGES + 4 + 8 + 1;
+  static constexpr int SMEM_BYTES =
+      1024 /*alignment slack*/ + STAGES * (A_BYTES + B_BYTES) + 8 * SLOT + NUM_BARS * 8 + 16;
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+namespace dev {
+
+// Bounded wait that ignores the abort flag (used to drain in-flight copies).
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return;
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > limit_ns) return;
+  }
+}
+
+template <int ROWB>
+__device__ __forceinline__ void store_row_bf16(uint32_t base, int lane, const uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    st_shared_v4(base + swz<3>(lane * 64 + j * 16), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+}
+
+}  // namespace dev
+
+template <class C>
+__global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constant__ GemmParams p) {
+  using namespace dev;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + C::STAGES * C::A_BYTES;
+  uint8_t* sEpi = sB + C::STAGES * C::B_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + 8 * C::SLOT);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::STAGES;
+  uint64_t* tfull = bars + 2 * C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* auxb = tempty + 2;  // [4 warps][2 slots]
+  uint64_t* fin = auxb + 8;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(fin + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    for (int i = 0; i < 8; ++i) mbar_init(&auxb[i], 1);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const WaitCtx w{p.status, abort_flag, p.timeout_ns};
+
+  const int tiles_per_group = p.tiles_m * p.tiles_n;
+  const int num_tiles = tiles_per_group * p.num_groups;
+  const int num_kb = (p.K + C::BK - 1) / C::BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && !(p.debug_flags & FP8MLP_DEBUG_STALL_PRODUCER)) {
+      for (int g = 0; g < p.num_groups; ++g) {
+        tma_prefetch_desc(&p.tmA[g]);
+        tma_prefetch_desc(&p.tmB[g]);
+      }
+      uint32_t stage = 0, phase = 0;
+      long long issued = 0;
+      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+        const int g = t / tiles_per_group;
+        const int tt = t - g * tiles_per_group;
+        const int m0 = (tt / p.tiles_n) * C::BM;
+        const int n0 = (tt % p.tiles_n) * C::BN;
+        const CUtensorMap* mA = &p.tmA[g];
+        const CUtensorMap* mB = &p.tmB[g];
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, w)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES);
+          uint8_t* a = sA + stage * C::A_BYTES;
+          uint8_t* b = sB + stage * C::B_BYTES;
+          const int k0 = kb * C::BK;
+          if constexpr (C::A_MN) {
+#pragma unroll
+            for (int i = 0; i < C::BM / 64; ++i) tma_load_2d(a + i * C::BK * 128, mA, &full[stage], m0 + i * 64, k0);
+          } else {
+            tma_load_2d(a, mA, &full[stage], k0, m0);
+          }
+          if constexpr (C::B_MN) {
+#pragma unroll
+            for (int i = 0; i < C::BN / 64; ++i) tma_load_2d(b + i * C::BK * 128, mB, &full[stage], n0 + i * 64, k0);
+          } else {
+            tma_load_2d(b, mB, &full[stage], k0, n0);
+          }
+          ++issued;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      // drain: the last issue into each stage must have landed before exit
+      const long long n_drain = issued < C::STAGES ? issued : C::STAGES;
+      for (long long i = 0; i < n_drain; ++i) {
+        const long long n = issued - 1 - i;
+        mbar_wait_drain(&full[n % C::STAGES], static_cast<uint32_t>((n / C::STAGES) & 1), p.timeout_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, w)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * C::BN;
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, w)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < C::BK / C::UMMA_K; ++k) {
+            const uint64_t ad = smem_desc(a0 + k * C::A_KSTEP, C::A_LBO, C::SBO);
+            const uint64_t bd = smem_desc(b0 + k * C::B_KSTEP, C::B_LBO, C::SBO);
+            const uint32_t accum = (kb | k) != 0;
+            if constexpr (C::FP8)
+              umma_f8(d_tmem, ad, bd, C::IDESC, accum);
+            else
+              umma_f16(d_tmem, ad, bd, C::IDESC, accum);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      // every UMMA this thread issued must be complete before TMEM is freed
+      tc_commit(fin);
+      mbar_wait_drain(fin, 0, p.timeout_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter == row block of 32 within the tile
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    uint32_t acc = 0, acc_phase = 0, ctr = 0;
+    float s_up = 0.f, comb = 1.f;
+    if constexpr (C::EPI == Epi::UpFused) {
+      if (p.write_q) s_up = p.st->scale;
+    }
+    if constexpr (C::EPI == Epi::DownScaled) comb = __fmul_rn(p.st->scale_inv, *p.w2_scale_inv);
+    uint32_t aux_issued[2] = {0u, 0u};  // post loads issued into each of this warp's two slots
+
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      const int g = t / tiles_per_group;
+      const int tt = t - g * tiles_per_group;
+      const int mb = tt / p.tiles_n, nb = tt % p.tiles_n;
+      const int m0 = mb * C::BM, n0 = nb * C::BN;
+      const int row0 = m0 + q * 32;
+
+      if constexpr (C::EPI == Epi::DPre) {
+        // prefetch the post chunk of column block 0 while the mainloop runs
+        const uint32_t b = ctr & 1u;
+        if (lane == 0) {
+          uint64_t* bar = &auxb[q * 2 + b];
+          mbar_arrive_expect_tx(bar, C::AUX_BUF);
+          tma_load_2d(sEpi + (q * 2 + b) * C::SLOT + C::OUT_BUF, &p.tmAux, bar, n0, row0);
+        }
+        ++aux_issued[b];
+      }
+
+      if (!mbar_wait(&tfull[acc], acc_phase, w)) break;
+      tc_fence_after();
+      float tmax = 0.f;
+      bool ok = true;
+#pragma unroll 1
+      for (int c = 0; c < C::NCHUNK; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem_base + lane_base + acc * C::BN + c * C::ECOLS, v);
+        if (c == C::NCHUNK - 1) {
+          tc_fence_before();
+          mbar_arrive(&tempty[acc]);
+        }
+        const uint32_t b = ctr & 1u;
+        uint8_t* slot = sEpi + (q * 2 + b) * C::SLOT;
+        const uint32_t sbase = smem_u32(slot);
+        if (lane == 0) bulk_wait_read<1>();  // the store issued from this slot two chunks ago has read it
+        __syncwarp();
+        const int col0 = n0 + c * C::ECOLS;
+
+        if constexpr (C::EPI == Epi::UpFused) {
+          uint32_t pk[16], qk[8];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a = fmaxf(__uint_as_float(v[2 * i]), 0.f);
+            const float bb = fmaxf(__uint_as_float(v[2 * i + 1]), 0.f);
+            const float sa = __fmul_rn(a, a), sb = __fmul_rn(bb, bb);
+            tmax = fmaxf(tmax, fmaxf(sa, sb));
+            pk[i] = pack_bf16x2(sa, sb);
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t q0 = pack_e4m3x2(__fmul_rn(bf16lo_to_f32(pk[2 * i]), s_up),
+                                            __fmul_rn(bf16hi_to_f32(pk[2 * i]), s_up));
+            const uint32_t q1 = pack_e4m3x2(__fmul_rn(bf16lo_to_f32(pk[2 * i + 1]), s_up),
+                                            __fmul_rn(bf16hi_to_f32(pk[2 * i + 1]), s_up));
+            qk[i] = q0 | (q1 << 16);
+          }
+          store_row_bf16<64>(sbase, lane, pk);
+          if (p.write_q) {
+            const uint32_t qb = sbase + C::OUT_BUF;
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              st_shared_v4(qb + swz<1>(lane * 32 + j * 16), qk[4 * j], qk[4 * j + 1], qk[4 * j + 2], qk[4 * j + 3]);
+          }
+          if (p.pre_debug != nullptr) {
+            const int m = row0 + lane;
+            if (m < p.M) {
+              float* dst = p.pre_debug + static_cast<size_t>(m) * p.N;
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (col0 + i < p.N) dst[col0 + i] = __uint_as_float(v[i]);
+            }
+          }
+        } else if constexpr (C::EPI == Epi::DownScaled || C::EPI == Epi::StoreBf16) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float a = __uint_as_float(v[2 * i]), bb = __uint_as_float(v[2 * i + 1]);
+            if constexpr (C::EPI == Epi::DownScaled) {
+              a = __fmul_rn(a, comb);
+              bb = __fmul_rn(bb, comb);
+            }
+            pk[i] = pack_bf16x2(a, bb);
+          }
+          store_row_bf16<64>(sbase, lane, pk);
+        } else if constexpr (C::EPI == Epi::DPre) {
+          // prefetch the next column block's post before consuming this one
+          if (c + 1 < C::NCHUNK) {
+            const uint32_t nb2 = (ctr + 1) & 1u;
+            if (lane == 0) {
+              uint64_t* bar = &auxb[q * 2 + nb2];
+              mbar_arrive_expect_tx(bar, C::AUX_BUF);
+              tma_load_2d(sEpi + (q * 2 + nb2) * C::SLOT + C::OUT_BUF, &p.tmAux, bar, col0 + C::ECOLS, row0);
+            }
+            ++aux_issued[nb2];
+          }
+          if (!mbar_wait(&auxb[q * 2 + b], (ctr >> 1) & 1u, w)) {
+            ok = false;
+          } else {
+            const uint32_t ab = sbase + C::OUT_BUF;
+            uint32_t pp[16], pk[16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              ld_shared_v4(ab + swz<3>(lane * 64 + j * 16), pp[4 * j], pp[4 * j + 1], pp[4 * j + 2], pp[4 * j + 3]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float r0 = 2.f * __fsqrt_rn(bf16lo_to_f32(pp[i]));
+              const float r1 = 2.f * __fsqrt_rn(bf16hi_to_f32(pp[i]));
+              pk[i] = pack_bf16x2(__fmul_rn(r0, __uint_as_float(v[2 * i])), __fmul_rn(r1, __uint_as_float(v[2 * i + 1])));
+            }
+            store_row_bf16<64>(sbase, lane, pk);
+          }
+        } else {  // StoreF32
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(sbase + swz<7>(lane * 128 + j * 16), v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+        if (!ok) break;
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&p.tmOut[g], slot, col0, row0);
+          if constexpr (C::EPI == Epi::UpFused) {
+            if (p.write_q) tma_store_2d(&p.tmOut2, slot + C::OUT_BUF, col0, row0);
+          }
+          bulk_commit();
+        }
+        ++ctr;
+      }
+      if (!ok) break;
+      if constexpr (C::EPI == Epi::UpFused) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
+        if (lane == 0) p.partial_amax[(mb * 4 + q) * p.tiles_n + nb] = round_bf16(tmax);
+      }
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+    if (lane == 0) {
+      if constexpr (C::EPI == Epi::DPre) {
+        // the last load issued into each slot must have landed before exit
+        for (int b = 0; b < 2; ++b)
+          if (aux_issued[b] > 0) mbar_wait_drain(&auxb[q * 2 + b], (aux_issued[b] - 1u) & 1u, p.timeout_ns);
+      }
+      bulk_wait<0>();
+    }
+    __syncwarp();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fp8mlp

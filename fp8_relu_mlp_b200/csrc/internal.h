@@ -1,0 +1,52 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fp8mlp.h"
+#include "gemm_sm100.cuh"
+
+namespace fp8mlp {
+
+// GEMM variants (one template instantiation each)
+enum class GemmKind : int {
+  Up = 0,       // K1: x . W1^T -> post, post_fp8, partial amax (BF16, K-major A/B)
+  Down8 = 1,    // K2: q . W2q_t^T -> out (e4m3, K-major A/B)
+  Bf16MnB = 2,  // post . W2 (eval) and dPre . W1 (dX): BF16, K-major A, MN-major B
+  DPre = 3,     // K5: dOut . W2^T -> dPre with the 2 sqrt(post) epilogue
+  DW = 4,       // K7/K8: dPre^T . x and post^T . dOut (BF16, MN-major A/B), fp32 out
+};
+constexpr int kGemmBM = 128;
+constexpr int kGemmBN = 256;
+
+struct DeviceInfo {
+  int device = -1;
+  int num_sms = 0;
+  unsigned int* status = nullptr;  // device status word
+};
+
+// Checks that the current device is compute capability 10.0; fills `info`.
+int current_device(DeviceInfo** info);
+
+cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int num_tiles, int num_sms, cudaStream_t s);
+
+// small kernels
+cudaError_t launch_state_init(fp8mlp_scale_state* st, float margin, float s0, cudaStream_t s);
+cudaError_t launch_amax_scale(const float* pa, int n, fp8mlp_scale_state* st, unsigned int* status, cudaStream_t s);
+cudaError_t launch_w2_cache(int h, int d, const uint16_t* W2, uint8_t* W2q_t, float* w2_scale_inv,
+                            unsigned int* amax_word, unsigned int* status, int num_sms, cudaStream_t s);
+cudaError_t launch_rmsnorm_fwd(int M, int d, const uint16_t* r, uint16_t* x, float* rstd, int num_sms,
+                               cudaStream_t s);
+cudaError_t launch_rmsnorm_bwd(int M, int d, const uint16_t* r, const float* rstd, const uint16_t* dx,
+                               const uint16_t* dr_in, uint16_t* dr_out, int num_sms, cudaStream_t s);
+cudaError_t launch_residual_add(int M, int d, const uint16_t* r, const uint16_t* out, uint16_t* r_next,
+                                int num_sms, cudaStream_t s);
+
+// number of kernels this library has launched (all devices, all threads)
+void count_launches(unsigned long long n);
+
+// status word symbol address on the current device
+cudaError_t status_word_address(unsigned int** ptr);
+
+}  // namespace fp8mlp

@@ -1,0 +1,279 @@
+/*
+ * fp8mlp -- fused FP8 ReLU^2 MLP block for NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Plain pointers and sizes; no C++ or framework types.
+ *
+ * The block (one transformer MLP, d -> h -> d):
+ *     pre  = x . W1^T                       (never stored)
+ *     post = relu(pre)^2                    BF16, kept for the backward
+ *     q    = e4m3(post * s_t)               FP8 copy under the delayed scale s_t
+ *     out  = (q . W2q_t^T) * s_t^-1 * s_w^-1   FP8 down-projection
+ * and its BF16 backward, which rebuilds relu(pre) as sqrt(post).
+ *
+ * Sources (page title, section):
+ *   "NanoGPT Speedrun (Track 1)", section "Changes vs Record #83", item 4:
+ *       the MLP kernel stores only post = relu(pre)^2; the backward rebuilds
+ *       relu(pre) = sqrt(post) in-kernel.
+ *   same page, "From Unoptimized / Approach", item 5: FP8 e4m3 MLP GEMMs in
+ *       the training forward, BF16 backward, BF16 at evaluation.
+ *   "A Retrospective on Our World Records", Modded-NanoGPT Main Track: the
+ *       fused up-projection writes BF16 post, an FP8 copy and a tiny
+ *       partial-amax tensor while post sits in registers; the scale of step t
+ *       comes from amax(t-1) times a safety margin; a transposed FP8 cache of
+ *       W2 is refreshed after optimizer updates; the BF16 backward is left
+ *       unchanged.  Same page, "A few implementation notes": an exact,
+ *       non-delayed W2 refresh is viable.
+ *
+ * Layouts (all row-major, element strides implied by the sizes):
+ *   x [M,d] bf16      W1 [h,d] bf16 (nn.Linear(d,h).weight)   W2 [h,d] bf16
+ *   post [M,h] bf16   post_fp8 [M,h] e4m3   W2q_t [d,h] e4m3 (W2 transposed)
+ *   out [M,d] bf16    dOut [M,d] bf16   dPre [M,h] bf16   dX [M,d] bf16
+ *   dW1 [h,d] fp32    dW2 [h,d] fp32
+ * BF16 and e4m3 tensors are passed as raw bit patterns (uint16 / uint8).
+ *
+ * Conventions shared by every entry point:
+ *   - Ownership: the caller owns and allocates every buffer; the library
+ *     allocates no device memory and keeps no pointer after the call.
+ *   - Device pointers must be 16-byte aligned (TMA).  Tensors are dense.
+ *   - Shapes: M >= 0 is arbitrary (M = 0 is a no-op that returns FP8MLP_OK);
+ *     d and h must be multiples of 16 and at least 16.
+ *   - Asynchrony: every call enqueues work on `stream` (NULL = the legacy
+ *     default stream) of the current device and returns without waiting.
+ *     No call reads device data back to the host, except
+ *     fp8mlp_get_device_status.
+ *   - Errors: argument checks run on the host before any CUDA call and
+ *     return FP8MLP_ERR_INVALID_ARG / FP8MLP_ERR_UNSUPPORTED_SHAPE with
+ *     nothing enqueued.  FP8MLP_ERR_NO_DEVICE: the current device is not a
+ *     compute-capability 10.0 GPU (or there is none).  FP8MLP_ERR_CUDA: a
+ *     CUDA call failed (fp8mlp_last_error_detail() says which).  Faults
+ *     found on the device (a bounded wait that gave up) are reported through
+ *     the device status word, read with fp8mlp_get_device_status.
+ *     There is no CPU fallback.
+ */
+#ifndef FP8MLP_H
+#define FP8MLP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fp8mlp_stream_t; /* same type as cudaStream_t */
+
+/* return codes */
+#define FP8MLP_OK 0
+#define FP8MLP_ERR_INVALID_ARG 1
+#define FP8MLP_ERR_UNSUPPORTED_SHAPE 2
+#define FP8MLP_ERR_CUDA 3
+#define FP8MLP_ERR_TIMEOUT 4
+#define FP8MLP_ERR_NO_DEVICE 5
+
+/* device status word bits (fp8mlp_get_device_status) */
+#define FP8MLP_STATUS_TIMEOUT 1u          /* a kernel's bounded wait gave up */
+#define FP8MLP_STATUS_NONFINITE_AMAX 2u   /* amax was NaN/inf: scale kept */
+#define FP8MLP_STATUS_W2_DEGENERATE 4u    /* max|W2| was 0 or not finite: s_w = 1 */
+
+/* Largest finite e4m3 value; the delayed scale maps margin * amax onto it. */
+#define FP8MLP_E4M3_MAX 448.0f
+
+/*
+ * Delayed-scaling state, device-resident, caller-allocated (32 bytes,
+ * 16-byte aligned).  "A Retrospective on Our World Records", Main Track: the
+ * FP8 activation scale of step t is derived from the amax measured at step
+ * t-1 multiplied by a safety margin; no rolling window.
+ * The caller may copy it out and back in to checkpoint / resume.
+ */
+typedef struct fp8mlp_scale_state {
+  float amax_prev; /* A_{t-1}: amax of post reduced at the last update       */
+  float scale;     /* s_t = 448 / (margin * A_{t-1}), used to quantise post  */
+  float scale_inv; /* 1 / s_t (fp32, round-to-nearest)                       */
+  float margin;    /* safety margin (> 0)                                     */
+  int32_t step;    /* number of updates applied                              */
+  int32_t flags;   /* FP8MLP_STATE_KEPT_SCALE: last update kept the scale    */
+  int32_t pad[2];
+} fp8mlp_scale_state;
+
+#define FP8MLP_STATE_KEPT_SCALE 1
+
+/* mlp_fwd / up_proj_fused flags */
+#define FP8MLP_FWD_EVAL_BF16 1 /* evaluation: BF16 down-projection from post and W2; no FP8 copy */
+#define FP8MLP_FWD_CALIBRATE 2 /* write post and partial amax only (step 0: no amax(t-1) yet)   */
+
+/* ------------------------------------------------------------------------
+ * Forward
+ * ------------------------------------------------------------------------ */
+
+/*
+ * Fused up-projection ("A Retrospective on Our World Records", Main Track:
+ * while the up-projection has the post-activation values in registers it
+ * writes the BF16 tensor for the backward, emits the FP8 version and
+ * accumulates a tiny partial-amax tensor; "NanoGPT Speedrun (Track 1)",
+ * Changes vs Record #83, item 4: only post = relu(pre)^2 is stored).
+ *
+ *   post[m,i]     = bf16( fp32(r*r) ),  r = max(fp32(x[m,:] . W1[i,:]), 0)
+ *   post_fp8[m,i] = e4m3_satfinite( fp32(post[m,i] * st->scale) )
+ *   partial_amax  = max of post over blocks of 32 rows x 256 columns,
+ *                   fp32, laid out [4*ceil(M/128)][ceil(h/256)]; blocks
+ *                   that lie wholly past row M hold 0
+ *                   (see fp8mlp_partial_amax_shape)
+ *   pre_debug     = optional fp32 pre [M,h] (NULL to skip; slow, for tests)
+ *
+ * st->scale is read on the device; the host never waits for it.
+ * flags: FP8MLP_FWD_CALIBRATE or FP8MLP_FWD_EVAL_BF16 skip post_fp8 (may be
+ * NULL then).  post and partial_amax are always written.
+ */
+int fp8mlp_up_proj_fused(int M, int d, int h, const uint16_t* x, const uint16_t* W1,
+                         const fp8mlp_scale_state* st, uint16_t* post, uint8_t* post_fp8,
+                         float* partial_amax, float* pre_debug, int flags, fp8mlp_stream_t stream);
+
+/*
+ * FP8 scaled down-projection ("A Retrospective on Our World Records", Main
+ * Track: the down-projection runs as an FP8 scaled matmul on both operands,
+ * against the transposed FP8 cache of W2):
+ *   out[m,j] = bf16( fp32( sum_i q[m,i] * W2q_t[j,i] ) * fp32(st->scale_inv * w2_scale_inv[0]) )
+ * with fp32 accumulation.  post_fp8 [M,h], W2q_t [d,h].
+ */
+int fp8mlp_down_proj_fp8(int M, int d, int h, const uint8_t* post_fp8, const uint8_t* W2q_t,
+                         const float* w2_scale_inv, const fp8mlp_scale_state* st, uint16_t* out,
+                         fp8mlp_stream_t stream);
+
+/*
+ * BF16 down-projection for evaluation ("NanoGPT Speedrun (Track 1)", From
+ * Unoptimized, item 5: BF16 at eval):  out = bf16(post . W2), W2 [h,d].
+ */
+int fp8mlp_down_proj_bf16(int M, int d, int h, const uint16_t* post, const uint16_t* W2, uint16_t* out,
+                          fp8mlp_stream_t stream);
+
+/*
+ * Whole forward: fp8mlp_up_proj_fused, then
+ *   default flags:          fp8mlp_down_proj_fp8 (W2q_t, w2_scale_inv used; W2 may be NULL)
+ *   FP8MLP_FWD_EVAL_BF16:   fp8mlp_down_proj_bf16 (W2 used; W2q_t, w2_scale_inv, post_fp8 may be NULL)
+ *   FP8MLP_FWD_CALIBRATE:   no down-projection (out, W2*, post_fp8 may be NULL)
+ */
+int fp8mlp_mlp_fwd(int M, int d, int h, const uint16_t* x, const uint16_t* W1, const uint8_t* W2q_t,
+                   const float* w2_scale_inv, const uint16_t* W2, const fp8mlp_scale_state* st, uint16_t* post,
+                   uint8_t* post_fp8, float* partial_amax, uint16_t* out, float* pre_debug, int flags,
+                   fp8mlp_stream_t stream);
+
+/* Number of row blocks and column blocks of the partial-amax tensor for an
+ * [M,h] post, and the block size in rows / columns.  Returns FP8MLP_OK. */
+int fp8mlp_partial_amax_shape(int M, int h, int* row_blocks, int* col_blocks, int* block_rows,
+                              int* block_cols);
+
+/* ------------------------------------------------------------------------
+ * Delayed scaling and the W2 cache
+ * ------------------------------------------------------------------------ */
+
+/* Initialise a state on the device: amax_prev 0, scale = initial_scale,
+ * scale_inv = 1/initial_scale, margin, step 0, flags 0.  margin > 0 and
+ * initial_scale > 0 (finite), else FP8MLP_ERR_INVALID_ARG. */
+int fp8mlp_scale_state_init(fp8mlp_scale_state* st, float margin, float initial_scale,
+                            fp8mlp_stream_t stream);
+
+/*
+ * Reduce the partial amax of this step and derive the next step's scale
+ * ("A Retrospective on Our World Records", Main Track: "we only reduce those
+ * partial amax values later"; scale of step t from amax(t-1) times a margin):
+ *   A = max(partial_amax[0..n)),   st->amax_prev = A,   st->step += 1
+ *   if A finite and > 0:  st->scale = fp32(448 / fp32(margin * A)),
+ *                         st->scale_inv = fp32(1 / st->scale), flag cleared
+ *   else (0, NaN, inf):   scale kept, FP8MLP_STATE_KEPT_SCALE set
+ *                         (NaN/inf also set FP8MLP_STATUS_NONFINITE_AMAX)
+ * n >= 0 (n = 0 gives A = 0).  One CTA; no host synchronisation.
+ */
+int fp8mlp_amax_reduce_update_scale(const float* partial_amax, int n, fp8mlp_scale_state* st,
+                                    fp8mlp_stream_t stream);
+
+/*
+ * Refresh the transposed FP8 cache of W2 ("A Retrospective on Our World
+ * Records", Main Track: transposed FP8 cache of W2 refreshed after optimizer
+ * updates; implementation notes: exact, non-delayed refresh is viable):
+ *   s_w = fp32(448 / max|W2|)   (1 if max|W2| is 0 or not finite)
+ *   W2q_t[j,i] = e4m3_satfinite( fp32(W2[i,j] * s_w) ),  w2_scale_inv[0] = fp32(1/s_w)
+ * W2 [h,d] bf16, W2q_t [d,h] e4m3.  workspace: at least
+ * fp8mlp_workspace_size(0,d,h) bytes of caller-owned device memory (a
+ * reduction word; cleared by the call).
+ */
+int fp8mlp_w2_fp8_cache_refresh(int h, int d, const uint16_t* W2, uint8_t* W2q_t, float* w2_scale_inv,
+                                void* workspace, fp8mlp_stream_t stream);
+
+/* Device workspace in bytes needed by the calls that take one. */
+size_t fp8mlp_workspace_size(int M, int d, int h);
+
+/* ------------------------------------------------------------------------
+ * Backward ("NanoGPT Speedrun (Track 1)", Changes vs Record #83, item 4;
+ * "A Retrospective on Our World Records": BF16 backward from the BF16 post)
+ * ------------------------------------------------------------------------ */
+
+/*
+ * dPost = dOut . W2^T (fp32 accumulate);  relu(pre) rebuilt as sqrt(post):
+ *   dPre[m,i] = bf16( fp32(2 * sqrt(post[m,i])) * dPost[m,i] )
+ * dOut [M,d], W2 [h,d], post [M,h] -> dPre [M,h].
+ */
+int fp8mlp_bwd_dpre(int M, int d, int h, const uint16_t* dOut, const uint16_t* W2, const uint16_t* post,
+                    uint16_t* dPre, fp8mlp_stream_t stream);
+
+/* dX = bf16(dPre . W1):  dPre [M,h], W1 [h,d] -> dX [M,d]. */
+int fp8mlp_bwd_dx(int M, int d, int h, const uint16_t* dPre, const uint16_t* W1, uint16_t* dX,
+                  fp8mlp_stream_t stream);
+
+/* dW1 = dPre^T . x and dW2 = post^T . dOut, fp32 [h,d] each, in one launch. */
+int fp8mlp_bwd_dw(int M, int d, int h, const uint16_t* x, const uint16_t* dPre, const uint16_t* post,
+                  const uint16_t* dOut, float* dW1, float* dW2, fp8mlp_stream_t stream);
+
+/* Whole backward: fp8mlp_bwd_dpre, fp8mlp_bwd_dx, fp8mlp_bwd_dw. */
+int fp8mlp_mlp_bwd(int M, int d, int h, const uint16_t* x, const uint16_t* W1, const uint16_t* W2,
+                   const uint16_t* post, const uint16_t* dOut, uint16_t* dPre, uint16_t* dX, float* dW1,
+                   float* dW2, fp8mlp_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Layer stack helpers (RMSNorm without gain, eps = 1e-6; residual add).
+ * The pages train 9-layer, 768-dim models with ReLU^2 MLPs ("nanochat
+ * autoresearch result", Method); they do not describe the norm, so this is
+ * the plain RMSNorm reading.
+ * ------------------------------------------------------------------------ */
+
+/* x = bf16(r * rstd), rstd[m] = 1/sqrt(mean(r[m,:]^2) + 1e-6) (fp32). */
+int fp8mlp_rmsnorm_fwd(int M, int d, const uint16_t* r, uint16_t* x, float* rstd, fp8mlp_stream_t stream);
+
+/* dr_out = bf16( dr_in + rstd * (dx - xhat * mean(dx * xhat)) ), xhat = r * rstd.
+ * dr_in may equal dr_out (in place). */
+int fp8mlp_rmsnorm_bwd(int M, int d, const uint16_t* r, const float* rstd, const uint16_t* dx,
+                       const uint16_t* dr_in, uint16_t* dr_out, fp8mlp_stream_t stream);
+
+/* r_next = bf16(r + out), [M,d]. */
+int fp8mlp_residual_add(int M, int d, const uint16_t* r, const uint16_t* out, uint16_t* r_next,
+                        fp8mlp_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Status and diagnostics
+ * ------------------------------------------------------------------------ */
+
+/* Synchronise `stream`, then copy the device status word of the current
+ * device into *status (FP8MLP_STATUS_* bits; 0 = clean). */
+int fp8mlp_get_device_status(unsigned int* status, fp8mlp_stream_t stream);
+/* Clear the device status word (enqueued on `stream`). */
+int fp8mlp_clear_device_status(fp8mlp_stream_t stream);
+/* Per-wait limit of the kernels' bounded waits, in ns (default 2e9). */
+int fp8mlp_set_wait_timeout_ns(unsigned long long ns);
+/* Test hook: FP8MLP_DEBUG_STALL_PRODUCER makes the next GEMM launches'
+ * load warp issue nothing, so the MMA warp's bounded wait runs out and the
+ * kernel returns with FP8MLP_STATUS_TIMEOUT set.  0 restores normal runs. */
+#define FP8MLP_DEBUG_STALL_PRODUCER 1
+int fp8mlp_set_debug_flags(int flags);
+
+const char* fp8mlp_error_string(int code);
+/* Text of the last error on this thread (empty if none). */
+const char* fp8mlp_last_error_detail(void);
+/* Library version string. */
+const char* fp8mlp_version(void);
+/* Number of CUDA kernels the library has launched in this process. */
+unsigned long long fp8mlp_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8MLP_H */

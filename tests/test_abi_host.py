@@ -1,0 +1,119 @@
+"""Host-side checks of the C-ABI library (no GPU needed, no compute calls).
+
+The library must load, export every function the public header declares, and
+reject bad arguments on the host before touching CUDA.  With valid arguments
+and no GPU present it must say so (FP8MLP_ERR_NO_DEVICE) rather than fall back.
+"""
+import ctypes
+import re
+
+import pytest
+
+from fp8_relu_mlp_b200 import _abi as A
+
+FAKE = 0x10000  # a 16-byte aligned non-null address; never dereferenced on the host
+
+
+def test_library_exports_every_header_symbol():
+    syms = A.header_symbols()
+    assert len(syms) >= 20
+    for s in syms:
+        assert hasattr(A.lib, s), s
+        assert hasattr(A, s), f"binding lacks {s}"
+
+
+def test_header_declares_the_boundary_calls():
+    syms = set(A.header_symbols())
+    for s in ["fp8mlp_mlp_fwd", "fp8mlp_mlp_bwd", "fp8mlp_w2_fp8_cache_refresh",
+              "fp8mlp_amax_reduce_update_scale", "fp8mlp_up_proj_fused", "fp8mlp_down_proj_fp8"]:
+        assert s in syms
+
+
+def test_scale_state_layout_is_32_bytes():
+    text = open(A.HEADER).read()
+    body = re.search(r"typedef struct fp8mlp_scale_state \{(.*?)\} fp8mlp_scale_state;", text, re.S).group(1)
+    fields = re.findall(r"(float|int32_t)\s+(\w+)(\[(\d+)\])?;", body)
+    assert [f[1] for f in fields] == ["amax_prev", "scale", "scale_inv", "margin", "step", "flags", "pad"]
+    assert sum(4 * (int(f[3]) if f[3] else 1) for f in fields) == 32
+
+
+def test_version_and_error_strings():
+    assert "sm_100a" in A.fp8mlp_version()
+    assert A.fp8mlp_error_string(0) == "ok"
+    assert A.fp8mlp_error_string(A.ERR_NO_DEVICE) == "no sm_100a device"
+    assert A.fp8mlp_error_string(99) == "unknown error code"
+
+
+def _rc(name, *args):
+    return getattr(A.lib, name)(*args)
+
+
+@pytest.mark.parametrize("M,d,h,code", [(-1, 64, 256, A.ERR_INVALID_ARG), (16, 8, 256, A.ERR_UNSUPPORTED_SHAPE),
+                                        (16, 64, 250, A.ERR_UNSUPPORTED_SHAPE), (16, 72, 0, A.ERR_UNSUPPORTED_SHAPE)])
+def test_shape_checks(M, d, h, code):
+    assert _rc("fp8mlp_up_proj_fused", M, d, h, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, None) == code
+    assert _rc("fp8mlp_bwd_dpre", M, d, h, FAKE, FAKE, FAKE, FAKE, None) == code
+
+
+def test_null_and_misaligned_pointers_rejected():
+    args = [256, 64, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, None]
+    for pos in (3, 4, 6, 7):          # x, W1, post, post_fp8
+        a = list(args)
+        a[pos] = None
+        assert _rc("fp8mlp_up_proj_fused", *a) == A.ERR_INVALID_ARG
+        a[pos] = FAKE + 8
+        assert _rc("fp8mlp_up_proj_fused", *a) == A.ERR_INVALID_ARG
+        assert "aligned" in A.fp8mlp_last_error_detail()
+    # state is needed only when the FP8 copy is written
+    a = list(args)
+    a[5] = None
+    assert _rc("fp8mlp_up_proj_fused", *a) == A.ERR_INVALID_ARG
+    a[10] = A.FWD_CALIBRATE
+    a[7] = None
+    assert _rc("fp8mlp_up_proj_fused", *a) in (A.ERR_NO_DEVICE, A.OK)
+
+
+def test_flag_checks():
+    assert _rc("fp8mlp_up_proj_fused", 16, 64, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 8, None) == A.ERR_INVALID_ARG
+    assert _rc("fp8mlp_mlp_fwd", 16, 64, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+               A.FWD_EVAL_BF16 | A.FWD_CALIBRATE, None) == A.ERR_INVALID_ARG
+    assert _rc("fp8mlp_set_debug_flags", 2) == A.ERR_INVALID_ARG
+    assert _rc("fp8mlp_set_wait_timeout_ns", 0) == A.ERR_INVALID_ARG
+
+
+def test_scale_state_init_checks():
+    assert _rc("fp8mlp_scale_state_init", FAKE, ctypes.c_float(0.0), ctypes.c_float(1.0), None) == A.ERR_INVALID_ARG
+    assert _rc("fp8mlp_scale_state_init", FAKE, ctypes.c_float(2.0), ctypes.c_float(-1.0), None) == A.ERR_INVALID_ARG
+    assert _rc("fp8mlp_scale_state_init", FAKE, ctypes.c_float(float("nan")), ctypes.c_float(1.0), None) == A.ERR_INVALID_ARG
+    assert _rc("fp8mlp_amax_reduce_update_scale", FAKE, -1, FAKE, None) == A.ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_no_op():
+    # M = 0: nothing to do, nothing enqueued, no device needed
+    assert _rc("fp8mlp_up_proj_fused", 0, 64, 256, None, None, None, None, None, None, None, 0, None) == A.OK
+    assert _rc("fp8mlp_down_proj_fp8", 0, 64, 256, None, None, None, None, None, None) == A.OK
+    assert _rc("fp8mlp_bwd_dx", 0, 64, 256, None, None, None, None) == A.OK
+
+
+def test_partial_amax_shape():
+    assert A.fp8mlp_partial_amax_shape(16384, 3072) == (512, 12, 32, 256)
+    assert A.fp8mlp_partial_amax_shape(129, 256) == (8, 1, 32, 256)
+    assert A.fp8mlp_partial_amax_shape(0, 256) == (0, 1, 32, 256)
+    assert A.fp8mlp_workspace_size(16384, 768, 3072) >= 4
+
+
+def test_valid_call_without_gpu_reports_no_device():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    rc = _rc("fp8mlp_up_proj_fused", 256, 64, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, None)
+    assert rc == A.ERR_NO_DEVICE
+    with pytest.raises(A.Fp8MlpError):
+        A.fp8mlp_bwd_dx(128, 64, 256, FAKE, FAKE, FAKE, stream=0)
+
+
+def test_python_binding_rejects_non_contiguous():
+    import torch
+    t = torch.zeros(4, 4)[:, ::2]
+    with pytest.raises(ValueError):
+        A.fp8mlp_bwd_dx(4, 16, 16, t, t, t, stream=0)

@@ -1,0 +1,174 @@
+"""Parity at the full benchmark sizes, in the launch configuration bench.py
+times (MLPBlock, one call per kernel), on outputs the oracle can compute one
+by one: sampled token rows of the forward and of dX, sampled entries of dW1
+and dW2, the full W2 cache, and properties that hold at any size.
+
+The oracle computes its own amax and scale over the whole batch (in row
+chunks); the GPU state is then set to the oracle's scale so that both sides
+quantise with the same s_t.  No oracle input comes from the GPU.
+"""
+import numpy as np
+import pytest
+import torch
+
+from fp8_relu_mlp_b200 import _abi as A
+from fp8_relu_mlp_b200 import synth
+from fp8_relu_mlp_b200.block import MLPBlock
+from oracle import ref
+from tests.gpu_util import host_bits, rel_fro
+from tests.test_gpu_parity import post_within_accumulation_bound
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_amax(x, W1, chunk=2048):
+    A_ = np.float32(0.0)
+    for i in range(0, x.shape[0], chunk):
+        A_ = max(A_, ref.amax(ref.relu2_post(ref.up_proj(x[i:i + chunk], W1))))
+    return np.float32(A_)
+
+
+def _sample_rows(M, n, seed):
+    g = np.random.default_rng(seed)
+    rows = set(g.choice(M, size=n, replace=False).tolist())
+    rows |= {0, M - 1, M - 128, M // 2}
+    return np.array(sorted(rows))
+
+
+def _load(blk, P):
+    dev = blk.device
+    blk.x.copy_(MLPBlock.bits_to_bf16(P["x"], dev))
+    blk.W1.copy_(MLPBlock.bits_to_bf16(P["W1"], dev))
+    blk.W2.copy_(MLPBlock.bits_to_bf16(P["W2"], dev))
+    if hasattr(blk, "dOut"):
+        blk.dOut.copy_(MLPBlock.bits_to_bf16(P["dOut"], dev))
+
+
+def _forward_checks(blk, P, W, rows, s_o):
+    """GPU forward at the oracle's scale s_o vs oracle rows."""
+    A.fp8mlp_scale_state_init(blk.state, W.margin, float(s_o))
+    blk.forward()
+    torch.cuda.synchronize()
+    W2q_o, _, s_wi = ref.w2_cache(P["W2"])
+    assert np.array_equal(host_bits(blk.W2q_t), W2q_o)
+    s_inv = np.float32(np.float32(1) / s_o)
+    f = ref.forward_rows(rows, P["x"], P["W1"], W2q_o, s_wi, s_o, s_inv)
+    post_g = host_bits(blk.post)[rows]
+    ok, frac = post_within_accumulation_bound(post_g, P["x"], P["W1"], rows=rows)
+    assert ok and frac < 1e-2, frac
+    q_g = host_bits(blk.post_fp8)[rows]
+    # equal wherever post agrees; elsewhere one FP8 step at most
+    same = post_g == f["post"]
+    assert np.array_equal(q_g[same], f["q"][same])
+    out_g = ref.bf16_to_f64(host_bits(blk.out)[rows])
+    assert rel_fro(out_g, ref.bf16_to_f64(f["out"])) < 2e-2
+    # partial amax: block max of the GPU's own post, and its max is the global max
+    pa = blk.partial_amax
+    assert float(pa.max()) == float(blk.post.float().max())
+    return f
+
+
+@pytest.mark.parametrize("name", ["fwd16k", "step16k"])
+def test_fullsize_forward_backward_sampled(name):
+    W = synth.WORKLOADS[name]
+    M, d, h = W.M, W.d, W.h
+    P = synth.make_problem(M, d, h, seed=0)
+    blk = MLPBlock(M, d, h, margin=W.margin, with_backward=W.backward)
+    _load(blk, P)
+    blk.refresh_w2_cache()
+    # GPU calibration vs the oracle's own amax over the whole batch
+    blk.calibrate()
+    torch.cuda.synchronize()
+    A_o = _oracle_amax(P["x"], P["W1"])
+    st_o = ref.scale_update(ref.scale_state_init(W.margin, 1.0), A_o)
+    g = blk.read_state()
+    assert abs(g["amax_prev"] / float(A_o) - 1) <= 2.0 ** -7
+    assert abs(g["scale"] / float(st_o["scale"]) - 1) <= 2.0 ** -7
+    rows = _sample_rows(M, 48, seed=1)
+    _forward_checks(blk, P, W, rows, st_o["scale"])
+    assert A.fp8mlp_get_device_status() == 0
+    if not W.backward:
+        return
+    blk.backward()
+    torch.cuda.synchronize()
+    dPre_o, dX_o = ref.dx_rows(rows, P["x"], P["W1"], P["W2"], P["dOut"])
+    assert rel_fro(ref.bf16_to_f64(host_bits(blk.dPre)[rows]), ref.bf16_to_f64(dPre_o)) < 1e-2
+    assert rel_fro(ref.bf16_to_f64(host_bits(blk.dX)[rows]), ref.bf16_to_f64(dX_o)) < 1e-2
+    gen = np.random.default_rng(2)
+    pairs = [(int(i), int(j)) for i, j in zip(gen.integers(0, h, 12), gen.integers(0, d, 12))]
+    pairs += [(h - 1, d - 1), (0, 0)]
+    w1_o, w2_o = ref.dw_entries(pairs, P["x"], P["W1"], P["W2"], P["dOut"])
+    dW1, dW2 = host_bits(blk.dW1), host_bits(blk.dW2)
+    w1_g = np.array([dW1[i, j] for i, j in pairs])
+    w2_g = np.array([dW2[i, j] for i, j in pairs])
+    assert rel_fro(w1_g, w1_o) < 1e-2
+    assert rel_fro(w2_g, w2_o) < 1e-2
+    assert A.fp8mlp_get_device_status() == 0
+
+
+def test_train49k_steps_sampled():
+    """Three steps of the M=49152 train workload: perturbed weights, W2 cache
+    refreshed per step, delayed scale tracked against the oracle's."""
+    W = synth.WORKLOADS["train49k"]
+    M, d, h = W.M, W.d, W.h
+    P = synth.make_problem(M, d, h, seed=0)
+    blk = MLPBlock(M, d, h, margin=W.margin)
+    _load(blk, P)
+    blk.refresh_w2_cache()
+    blk.calibrate()
+    o = ref.scale_update(ref.scale_state_init(W.margin, 1.0), _oracle_amax(P["x"], P["W1"]))
+    steps = 3
+    for step in range(steps):
+        blk.train_step()
+        A_o = _oracle_amax(P["x"], P["W1"])
+        o = ref.scale_update(o, A_o)
+        g = blk.read_state()
+        assert abs(g["scale"] / float(o["scale"]) - 1) <= 2.0 ** -7
+        # optimizer stand-in: perturb the weights, refresh the W2 cache
+        P["W1"] = synth.perturb(P["W1"], 0, step, W.perturb_var, "W1")
+        P["W2"] = synth.perturb(P["W2"], 0, step, W.perturb_var, "W2")
+        _load(blk, P)
+        blk.refresh_w2_cache()
+    rows = _sample_rows(M, 32, seed=3)
+    _forward_checks(blk, P, W, rows, o["scale"])
+    blk.backward()
+    torch.cuda.synchronize()
+    _, dX_o = ref.dx_rows(rows, P["x"], P["W1"], P["W2"], P["dOut"])
+    assert rel_fro(ref.bf16_to_f64(host_bits(blk.dX)[rows]), ref.bf16_to_f64(dX_o)) < 1e-2
+    pairs = [(5, 7), (h - 1, 3), (1000, d - 1), (2048, 100)]
+    w1_o, w2_o = ref.dw_entries(pairs, P["x"], P["W1"], P["W2"], P["dOut"])
+    dW1, dW2 = host_bits(blk.dW1), host_bits(blk.dW2)
+    assert rel_fro(np.array([dW1[i, j] for i, j in pairs]), w1_o) < 1e-2
+    assert rel_fro(np.array([dW2[i, j] for i, j in pairs]), w2_o) < 1e-2
+    assert A.fp8mlp_get_device_status() == 0
+
+
+def test_heavytail_spike_saturates_and_matches():
+    """M=65536, d=1024, h=4096, Student-t(3) inputs: with the delayed scale of
+    the previous (normal) step, the 2x spike step saturates the FP8 copy; both
+    sides saturate the same elements."""
+    W = synth.WORKLOADS["heavytail"]
+    M, d, h = W.M, W.d, W.h
+    P = synth.make_problem(M, d, h, seed=0, x_dist=W.x_dist)
+    blk = MLPBlock(M, d, h, margin=W.margin)
+    _load(blk, P)
+    blk.refresh_w2_cache()
+    blk.calibrate()
+    torch.cuda.synchronize()
+    A_o = _oracle_amax(P["x"], P["W1"])
+    s_o = ref.scale_update(ref.scale_state_init(W.margin, 1.0), A_o)["scale"]
+    assert abs(blk.read_state()["scale"] / float(s_o) - 1) <= 2.0 ** -7
+    # spike step: x * 2 (post * 4) quantised with the scale of the normal step
+    xs = synth.to_bf16_bits(ref.bf16_to_f64(P["x"]).astype(np.float32) * W.spike_factor)
+    P2 = dict(P, x=xs)
+    _load(blk, P2)
+    rows = _sample_rows(M, 32, seed=4)
+    f = _forward_checks(blk, P2, W, rows, s_o)
+    sat_g = float(((blk.post_fp8 & 0x7F) == 0x7E).float().mean())
+    assert sat_g > 0
+    assert np.array_equal((f["q"] & 0x7F) == 0x7E, (host_bits(blk.post_fp8)[rows] & 0x7F) == 0x7E) or \
+        np.mean(((f["q"] & 0x7F) == 0x7E) != ((host_bits(blk.post_fp8)[rows] & 0x7F) == 0x7E)) < 1e-4
+    # the next scale follows the spike's amax
+    blk.update_scale()
+    A_spike = _oracle_amax(xs, P["W1"])
+    assert abs(blk.read_state()["amax_prev"] / float(A_spike) - 1) <= 2.0 ** -7

@@ -1,0 +1,500 @@
+"""Parity of the CUDA path (through the C ABI) against the CPU oracle.
+
+Bit-exact where the result is unique: post, the FP8 codes, the partial amax,
+the scale sequence, the W2 cache.  For those the up-projection inputs are
+drawn on a grid (small integers times powers of two) so that the fp32
+accumulation is exact in any order.  Within the stated tolerances elsewhere:
+relative Frobenius error <= 2e-2 for the FP8 forward output, <= 1e-2 for
+the BF16 gradients.  Every output buffer is surrounded by canaries.
+"""
+import numpy as np
+import pytest
+import torch
+
+from fp8_relu_mlp_b200 import _abi as A
+from fp8_relu_mlp_b200 import synth
+from oracle import ref
+from tests.gpu_util import Guarded, bf16_ulps, dev_bf16, dev_f32, dev_u8, host_bits, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+TOL_OUT = 2e-2
+TOL_GRAD = 1e-2
+
+SHAPES = [  # (M, d, h): several tiles, ragged tails in every dimension
+    (256, 64, 256),
+    (300, 80, 272),
+    (1, 64, 256),
+    (129, 128, 512),
+    (1000, 768, 3072),
+]
+
+
+def _state(margin=2.0, s0=1.0):
+    st = torch.zeros(8, dtype=torch.float32, device="cuda")
+    A.fp8mlp_scale_state_init(st, margin, s0)
+    return st
+
+
+def _read_state(st):
+    s = st.cpu()
+    i = s.view(torch.int32)
+    return dict(amax_prev=np.float32(s[0]), scale=np.float32(s[1]), scale_inv=np.float32(s[2]),
+                margin=np.float32(s[3]), step=int(i[4]), flags=int(i[5]))
+
+
+def _pa_oracle(post, M, h):
+    rb, cb, br, bc = A.fp8mlp_partial_amax_shape(M, h)
+    pa = ref.partial_amax(post, br, bc)
+    full = np.zeros((rb, cb), np.float32)
+    full[:pa.shape[0], :pa.shape[1]] = pa
+    return full
+
+
+def _up(M, d, h, x, W1, st, flags=0, pre=False):
+    post = Guarded((M, h), torch.bfloat16)
+    q = Guarded((M, h), torch.uint8)
+    rb, cb, _, _ = A.fp8mlp_partial_amax_shape(M, h)
+    pa = Guarded((rb, cb), torch.float32)
+    pre_t = Guarded((M, h), torch.float32) if pre else None
+    A.fp8mlp_up_proj_fused(M, d, h, x, W1, st, post.t, q.t, pa.t, pre_t.t if pre else None, flags)
+    torch.cuda.synchronize()
+    for g in (post, q, pa) + ((pre_t,) if pre else ()):
+        assert g.intact(), "write outside an output buffer"
+    return post, q, pa, pre_t
+
+
+# ---------------------------------------------------------------------------
+# K1: fused up-projection epilogue, bit-exact on grid inputs
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,d,h", SHAPES)
+def test_up_proj_fused_bit_exact_grid(M, d, h):
+    P = synth.make_problem(M, d, h, seed=M + d, x_dist="grid", w_dist="grid")
+    s = np.float32(448.0 / 37.0)
+    st = _state(2.0, float(s))
+    post, q, pa, pre = _up(M, d, h, dev_bf16(P["x"]), dev_bf16(P["W1"]), st, pre=True)
+    pre_o = ref.up_proj(P["x"], P["W1"])
+    # grid inputs: every partial sum is exact in fp32, so pre must match exactly
+    assert np.array_equal(host_bits(pre.t), pre_o.astype(np.float32))
+    post_o = ref.relu2_post(pre_o)
+    assert np.array_equal(host_bits(post.t), post_o)
+    assert np.array_equal(host_bits(q.t), ref.quantise_post(post_o, s))
+    assert np.array_equal(host_bits(pa.t), _pa_oracle(post_o, M, h))
+
+
+@pytest.mark.parametrize("flags", [A.FWD_CALIBRATE, A.FWD_EVAL_BF16])
+def test_up_proj_without_fp8_copy(flags):
+    M, d, h = 300, 64, 256
+    P = synth.make_problem(M, d, h, seed=3, x_dist="grid", w_dist="grid")
+    post = Guarded((M, h), torch.bfloat16)
+    q = Guarded((M, h), torch.uint8, fill=7)
+    rb, cb, _, _ = A.fp8mlp_partial_amax_shape(M, h)
+    pa = Guarded((rb, cb), torch.float32)
+    A.fp8mlp_up_proj_fused(M, d, h, dev_bf16(P["x"]), dev_bf16(P["W1"]), None, post.t, q.t, pa.t, None, flags)
+    torch.cuda.synchronize()
+    post_o = ref.relu2_post(ref.up_proj(P["x"], P["W1"]))
+    assert np.array_equal(host_bits(post.t), post_o)
+    assert (host_bits(q.t) == 7).all(), "the FP8 copy must not be written"
+    assert np.array_equal(host_bits(pa.t), _pa_oracle(post_o, M, h))
+    assert post.intact() and q.intact() and pa.intact()
+
+
+def post_within_accumulation_bound(post_gpu, x, W1, rows=None):
+    """post_gpu may differ from the oracle's post only through the fp32
+    accumulation of pre: with |fl(pre) - pre| <= K 2^-24 sum_k |x_k w_k|
+    (the usual recursive-summation bound), post = r^2 moves by at most
+    2 r delta + delta^2, plus one BF16 rounding step on each side."""
+    X = ref.bf16_to_f64(x if rows is None else x[rows])
+    W = ref.bf16_to_f64(W1)
+    pre = X @ W.T
+    delta = X.shape[1] * 2.0 ** -24 * (np.abs(X) @ np.abs(W).T)
+    r = np.maximum(pre, 0)
+    post_o = ref.relu2_post(pre)
+    g = ref.bf16_to_f64(post_gpu)
+    o = ref.bf16_to_f64(post_o)
+    bound = 2 * (r + delta) * delta + 2.0 ** -7 * np.maximum(g, o) + 1e-30
+    ok = np.abs(g - o) <= bound
+    return bool(ok.all()), float((post_gpu != post_o).mean())
+
+
+@pytest.mark.parametrize("M,d,h", [(256, 64, 256), (1000, 768, 3072)])
+def test_up_proj_fused_normal_inputs(M, d, h):
+    P = synth.make_problem(M, d, h, seed=11)
+    s = np.float32(20.0)
+    st = _state(2.0, float(s))
+    post, q, pa, _ = _up(M, d, h, dev_bf16(P["x"]), dev_bf16(P["W1"]), st)
+    pg = host_bits(post.t)
+    ok, frac = post_within_accumulation_bound(pg, P["x"], P["W1"])
+    assert ok and frac < 1e-2, frac
+    # the FP8 copy is the e4m3 of this post times s (library cast as check)
+    pv = torch.from_numpy(pg.view(np.int16)).view(torch.bfloat16).float() * float(s)
+    want = pv.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(host_bits(q.t), want)
+    # the partial amax is the block max of this post
+    assert np.array_equal(host_bits(pa.t), _pa_oracle(pg, M, h))
+
+
+# ---------------------------------------------------------------------------
+# K3: amax reduction + delayed scale, bit-exact
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n", [0, 1, 7, 1000, 6144, 65537])
+def test_amax_reduce_update_scale_bit_exact(n):
+    pa = synth.make_partials(n, seed=n, scale=37.0)
+    st = _state(2.0, 1.0)
+    o = ref.scale_state_init(2.0, 1.0)
+    pa_d = dev_f32(pa) if n else torch.zeros(1, device="cuda")
+    for _ in range(2):
+        A.fp8mlp_amax_reduce_update_scale(pa_d, n, st)
+        o = ref.scale_update(o, ref.reduce_partials(pa))
+    g = _read_state(st)
+    for k in ("amax_prev", "scale", "scale_inv", "margin"):
+        assert g[k] == o[k], k
+    assert g["step"] == o["step"] == 2 and g["flags"] == o["flags"]
+
+
+def test_scale_keeps_previous_on_nonfinite_amax():
+    A.fp8mlp_clear_device_status()
+    st = _state(1.5, 1.0)
+    A.fp8mlp_amax_reduce_update_scale(dev_f32(np.array([3.0, 9.0], np.float32)), 2, st)
+    before = _read_state(st)
+    A.fp8mlp_amax_reduce_update_scale(dev_f32(np.array([3.0, np.nan], np.float32)), 2, st)
+    after = _read_state(st)
+    assert after["scale"] == before["scale"] and after["flags"] & A.STATE_KEPT_SCALE
+    assert A.fp8mlp_get_device_status() & A.STATUS_NONFINITE_AMAX
+    A.fp8mlp_amax_reduce_update_scale(dev_f32(np.zeros(4, np.float32)), 4, st)
+    assert _read_state(st)["flags"] & A.STATE_KEPT_SCALE
+    A.fp8mlp_clear_device_status()
+    assert A.fp8mlp_get_device_status() == 0
+
+
+def test_scale_state_checkpoint_resume():
+    seq = [synth.make_partials(50, seed=i, scale=1.0 + i) for i in range(5)]
+    st = _state(2.0, 1.0)
+    saved = None
+    for i, pa in enumerate(seq):
+        A.fp8mlp_amax_reduce_update_scale(dev_f32(pa), 50, st)
+        if i == 1:
+            saved = st.clone()
+    final = st.clone()
+    st2 = saved.clone()
+    for pa in seq[2:]:
+        A.fp8mlp_amax_reduce_update_scale(dev_f32(pa), 50, st2)
+    assert torch.equal(st2, final)
+
+
+# ---------------------------------------------------------------------------
+# K4: transposed FP8 W2 cache, bit-exact on any input
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("h,d", [(256, 64), (272, 80), (3072, 768), (4096, 1024), (16, 16)])
+def test_w2_cache_bit_exact(h, d):
+    W2 = synth.make_problem(1, d, h, seed=h)["W2"]
+    Wq = Guarded((d, h), torch.uint8)
+    inv = Guarded((4,), torch.float32)
+    ws = torch.empty(A.fp8mlp_workspace_size(0, d, h), dtype=torch.uint8, device="cuda")
+    A.fp8mlp_w2_fp8_cache_refresh(h, d, dev_bf16(W2), Wq.t, inv.t, ws)
+    torch.cuda.synchronize()
+    q_o, s_w, s_wi = ref.w2_cache(W2)
+    assert np.array_equal(host_bits(Wq.t), q_o)
+    assert host_bits(inv.t)[0] == s_wi
+    assert Wq.intact() and inv.intact()
+
+
+def test_w2_cache_zero_weights_flagged():
+    A.fp8mlp_clear_device_status()
+    h, d = 64, 32
+    Wq = torch.full((d, h), 9, dtype=torch.uint8, device="cuda")
+    inv = torch.zeros(4, device="cuda")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    A.fp8mlp_w2_fp8_cache_refresh(h, d, torch.zeros(h, d, dtype=torch.bfloat16, device="cuda"), Wq, inv, ws)
+    assert (Wq == 0).all() and float(inv[0]) == 1.0
+    assert A.fp8mlp_get_device_status() & A.STATUS_W2_DEGENERATE
+    A.fp8mlp_clear_device_status()
+
+
+# ---------------------------------------------------------------------------
+# K2: FP8 down-projection
+# ---------------------------------------------------------------------------
+
+def _rand_codes(g, shape):
+    c = g.integers(0, 256, size=shape).astype(np.uint8)
+    c[(c & 0x7F) == 0x7F] = 0x30   # no NaN codes
+    return c
+
+
+@pytest.mark.parametrize("M,d,h", SHAPES)
+def test_down_proj_fp8(M, d, h):
+    g = np.random.default_rng(M * 7 + h)
+    q = _rand_codes(g, (M, h))
+    Wq = _rand_codes(g, (d, h))
+    sinv, swinv = np.float32(1 / 37.0), np.float32(1 / 150.0)
+    st = _state(2.0, float(np.float32(1) / sinv))
+    A.fp8mlp_amax_reduce_update_scale(torch.zeros(1, device="cuda"), 0, st)  # keeps scale; exercises the state
+    s_now = _read_state(st)
+    out = Guarded((M, d), torch.bfloat16)
+    A.fp8mlp_down_proj_fp8(M, d, h, dev_u8(q), dev_u8(Wq), dev_f32(np.array([swinv, 0, 0, 0], np.float32)), st, out.t)
+    torch.cuda.synchronize()
+    want = ref.down_proj_fp8(q, Wq, s_now["scale_inv"], swinv)
+    got = host_bits(out.t)
+    # only the fp32 accumulation order and the final BF16 rounding differ
+    assert rel_fro(ref.bf16_to_f64(got), ref.bf16_to_f64(want)) < 4e-3
+    assert out.intact()
+
+
+@pytest.mark.parametrize("M,d,h", [(256, 64, 256), (300, 80, 272), (1000, 768, 3072)])
+def test_down_proj_bf16_eval(M, d, h):
+    P = synth.make_problem(M, d, h, seed=5)
+    post = ref.relu2_post(ref.up_proj(P["x"], P["W1"]))
+    out = Guarded((M, d), torch.bfloat16)
+    A.fp8mlp_down_proj_bf16(M, d, h, dev_bf16(post), dev_bf16(P["W2"]), out.t)
+    torch.cuda.synchronize()
+    want = ref.down_proj_bf16(post, P["W2"])
+    assert rel_fro(ref.bf16_to_f64(host_bits(out.t)), ref.bf16_to_f64(want)) < 4e-3
+    assert out.intact()
+
+
+# ---------------------------------------------------------------------------
+# whole forward, FP8 path, vs the oracle
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,d,h", SHAPES)
+def test_mlp_fwd_fp8(M, d, h):
+    P = synth.make_problem(M, d, h, seed=21)
+    W2q_t, s_w, s_wi = ref.w2_cache(P["W2"])
+    st = _state(2.0, 1.0)
+    x, W1 = dev_bf16(P["x"]), dev_bf16(P["W1"])
+    rb, cb, _, _ = A.fp8mlp_partial_amax_shape(M, h)
+    post = torch.empty(M, h, dtype=torch.bfloat16, device="cuda")
+    pa = torch.empty(rb, cb, device="cuda")
+    # step 0: calibration, then the first scale
+    A.fp8mlp_mlp_fwd(M, d, h, x, W1, None, None, None, st, post, None, pa, None, None, A.FWD_CALIBRATE)
+    A.fp8mlp_amax_reduce_update_scale(pa, pa.numel(), st)
+    s1 = _read_state(st)
+    q = torch.empty(M, h, dtype=torch.uint8, device="cuda")
+    out = Guarded((M, d), torch.bfloat16)
+    inv = dev_f32(np.array([s_wi, 0, 0, 0], np.float32))
+    A.fp8mlp_mlp_fwd(M, d, h, x, W1, dev_u8(W2q_t), inv, None, st, post, q, pa, out.t, None, 0)
+    torch.cuda.synchronize()
+    o_st = ref.scale_update(ref.scale_state_init(2.0, 1.0),
+                            ref.amax(ref.relu2_post(ref.up_proj(P["x"], P["W1"]))))
+    assert abs(float(s1["scale"]) / float(o_st["scale"]) - 1) < 1e-2
+    f = ref.forward(P["x"], P["W1"], W2q_t, s_wi, s1["scale"], s1["scale_inv"])
+    assert rel_fro(ref.bf16_to_f64(host_bits(out.t)), ref.bf16_to_f64(f["out"])) < TOL_OUT
+    # and the FP8 forward stays close to the exact BF16 network
+    exact = ref.bf16_to_f64(ref.down_proj_bf16(f["post"], P["W2"]))
+    assert rel_fro(ref.bf16_to_f64(host_bits(out.t)), exact) < 6e-2
+    assert out.intact()
+
+
+# ---------------------------------------------------------------------------
+# backward kernels
+# ---------------------------------------------------------------------------
+
+def _post_like(g, M, h):
+    v = np.maximum(g.standard_normal((M, h)), 0).astype(np.float32) ** 2
+    return synth.to_bf16_bits(v)
+
+
+@pytest.mark.parametrize("M,d,h", SHAPES)
+def test_bwd_dpre(M, d, h):
+    P = synth.make_problem(M, d, h, seed=31)
+    post = _post_like(np.random.default_rng(M), M, h)
+    dPre = Guarded((M, h), torch.bfloat16)
+    A.fp8mlp_bwd_dpre(M, d, h, dev_bf16(P["dOut"]), dev_bf16(P["W2"]), dev_bf16(post), dPre.t)
+    torch.cuda.synchronize()
+    want = ref.bwd_dpre(post, P["dOut"], P["W2"])
+    got = host_bits(dPre.t)
+    assert rel_fro(ref.bf16_to_f64(got), ref.bf16_to_f64(want)) < 4e-3
+    # zero post gives exactly zero dPre (relu'(pre) = 0 there)
+    assert (ref.bf16_to_f64(got)[ref.bf16_to_f64(post) == 0] == 0).all()
+    assert dPre.intact()
+
+
+@pytest.mark.parametrize("M,d,h", SHAPES)
+def test_bwd_dx(M, d, h):
+    P = synth.make_problem(M, d, h, seed=41)
+    g = np.random.default_rng(M + 1)
+    dPre = synth.to_bf16_bits(g.standard_normal((M, h)).astype(np.float32))
+    dX = Guarded((M, d), torch.bfloat16)
+    A.fp8mlp_bwd_dx(M, d, h, dev_bf16(dPre), dev_bf16(P["W1"]), dX.t)
+    torch.cuda.synchronize()
+    want = ref.bwd_dx(dPre, P["W1"])
+    assert rel_fro(ref.bf16_to_f64(host_bits(dX.t)), ref.bf16_to_f64(want)) < 4e-3
+    assert dX.intact()
+
+
+@pytest.mark.parametrize("M,d,h", SHAPES)
+def test_bwd_dw(M, d, h):
+    P = synth.make_problem(M, d, h, seed=51)
+    g = np.random.default_rng(M + 2)
+    dPre = synth.to_bf16_bits(g.standard_normal((M, h)).astype(np.float32))
+    post = _post_like(g, M, h)
+    dW1, dW2 = Guarded((h, d), torch.float32), Guarded((h, d), torch.float32)
+    A.fp8mlp_bwd_dw(M, d, h, dev_bf16(P["x"]), dev_bf16(dPre), dev_bf16(post), dev_bf16(P["dOut"]), dW1.t, dW2.t)
+    torch.cuda.synchronize()
+    assert rel_fro(host_bits(dW1.t), ref.bwd_dw1(dPre, P["x"])) < 1e-4
+    assert rel_fro(host_bits(dW2.t), ref.bwd_dw2(post, P["dOut"])) < 1e-4
+    assert dW1.intact() and dW2.intact()
+
+
+@pytest.mark.parametrize("M,d,h", SHAPES)
+def test_mlp_bwd_vs_oracle(M, d, h):
+    P = synth.make_problem(M, d, h, seed=61)
+    post = ref.relu2_post(ref.up_proj(P["x"], P["W1"]))
+    dPre = torch.empty(M, h, dtype=torch.bfloat16, device="cuda")
+    dX = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+    dW1 = torch.empty(h, d, device="cuda")
+    dW2 = torch.empty(h, d, device="cuda")
+    A.fp8mlp_mlp_bwd(M, d, h, dev_bf16(P["x"]), dev_bf16(P["W1"]), dev_bf16(P["W2"]), dev_bf16(post),
+                     dev_bf16(P["dOut"]), dPre, dX, dW1, dW2)
+    torch.cuda.synchronize()
+    b = ref.backward(P["x"], P["W1"], P["W2"], post, P["dOut"])
+    assert rel_fro(ref.bf16_to_f64(host_bits(dX)), ref.bf16_to_f64(b["dX"])) < TOL_GRAD
+    assert rel_fro(host_bits(dW1), b["dW1"]) < TOL_GRAD
+    assert rel_fro(host_bits(dW2), b["dW2"]) < TOL_GRAD
+
+
+def test_bwd_dw_empty_batch_zeroes():
+    h, d = 256, 64
+    dW1 = torch.full((h, d), 3.0, device="cuda")
+    dW2 = torch.full((h, d), 3.0, device="cuda")
+    A.fp8mlp_bwd_dw(0, d, h, None, None, None, None, dW1, dW2)
+    assert (dW1 == 0).all() and (dW2 == 0).all()
+
+
+# ---------------------------------------------------------------------------
+# delayed scaling over steps (the tiny workload), bit-exact on grid inputs
+# ---------------------------------------------------------------------------
+
+def _grid_perturb(W, seed):
+    g = np.random.default_rng(seed)
+    v = ref.bf16_to_f64(W) + g.integers(-2, 3, W.shape) / 256.0
+    return synth.to_bf16_bits(np.clip(v, -0.25, 0.25).astype(np.float32))
+
+
+def test_tiny_three_steps_bit_exact_grid():
+    W = synth.WORKLOADS["tiny"]
+    M, d, h = W.M, W.d, W.h
+    P = synth.make_problem(M, d, h, seed=0, x_dist="grid", w_dist="grid")
+    W1, W2 = P["W1"], P["W2"]
+    st = _state(W.margin, 1.0)
+    o = ref.scale_state_init(W.margin, 1.0)
+    rb, cb, _, _ = A.fp8mlp_partial_amax_shape(M, h)
+    x = dev_bf16(P["x"])
+    post = torch.empty(M, h, dtype=torch.bfloat16, device="cuda")
+    q = torch.empty(M, h, dtype=torch.uint8, device="cuda")
+    pa = torch.empty(rb, cb, device="cuda")
+    out = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+    Wq = torch.empty(d, h, dtype=torch.uint8, device="cuda")
+    inv = torch.empty(4, device="cuda")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    # calibration step
+    A.fp8mlp_mlp_fwd(M, d, h, x, dev_bf16(W1), None, None, None, st, post, None, pa, None, None, A.FWD_CALIBRATE)
+    A.fp8mlp_amax_reduce_update_scale(pa, pa.numel(), st)
+    o = ref.scale_update(o, ref.amax(ref.relu2_post(ref.up_proj(P["x"], W1))))
+    for step in range(W.steps):
+        A.fp8mlp_w2_fp8_cache_refresh(h, d, dev_bf16(W2), Wq, inv, ws)
+        W2q_o, _, s_wi_o = ref.w2_cache(W2)
+        A.fp8mlp_mlp_fwd(M, d, h, x, dev_bf16(W1), Wq, inv, None, st, post, q, pa, out, None, 0)
+        A.fp8mlp_amax_reduce_update_scale(pa, pa.numel(), st)
+        f = ref.forward(P["x"], W1, W2q_o, s_wi_o, o["scale"], o["scale_inv"])
+        assert np.array_equal(host_bits(Wq), W2q_o)
+        assert np.array_equal(host_bits(post), f["post"])
+        assert np.array_equal(host_bits(q), f["q"])
+        assert rel_fro(ref.bf16_to_f64(host_bits(out)), ref.bf16_to_f64(f["out"])) < 4e-3
+        o = ref.scale_update(o, f["amax"])
+        g = _read_state(st)
+        assert g["scale"] == o["scale"] and g["scale_inv"] == o["scale_inv"] and g["amax_prev"] == o["amax_prev"]
+        W1 = _grid_perturb(W1, 1000 * step)
+        W2 = _grid_perturb(W2, 1000 * step + 1)
+
+
+def test_tiny_three_steps_normal_perturbed():
+    W = synth.WORKLOADS["tiny"]
+    M, d, h = W.M, W.d, W.h
+    P = synth.make_problem(M, d, h, seed=0)
+    W1, W2 = P["W1"], P["W2"]
+    st = _state(W.margin, 1.0)
+    o = ref.scale_state_init(W.margin, 1.0)
+    rb, cb, _, _ = A.fp8mlp_partial_amax_shape(M, h)
+    x = dev_bf16(P["x"])
+    post = torch.empty(M, h, dtype=torch.bfloat16, device="cuda")
+    q = torch.empty(M, h, dtype=torch.uint8, device="cuda")
+    pa = torch.empty(rb, cb, device="cuda")
+    out = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+    Wq = torch.empty(d, h, dtype=torch.uint8, device="cuda")
+    inv = torch.empty(4, device="cuda")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    A.fp8mlp_mlp_fwd(M, d, h, x, dev_bf16(W1), None, None, None, st, post, None, pa, None, None, A.FWD_CALIBRATE)
+    A.fp8mlp_amax_reduce_update_scale(pa, pa.numel(), st)
+    o = ref.scale_update(o, ref.amax(ref.relu2_post(ref.up_proj(P["x"], W1))))
+    for step in range(W.steps):
+        A.fp8mlp_w2_fp8_cache_refresh(h, d, dev_bf16(W2), Wq, inv, ws)
+        W2q_o, _, s_wi_o = ref.w2_cache(W2)
+        assert np.array_equal(host_bits(Wq), W2q_o)
+        A.fp8mlp_mlp_fwd(M, d, h, x, dev_bf16(W1), Wq, inv, None, st, post, q, pa, out, None, 0)
+        A.fp8mlp_amax_reduce_update_scale(pa, pa.numel(), st)
+        f = ref.forward(P["x"], W1, W2q_o, s_wi_o, o["scale"], o["scale_inv"])
+        assert rel_fro(ref.bf16_to_f64(host_bits(out)), ref.bf16_to_f64(f["out"])) < TOL_OUT
+        o = ref.scale_update(o, f["amax"])
+        g = _read_state(st)
+        assert abs(float(g["scale"]) / float(o["scale"]) - 1) < 1e-2
+        W1 = synth.perturb(W1, 0, step, W.perturb_var, "W1")
+        W2 = synth.perturb(W2, 0, step, W.perturb_var, "W2")
+
+
+# ---------------------------------------------------------------------------
+# failure detection: a bounded wait runs out, the context stays usable
+# ---------------------------------------------------------------------------
+
+def test_bounded_wait_times_out_and_reports():
+    M, d, h = 256, 64, 256
+    P = synth.make_problem(M, d, h, seed=1, x_dist="grid", w_dist="grid")
+    st = _state(2.0, 4.0)
+    A.fp8mlp_clear_device_status()
+    A.fp8mlp_set_wait_timeout_ns(50_000_000)
+    A.fp8mlp_set_debug_flags(A.DEBUG_STALL_PRODUCER)
+    try:
+        post, q, pa, _ = _up(M, d, h, dev_bf16(P["x"]), dev_bf16(P["W1"]), st)
+        status = A.fp8mlp_get_device_status()
+    finally:
+        A.fp8mlp_set_debug_flags(0)
+        A.fp8mlp_set_wait_timeout_ns(2_000_000_000)
+    assert status & A.STATUS_TIMEOUT
+    A.fp8mlp_clear_device_status()
+    # the same call now runs normally and is correct
+    post, q, pa, _ = _up(M, d, h, dev_bf16(P["x"]), dev_bf16(P["W1"]), st)
+    assert A.fp8mlp_get_device_status() == 0
+    assert np.array_equal(host_bits(post.t), ref.relu2_post(ref.up_proj(P["x"], P["W1"])))
+
+
+# ---------------------------------------------------------------------------
+# RMSNorm / residual helpers of the layer stack
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,d", [(1, 768), (300, 64), (4096, 768), (77, 1024)])
+def test_rmsnorm_and_residual(M, d):
+    g = np.random.default_rng(M + d)
+    r = synth.to_bf16_bits(g.standard_normal((M, d)).astype(np.float32) * 3)
+    dx = synth.to_bf16_bits(g.standard_normal((M, d)).astype(np.float32))
+    dr = synth.to_bf16_bits(g.standard_normal((M, d)).astype(np.float32))
+    o = synth.to_bf16_bits(g.standard_normal((M, d)).astype(np.float32))
+    x = Guarded((M, d), torch.bfloat16)
+    rstd = Guarded((M,), torch.float32)
+    A.fp8mlp_rmsnorm_fwd(M, d, dev_bf16(r), x.t, rstd.t)
+    xo, rso = ref.rmsnorm_fwd(r)
+    torch.cuda.synchronize()
+    xg, xw = ref.bf16_to_f64(host_bits(x.t)), ref.bf16_to_f64(xo)
+    assert (np.abs(xg - xw) <= 2.0 ** -7 * np.abs(xw) + 1e-30).all()   # at most one BF16 step
+    np.testing.assert_allclose(host_bits(rstd.t), rso, rtol=1e-5)
+    dro = Guarded((M, d), torch.bfloat16)
+    A.fp8mlp_rmsnorm_bwd(M, d, dev_bf16(r), rstd.t, dev_bf16(dx), dev_bf16(dr), dro.t)
+    want = ref.bf16_to_f64(dr) + ref.rmsnorm_bwd(r, dx)
+    assert rel_fro(ref.bf16_to_f64(host_bits(dro.t)), want) < 4e-3
+    rn = Guarded((M, d), torch.bfloat16)
+    A.fp8mlp_residual_add(M, d, dev_bf16(r), dev_bf16(o), rn.t)
+    torch.cuda.synchronize()
+    assert np.array_equal(host_bits(rn.t), ref.residual_add(r, o))
+    assert x.intact() and rstd.intact() and dro.intact() and rn.intact()
