@@ -6,7 +6,7 @@ namespace fp8mlp {
 using CfgUp = GemmCfg<kGemmBN, 4, false, false, false, Epi::UpFused>;
 using CfgDown8 = GemmCfg<kGemmBN, 4, true, false, false, Epi::DownScaled>;
 using CfgBf16MnB = GemmCfg<kGemmBN, 4, false, false, true, Epi::StoreBf16>;
-using CfgDPre = GemmCfg<kGemmBN, 4, false, false, false, Epi::DPre>;
+using CfgDPre = GemmCfg<kGemmBN, 3, false, false, false, Epi::DPre>;
 using CfgDW = GemmCfg<kGemmBN, 4, false, true, true, Epi::StoreF32>;
 
 namespace {

@@ -77,14 +77,18 @@ struct GemmCfg {
   static constexpr int NCHUNK = BN / ECOLS;
   static constexpr int OUT_BUF = 32 * ECOLS * (EPI == Epi::StoreF32 ? 4 : 2);
   static constexpr int OUT2_BUF = EPI == Epi::UpFused ? 32 * ECOLS : 0;
-  static constexpr int AUX_BUF = EPI == Epi::DPre ? 32 * ECOLS * 2 : 0;
-  static constexpr int SLOT = OUT_BUF + OUT2_BUF + AUX_BUF;  // multiple of 1024
+  static constexpr int SLOT = OUT_BUF + OUT2_BUF;  // one output staging slot (two per epilogue warp)
   static_assert(SLOT % 1024 == 0, "slot alignment");
+  // DPre: each epilogue warp keeps the post block of a whole tile (NCHUNK
+  // chunks of 32x32) in its own ring, loaded one tile ahead
+  static constexpr int AUX_CHUNK = EPI == Epi::DPre ? 32 * ECOLS * 2 : 0;
+  static constexpr int AUX_WARP = AUX_CHUNK * NCHUNK;
+  static constexpr int NAUX = EPI == Epi::DPre ? NCHUNK : 0;
   static constexpr int TMEM_COLS = 512;
   static_assert(2 * BN <= TMEM_COLS, "two accumulators");
-  static constexpr int NUM_BARS = 2 * STAGES + 4 + 8 + 1;
+  static constexpr int NUM_BARS = 2 * STAGES + 4 + 4 * NAUX + 1;
   static constexpr int SMEM_BYTES =
-      1024 /*alignment slack*/ + STAGES * (A_BYTES + B_BYTES) + 8 * SLOT + NUM_BARS * 8 + 16;
+      1024 /*alignment slack*/ + STAGES * (A_BYTES + B_BYTES) + 8 * SLOT + 4 * AUX_WARP + NUM_BARS * 8 + 16;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
@@ -117,13 +121,14 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
   uint8_t* sA = smem;
   uint8_t* sB = sA + C::STAGES * C::A_BYTES;
   uint8_t* sEpi = sB + C::STAGES * C::B_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + 8 * C::SLOT);
+  uint8_t* sAux = sEpi + 8 * C::SLOT;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sAux + 4 * C::AUX_WARP);
   uint64_t* full = bars;
   uint64_t* empty = bars + C::STAGES;
   uint64_t* tfull = bars + 2 * C::STAGES;
   uint64_t* tempty = tfull + 2;
-  uint64_t* auxb = tempty + 2;  // [4 warps][2 slots]
-  uint64_t* fin = auxb + 8;
+  uint64_t* auxb = tempty + 2;  // [4 warps][NAUX chunks]
+  uint64_t* fin = auxb + 4 * C::NAUX;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(fin + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -139,7 +144,7 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 128);
     }
-    for (int i = 0; i < 8; ++i) mbar_init(&auxb[i], 1);
+    for (int i = 0; i < 4 * C::NAUX; ++i) mbar_init(&auxb[i], 1);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -265,7 +270,30 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
       if (p.write_q) s_up = p.st->scale;
     }
     if constexpr (C::EPI == Epi::DownScaled) comb = __fmul_rn(p.st->scale_inv, *p.w2_scale_inv);
-    uint32_t aux_issued[2] = {0u, 0u};  // post loads issued into each of this warp's two slots
+    // DPre: rounds of post prefetch started (one round = a tile's NAUX chunks,
+    // ring slot c = chunk c) and how many slots the latest round has reached
+    uint32_t aux_rounds = 0, aux_last = 0;
+    uint8_t* aux_ring = sAux + q * C::AUX_WARP;
+    auto issue_post_tile = [&](int tile) {
+      if constexpr (C::EPI == Epi::DPre) {
+        const int g2 = tile / tiles_per_group;
+        const int t2 = tile - g2 * tiles_per_group;
+        const int r0 = (t2 / p.tiles_n) * C::BM + q * 32;
+        const int c0 = (t2 % p.tiles_n) * C::BN;
+        for (int c = 0; c < C::NAUX; ++c) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&auxb[q * C::NAUX + c], C::AUX_CHUNK);
+            tma_load_2d(aux_ring + c * C::AUX_CHUNK, &p.tmAux, &auxb[q * C::NAUX + c], c0 + c * C::ECOLS, r0);
+          }
+        }
+        aux_rounds = 1;
+        aux_last = C::NAUX;
+      }
+    };
+    uint32_t iter = 0;  // tiles processed by this CTA
+    if constexpr (C::EPI == Epi::DPre) {
+      if (static_cast<int>(blockIdx.x) < num_tiles) issue_post_tile(blockIdx.x);
+    }
 
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
       const int g = t / tiles_per_group;
@@ -274,17 +302,7 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
       const int m0 = mb * C::BM, n0 = nb * C::BN;
       const int row0 = m0 + q * 32;
 
-      if constexpr (C::EPI == Epi::DPre) {
-        // prefetch the post chunk of column block 0 while the mainloop runs
-        const uint32_t b = ctr & 1u;
-        if (lane == 0) {
-          uint64_t* bar = &auxb[q * 2 + b];
-          mbar_arrive_expect_tx(bar, C::AUX_BUF);
-          tma_load_2d(sEpi + (q * 2 + b) * C::SLOT + C::OUT_BUF, &p.tmAux, bar, n0, row0);
-        }
-        ++aux_issued[b];
-      }
-
+      const int next_tile = t + static_cast<int>(gridDim.x);
       if (!mbar_wait(&tfull[acc], acc_phase, w)) break;
       tc_fence_after();
       float tmax = 0.f;
@@ -351,24 +369,28 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
           }
           store_row_bf16<64>(sbase, lane, pk);
         } else if constexpr (C::EPI == Epi::DPre) {
-          // prefetch the next column block's post before consuming this one
-          if (c + 1 < C::NCHUNK) {
-            const uint32_t nb2 = (ctr + 1) & 1u;
-            if (lane == 0) {
-              uint64_t* bar = &auxb[q * 2 + nb2];
-              mbar_arrive_expect_tx(bar, C::AUX_BUF);
-              tma_load_2d(sEpi + (q * 2 + nb2) * C::SLOT + C::OUT_BUF, &p.tmAux, bar, col0 + C::ECOLS, row0);
-            }
-            ++aux_issued[nb2];
-          }
-          if (!mbar_wait(&auxb[q * 2 + b], (ctr >> 1) & 1u, w)) {
+          // post of this chunk was loaded one tile ahead into ring slot c
+          if (!mbar_wait(&auxb[q * C::NAUX + c], iter & 1u, w)) {
             ok = false;
           } else {
-            const uint32_t ab = sbase + C::OUT_BUF;
+            const uint32_t ab = smem_u32(aux_ring + c * C::AUX_CHUNK);
             uint32_t pp[16], pk[16];
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               ld_shared_v4(ab + swz<3>(lane * 64 + j * 16), pp[4 * j], pp[4 * j + 1], pp[4 * j + 2], pp[4 * j + 3]);
+            __syncwarp();
+            // ring slot c is free again: fetch the next tile's chunk c into it
+            if (next_tile < num_tiles) {
+              const int g2 = next_tile / tiles_per_group;
+              const int t2 = next_tile - g2 * tiles_per_group;
+              if (lane == 0) {
+                mbar_arrive_expect_tx(&auxb[q * C::NAUX + c], C::AUX_CHUNK);
+                tma_load_2d(aux_ring + c * C::AUX_CHUNK, &p.tmAux, &auxb[q * C::NAUX + c],
+                            (t2 % p.tiles_n) * C::BN + c * C::ECOLS, (t2 / p.tiles_n) * C::BM + q * 32);
+              }
+              if (c == 0) aux_rounds = iter + 2;
+              aux_last = c + 1;
+            }
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float r0 = 2.f * __fsqrt_rn(bf16lo_to_f32(pp[i]));
@@ -404,12 +426,15 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
         acc = 0;
         acc_phase ^= 1u;
       }
+      ++iter;
     }
     if (lane == 0) {
       if constexpr (C::EPI == Epi::DPre) {
-        // the last load issued into each slot must have landed before exit
-        for (int b = 0; b < 2; ++b)
-          if (aux_issued[b] > 0) mbar_wait_drain(&auxb[q * 2 + b], (aux_issued[b] - 1u) & 1u, p.timeout_ns);
+        // the last load issued into each ring slot must have landed before exit
+        for (int c = 0; c < C::NAUX; ++c) {
+          const uint32_t n = static_cast<uint32_t>(c) < aux_last ? aux_rounds : aux_rounds - 1u;
+          if (n > 0) mbar_wait_drain(&auxb[q * C::NAUX + c], (n - 1u) & 1u, p.timeout_ns);
+        }
       }
       bulk_wait<0>();
     }
