@@ -24,7 +24,7 @@ enum class Epi : int {
   UpFused = 0,     // post = bf16(relu(acc)^2), q = e4m3(post*s), partial amax
   DownScaled = 1,  // out = bf16(acc * s^-1 * s_w^-1)
   StoreBf16 = 2,   // out = bf16(acc)
-  DPre = 3,        // dPre = bf16(2 sqrt(post) * acc), post read by TMA
+  DPre = 3,        // dPre = bf16(2 sqrt(post) * acc), post read by TMA (hardware sqrt.approx)
   StoreF32 = 4,    // out = acc (fp32)
 };
 
@@ -393,8 +393,8 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
             }
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float r0 = 2.f * __fsqrt_rn(bf16lo_to_f32(pp[i]));
-              const float r1 = 2.f * __fsqrt_rn(bf16hi_to_f32(pp[i]));
+              const float r0 = 2.f * sqrt_approx(bf16lo_to_f32(pp[i]));
+              const float r1 = 2.f * sqrt_approx(bf16hi_to_f32(pp[i]));
               pk[i] = pack_bf16x2(__fmul_rn(r0, __uint_as_float(v[2 * i])), __fmul_rn(r1, __uint_as_float(v[2 * i + 1])));
             }
             store_row_bf16<64>(sbase, lane, pk);

@@ -251,6 +251,12 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
 }
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t packed) { return __uint_as_float(packed << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t packed) { return __uint_as_float(packed & 0xFFFF0000u); }
+// hardware approximate square root (sqrt.approx.f32, no flush to zero)
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float y;
+  asm("sqrt.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 // fp32 -> nearest bf16 value, returned as fp32
 __device__ __forceinline__ float round_bf16(float x) { return bf16lo_to_f32(pack_bf16x2(x, 0.f)); }
 

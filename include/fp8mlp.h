@@ -210,6 +210,8 @@ size_t fp8mlp_workspace_size(int M, int d, int h);
 /*
  * dPost = dOut . W2^T (fp32 accumulate);  relu(pre) rebuilt as sqrt(post):
  *   dPre[m,i] = bf16( fp32(2 * sqrt(post[m,i])) * dPost[m,i] )
+ * sqrt is the hardware approximation (sqrt.approx.f32, about one fp32 ulp),
+ * far below the BF16 rounding of dPre that follows.
  * dOut [M,d], W2 [h,d], post [M,h] -> dPre [M,h].
  */
 int fp8mlp_bwd_dpre(int M, int d, int h, const uint16_t* dOut, const uint16_t* W2, const uint16_t* post,
