@@ -10,8 +10,9 @@ down-projection, the BF16 backward (dPre through sqrt(post), dX, dW1, dW2),
 the partial-amax reduction with the delayed-scale update, and the W2 FP8
 cache refresh.  Inputs are resident in HBM when the timed region starts; L2
 is flushed (a 256 MiB write) between timed steps, outside the step's events.
-The per-kernel CUDA events are recorded on the launching stream inside the
-timed steps.  ``e2e`` repeats the measurement through the same public API
+Each timed step is one CUDA-graph replay whose event-record nodes mark the
+step and the dominant kernel (on the launching stream); a per-kernel
+breakdown comes from separate untimed steps.  ``e2e`` repeats the measurement through the same public API
 with the step's inputs copied in from pinned host memory and its results
 (out, dX) copied back, inside the timed region.
 
@@ -51,6 +52,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
+    ap.add_argument("--eager", action="store_true", help="launch every call from the host instead of replaying a CUDA graph")
     return ap.parse_args()
 
 
@@ -286,8 +288,8 @@ def run_ours(a, W, world, rank, local_rank):
 
     def step(ev=None):
         def mark(i):
-            if ev is not None:
-                ev[i].record(stream)
+            if ev is not None and ev[i] is not None:
+                ev[i].record()  # the current stream: the capture stream while capturing
         mark(0)
         A.fp8mlp_up_proj_fused(M, d, h, blk.x, blk.W1, blk.state, blk.post, blk.post_fp8, blk.partial_amax)
         mark(1)
@@ -304,31 +306,68 @@ def run_ours(a, W, world, rank, local_rank):
         blk.refresh_w2_cache()
         mark(7)
 
+    # one step = one CUDA-graph replay of the whole call sequence.  A first,
+    # untimed pass with an event between every kernel gives the per-kernel
+    # breakdown and picks the dominant kernel; the timed steps carry only four
+    # events (start, around the dominant kernel, end) to keep event overhead
+    # out of the measured step.
+    step()
+    torch.cuda.synchronize()
+
+    def graph_of(marks):
+        evs = [torch.cuda.Event(enable_timing=True, external=not a.eager) for _ in range(8)]
+        want = set(marks)
+        sub = [evs[i] if i in want else None for i in range(8)]
+        g = None if a.eager else blk.capture(lambda: step(sub))
+        return g, evs
+
+    def replay(g, evs, marks):
+        if g is not None:
+            g.replay()
+        else:
+            step([evs[i] if i in marks else None for i in range(8)])
+
+    all_marks = list(range(8))
+    g_all, ev_all = graph_of(all_marks)
     for _ in range(max(a.warmup, 3)):
         flush.zero_()
-        step()
+        replay(g_all, ev_all, all_marks)
+    torch.cuda.synchronize()
+    per_kernel = {n: [] for n in names}
+    for _ in range(5):
+        flush.zero_()
+        replay(g_all, ev_all, all_marks)
+        ev_all[7].synchronize()
+        for k, n in enumerate(names):
+            per_kernel[n].append(ev_all[k].elapsed_time(ev_all[k + 1]))
+    breakdown = {n: statistics.median(v) for n, v in per_kernel.items()}
+    dom_i = max(range(len(names)), key=lambda k: breakdown[names[k]])
+    marks = [0, dom_i, dom_i + 1, 7]
+    n_cap0 = A.fp8mlp_kernel_launch_count()
+    g_t, ev_t = graph_of(marks)
+    kernels_per_step = A.fp8mlp_kernel_launch_count() - n_cap0 if g_t is not None else None
+    for _ in range(2):
+        flush.zero_()
+        replay(g_t, ev_t, marks)
     torch.cuda.synchronize()
     A.fp8mlp_clear_device_status()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(a.steps)]
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     n0 = A.fp8mlp_kernel_launch_count()
+    step_ms, dom_ms = [], []
     with ClockSampler(local_rank) as clk:
         for i in range(a.steps):
             flush.zero_()
-            step(evs[i])
+            replay(g_t, ev_t, marks)
+            ev_t[7].synchronize()
+            step_ms.append(ev_t[0].elapsed_time(ev_t[7]))
+            dom_ms.append(ev_t[dom_i].elapsed_time(ev_t[dom_i + 1]))
         torch.cuda.synchronize()
-    launches = A.fp8mlp_kernel_launch_count() - n0
+    launches = (A.fp8mlp_kernel_launch_count() - n0) if g_t is None else kernels_per_step * a.steps
     if dist:
         dist.barrier()
     status = A.fp8mlp_get_device_status()
-    per_kernel = {n: [] for n in names}
-    step_ms = []
-    for ev in evs:
-        for k, n in enumerate(names):
-            per_kernel[n].append(ev[k].elapsed_time(ev[k + 1]))
-        step_ms.append(ev[0].elapsed_time(ev[7]))
     total_s = sum(step_ms) * 1e-3
     if dist:
         t = torch.tensor([total_s], device=dev, dtype=torch.float64)
@@ -336,13 +375,15 @@ def run_ours(a, W, world, rank, local_rank):
         total_s = float(t.item())
     value = M * world * a.steps / total_s
 
-    # roofline of the dominant kernel and of the whole step
+    # roofline of the dominant kernel (timed live inside the timed steps) and
+    # of the whole step
     work = kernel_work(M, d, h)
-    avg = {n: statistics.mean(v) * 1e-3 for n, v in per_kernel.items()}
-    dom = max(avg, key=lambda n: avg[n])
+    avg = {n: v * 1e-3 for n, v in breakdown.items()}
+    dom = names[dom_i]
+    dom_s = statistics.mean(dom_ms) * 1e-3
     wd = work[dom]
     peak_dom = fp8_peak if wd["fp8"] else peaks["bf16_tflops"]
-    achieved = (wd["bf16"] + wd["fp8"]) / avg[dom] / 1e12
+    achieved = (wd["bf16"] + wd["fp8"]) / dom_s / 1e12
     traffic = load_traffic(W.name).get(dom)
     roof_t = 0.0
     for n, w in work.items():
@@ -375,8 +416,10 @@ def run_ours(a, W, world, rank, local_rank):
                               "fwd_frac": fwd_roof / fwd_s, "fwd_tokens_per_s": M / fwd_s,
                               "peaks": {"bf16_tflops": peaks["bf16_tflops"], "fp8_tflops": fp8_peak,
                                         "hbm_gbs": peaks["hbm_gbs"]}},
-            "kernels_ms": {n: statistics.mean(v) for n, v in per_kernel.items()},
+            "kernels_ms": breakdown,
+            "kernels_ms_note": "median of 5 untimed steps with an event between every kernel",
             "clocks": clocks, "gpu_launches": int(launches), "device_status": status,
+            "launch_mode": "eager" if g_t is None else "cuda_graph",
         }
         if e2e:
             line["e2e"] = e2e
@@ -392,14 +435,15 @@ def run_ours(a, W, world, rank, local_rank):
 def measure_e2e(a, blk, P, torch, dev, stream, M, world, dist):
     """Same step through the public API with host buffers: the step's inputs
     (x, dOut) come from pinned host memory and its results (out, dX) go back
-    to pinned host memory inside the timed region."""
+    to pinned host memory inside the timed region (copies and kernels replayed
+    as one CUDA graph per step)."""
     import numpy as np
     xh = torch.from_numpy(P["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
     gh = torch.from_numpy(P["dOut"].view(np.int16)).view(torch.bfloat16).pin_memory()
     oh = torch.empty_like(blk.out, device="cpu").pin_memory()
     dxh = torch.empty_like(blk.dX, device="cpu").pin_memory()
 
-    def step():
+    def body():
         blk.x.copy_(xh, non_blocking=True)
         blk.dOut.copy_(gh, non_blocking=True)
         blk.forward()
@@ -408,6 +452,16 @@ def measure_e2e(a, blk, P, torch, dev, stream, M, world, dist):
         blk.refresh_w2_cache()
         oh.copy_(blk.out, non_blocking=True)
         dxh.copy_(blk.dX, non_blocking=True)
+
+    body()
+    torch.cuda.synchronize()
+    graph = None if a.eager else blk.capture(body)
+
+    def step():
+        if graph is not None:
+            graph.replay()
+        else:
+            body()
 
     for _ in range(max(a.warmup, 3)):
         step()

@@ -78,6 +78,17 @@ class MLPBlock:
         self.backward()
         self.update_scale()
 
+    # ------------------------------------------------------------ CUDA graph
+    def capture(self, fn):
+        """Record the library calls made by ``fn()`` into a CUDA graph and return
+        it (``torch.cuda.CUDAGraph``; ``.replay()`` re-issues them).  The calls
+        bake this block's buffer addresses into the graph, so the buffers must
+        stay alive and in place.  Run ``fn()`` once eagerly before capturing."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        return g
+
     # --------------------------------------------------------------- helpers
     def read_state(self) -> dict:
         s = self.state.cpu()

@@ -115,11 +115,11 @@ int map_tile32(CUtensorMap* m, const void* p, CUtensorMapDataType dt, int esize,
 
 int cdiv(int a, int b) { return (a + b - 1) / b; }
 
-void fill_common(GemmParams& p, const DeviceInfo* di, int M, int N, int K, int groups) {
+void fill_common(GemmParams& p, GemmKind kind, const DeviceInfo* di, int M, int N, int K, int groups) {
   p.M = M;
   p.N = N;
   p.K = K;
-  p.tiles_m = cdiv(M, kGemmBM);
+  p.tiles_m = cdiv(M, gemm_tile_m(kind));
   p.tiles_n = cdiv(N, kGemmBN);
   p.num_groups = groups;
   p.status = di->status;
@@ -179,10 +179,12 @@ extern "C" {
 
 int fp8mlp_partial_amax_shape(int M, int h, int* row_blocks, int* col_blocks, int* block_rows, int* block_cols) {
   if (M < 0 || h < 0) return fail(FP8MLP_ERR_INVALID_ARG, "negative size");
-  if (row_blocks) *row_blocks = 4 * cdiv(M, kGemmBM);
-  if (col_blocks) *col_blocks = cdiv(h, kGemmBN);
+  const int tm = gemm_tile_m(GemmKind::Up);
+  if (row_blocks) *row_blocks = (tm / 32) * cdiv(M, tm);
+  const int pc = up_partial_cols();
+  if (col_blocks) *col_blocks = cdiv(h, kGemmBN) * (kGemmBN / pc);
   if (block_rows) *block_rows = kGemmBM / 4;
-  if (block_cols) *block_cols = kGemmBN;
+  if (block_cols) *block_cols = pc;
   return FP8MLP_OK;
 }
 
@@ -216,10 +218,10 @@ int fp8mlp_up_proj_fused(int M, int d, int h, const uint16_t* x, const uint16_t*
   TRY(current_device(&di));
   GemmParams p{};
   TRY(map_kmajor(&p.tmA[0], x, BF16, 2, M, d, kGemmBM, "x"));
-  TRY(map_kmajor(&p.tmB[0], W1, BF16, 2, h, d, kGemmBN, "W1"));
+  TRY(map_kmajor(&p.tmB[0], W1, BF16, 2, h, d, kGemmBN * kGemmBM / gemm_tile_m(GemmKind::Up), "W1"));
   TRY(map_tile32(&p.tmOut[0], post, BF16, 2, M, h, "post"));
   if (write_q) TRY(map_tile32(&p.tmOut2, post_fp8, U8, 1, M, h, "post_fp8"));
-  fill_common(p, di, M, h, d, 1);
+  fill_common(p, GemmKind::Up, di, M, h, d, 1);
   p.write_q = write_q ? 1 : 0;
   p.partial_amax = partial_amax;
   p.pre_debug = pre_debug;
@@ -242,9 +244,9 @@ int fp8mlp_down_proj_fp8(int M, int d, int h, const uint8_t* post_fp8, const uin
   TRY(current_device(&di));
   GemmParams p{};
   TRY(map_kmajor(&p.tmA[0], post_fp8, U8, 1, M, h, kGemmBM, "post_fp8"));
-  TRY(map_kmajor(&p.tmB[0], W2q_t, U8, 1, d, h, kGemmBN, "W2q_t"));
+  TRY(map_kmajor(&p.tmB[0], W2q_t, U8, 1, d, h, kGemmBN * kGemmBM / gemm_tile_m(GemmKind::Down8), "W2q_t"));
   TRY(map_tile32(&p.tmOut[0], out, BF16, 2, M, d, "out"));
-  fill_common(p, di, M, d, h, 1);
+  fill_common(p, GemmKind::Down8, di, M, d, h, 1);
   p.st = st;
   p.w2_scale_inv = w2_scale_inv;
   return launch(GemmKind::Down8, p, di, stream, "down_proj_fp8 launch");
@@ -264,7 +266,7 @@ int fp8mlp_down_proj_bf16(int M, int d, int h, const uint16_t* post, const uint1
   TRY(map_kmajor(&p.tmA[0], post, BF16, 2, M, h, kGemmBM, "post"));
   TRY(map_mnmajor(&p.tmB[0], W2, h, d, "W2"));
   TRY(map_tile32(&p.tmOut[0], out, BF16, 2, M, d, "out"));
-  fill_common(p, di, M, d, h, 1);
+  fill_common(p, GemmKind::Bf16MnB, di, M, d, h, 1);
   return launch(GemmKind::Bf16MnB, p, di, stream, "down_proj_bf16 launch");
 }
 
@@ -344,10 +346,10 @@ int fp8mlp_bwd_dpre(int M, int d, int h, const uint16_t* dOut, const uint16_t* W
   TRY(current_device(&di));
   GemmParams p{};
   TRY(map_kmajor(&p.tmA[0], dOut, BF16, 2, M, d, kGemmBM, "dOut"));
-  TRY(map_kmajor(&p.tmB[0], W2, BF16, 2, h, d, kGemmBN, "W2"));
+  TRY(map_kmajor(&p.tmB[0], W2, BF16, 2, h, d, kGemmBN * kGemmBM / gemm_tile_m(GemmKind::DPre), "W2"));
   TRY(map_tile32(&p.tmOut[0], dPre, BF16, 2, M, h, "dPre"));
   TRY(map_tile32(&p.tmAux, post, BF16, 2, M, h, "post"));
-  fill_common(p, di, M, h, d, 1);
+  fill_common(p, GemmKind::DPre, di, M, h, d, 1);
   return launch(GemmKind::DPre, p, di, stream, "bwd_dpre launch");
 }
 
@@ -365,7 +367,7 @@ int fp8mlp_bwd_dx(int M, int d, int h, const uint16_t* dPre, const uint16_t* W1,
   TRY(map_kmajor(&p.tmA[0], dPre, BF16, 2, M, h, kGemmBM, "dPre"));
   TRY(map_mnmajor(&p.tmB[0], W1, h, d, "W1"));
   TRY(map_tile32(&p.tmOut[0], dX, BF16, 2, M, d, "dX"));
-  fill_common(p, di, M, d, h, 1);
+  fill_common(p, GemmKind::Bf16MnB, di, M, d, h, 1);
   return launch(GemmKind::Bf16MnB, p, di, stream, "bwd_dx launch");
 }
 
@@ -397,7 +399,7 @@ int fp8mlp_bwd_dw(int M, int d, int h, const uint16_t* x, const uint16_t* dPre, 
   TRY(map_mnmajor(&p.tmA[1], post, M, h, "post"));
   TRY(map_mnmajor(&p.tmB[1], dOut, M, d, "dOut"));
   TRY(map_tile32(&p.tmOut[1], dW2, F32, 4, h, d, "dW2"));
-  fill_common(p, di, h, d, M, 2);
+  fill_common(p, GemmKind::DW, di, h, d, M, 2);
   return launch(GemmKind::DW, p, di, stream, "bwd_dw launch");
 }
 

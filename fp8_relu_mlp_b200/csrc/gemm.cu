@@ -3,11 +3,14 @@
 
 namespace fp8mlp {
 
-using CfgUp = GemmCfg<kGemmBN, 4, false, false, false, Epi::UpFused>;
-using CfgDown8 = GemmCfg<kGemmBN, 4, true, false, false, Epi::DownScaled>;
-using CfgBf16MnB = GemmCfg<kGemmBN, 4, false, false, true, Epi::StoreBf16>;
-using CfgDPre = GemmCfg<kGemmBN, 3, false, false, false, Epi::DPre>;
-using CfgDW = GemmCfg<kGemmBN, 4, false, true, true, Epi::StoreF32>;
+// 2-CTA UMMA (cluster pairs, 256x256 tiles): each SM streams its 128 rows of
+// A and half of B, a third less operand traffic per FLOP than 1-CTA tiles
+using CfgUp = GemmCfg<2, kGemmBN, 5, false, false, false, Epi::UpFused>;
+using CfgDown8 = GemmCfg<2, kGemmBN, 6, true, false, false, Epi::DownScaled>;
+using CfgBf16MnB = GemmCfg<2, kGemmBN, 6, false, false, true, Epi::StoreBf16>;
+using CfgDPre = GemmCfg<2, kGemmBN, 3, false, false, false, Epi::DPre>;
+// dW: one long tile per CTA pair, so a light epilogue (4 warps) and more stages
+using CfgDW = GemmCfg<2, kGemmBN, 6, false, true, true, Epi::StoreF32, 4>;
 
 namespace {
 
@@ -24,14 +27,47 @@ cudaError_t launch_one(const GemmParams& p, int num_tiles, int num_sms, cudaStre
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
   }
-  const int grid = num_tiles < num_sms ? num_tiles : num_sms;
-  if (grid <= 0) return cudaSuccess;
-  gemm_sm100_kernel<C><<<grid, 192, C::SMEM_BYTES, s>>>(p);
+  // persistent: one CTA (pair) per SM (pair), never more than the tiles
+  const int units = num_sms / C::CG;
+  const int pairs = num_tiles < units ? num_tiles : units;
+  if (pairs <= 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pairs * C::CG, 1, 1);
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C::CG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemm_sm100_kernel<C>, p);
   count_launches(1);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 }  // namespace
+
+int up_partial_cols() { return CfgUp::BN / CfgUp::EPI_SPLIT; }
+
+int gemm_tile_m(GemmKind kind) {
+  switch (kind) {
+    case GemmKind::Up:
+      return CfgUp::TILE_M;
+    case GemmKind::Down8:
+      return CfgDown8::TILE_M;
+    case GemmKind::Bf16MnB:
+      return CfgBf16MnB::TILE_M;
+    case GemmKind::DPre:
+      return CfgDPre::TILE_M;
+    case GemmKind::DW:
+      return CfgDW::TILE_M;
+  }
+  return 128;
+}
 
 cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int num_tiles, int num_sms, cudaStream_t s) {
   switch (kind) {

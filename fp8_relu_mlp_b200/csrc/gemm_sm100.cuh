@@ -2,13 +2,16 @@
 //
 //   D[m, n] = sum_k A[m, k] * B[n, k]      (fp32 accumulate in TMEM)
 //
-// One CTA per SM (192 threads):
+// One CTA per SM (320 threads); with CG = 2 the CTAs of a cluster pair share
+// a 2-CTA UMMA over a 256-row tile (each CTA loads its 128 rows of A and half
+// of B; the leader issues the UMMA; each CTA drains its own 128 TMEM lanes):
 //   warp 0      TMA producer: streams A/B k-blocks into a STAGES-deep smem ring
 //   warp 1      allocates 512 TMEM columns (two 256-column accumulators) and
 //               issues the UMMAs from one thread
-//   warps 2..5  epilogue: TMEM -> registers -> fused math -> swizzled smem ->
+//   warps 2..9  epilogue: TMEM -> registers -> fused math -> swizzled smem ->
 //               TMA store, 32 columns at a time; warp w owns TMEM lanes
-//               32*(w%4) .. +31, i.e. tile rows 32*(w%4) .. +31
+//               32*(w%4) .. +31 (tile rows 32*(w%4) .. +31) and one half of
+//               the tile's columns, so two warps share each SM sub-partition
 // The two accumulators let the epilogue of tile i overlap the mainloop of
 // tile i+1.  Operands are BF16 (kind::f16) or e4m3 (kind::f8f6f4), each
 // K-major or MN-major, staged with 128-byte swizzle.  TMA zero-fills rows and
@@ -48,22 +51,27 @@ struct alignas(64) GemmParams {
   int debug_flags;
 };
 
-template <int BN_, int STAGES_, bool FP8_, bool A_MN_, bool B_MN_, Epi EPI_>
+template <int CG_, int BN_, int STAGES_, bool FP8_, bool A_MN_, bool B_MN_, Epi EPI_, int NEPI_ = 8>
 struct GemmCfg {
-  static constexpr int BM = 128;
-  static constexpr int BN = BN_;
+  static constexpr int CG = CG_;           // CTAs per UMMA (1, or 2 = the pair of a cluster)
+  static constexpr int BM = 128;           // accumulator rows per CTA (TMEM lanes)
+  static constexpr int TILE_M = BM * CG;   // rows of one output tile
+  static constexpr int BN = BN_;           // columns of one output tile
+  static constexpr int B_ROWS = BN / CG;   // rows of B (N) each CTA loads
   static constexpr int STAGES = STAGES_;
   static constexpr bool FP8 = FP8_;
   static constexpr bool A_MN = A_MN_;
   static constexpr bool B_MN = B_MN_;
   static constexpr Epi EPI = EPI_;
+  static_assert(CG == 1 || CG == 2, "CTA group");
   static_assert(!(FP8 && (A_MN || B_MN)), "MN-major operands are BF16 only here");
-  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256 && B_ROWS % 64 == 0, "BN");
   static constexpr int ELEM = FP8 ? 1 : 2;
   static constexpr int BK = 128 / ELEM;     // K elements per stage (one 128-byte swizzle row)
   static constexpr int UMMA_K = 32 / ELEM;  // K per UMMA instruction (32 bytes)
   static constexpr int A_BYTES = BM * BK * ELEM;
-  static constexpr int B_BYTES = BN * BK * ELEM;
+  static constexpr int B_BYTES = B_ROWS * BK * ELEM;
+  static constexpr int STAGE_TX = CG * (A_BYTES + B_BYTES);  // bytes landing on the leader's barrier per stage
   // descriptor strides: K-major: 8-row groups 1024 B apart (LBO unused);
   // MN-major: 64-element MN atoms BK*128 B apart (LBO), 8-k-row groups 1024 B apart
   static constexpr uint32_t A_LBO = A_MN ? BK * 128 : 16;
@@ -71,10 +79,15 @@ struct GemmCfg {
   static constexpr uint32_t SBO = 1024;
   static constexpr uint32_t A_KSTEP = A_MN ? UMMA_K * 128 : UMMA_K * ELEM;
   static constexpr uint32_t B_KSTEP = B_MN ? UMMA_K * 128 : UMMA_K * ELEM;
-  static constexpr uint32_t IDESC =
-      dev::instr_desc(FP8 ? dev::FMT_E4M3 : dev::FMT_BF16, FP8 ? dev::FMT_E4M3 : dev::FMT_BF16, A_MN, B_MN, BM, BN);
+  static constexpr uint32_t IDESC = dev::instr_desc(FP8 ? dev::FMT_E4M3 : dev::FMT_BF16,
+                                                    FP8 ? dev::FMT_E4M3 : dev::FMT_BF16, A_MN, B_MN, TILE_M, BN);
   static constexpr int ECOLS = 32;
-  static constexpr int NCHUNK = BN / ECOLS;
+  static constexpr int NCHUNK = BN / ECOLS;      // 32-column chunks per tile row block
+  static constexpr int NEPI = NEPI_;             // epilogue warps: NEPI/4 per TMEM lane quarter
+  static constexpr int EPI_SPLIT = NEPI / 4;     // column groups per lane quarter
+  static constexpr int NCH_W = NCHUNK / EPI_SPLIT;  // chunks per epilogue warp per tile
+  static constexpr int THREADS = 64 + 32 * NEPI;
+  static_assert(NEPI % 4 == 0 && NCHUNK % EPI_SPLIT == 0, "chunks per warp");
   static constexpr int OUT_BUF = 32 * ECOLS * (EPI == Epi::StoreF32 ? 4 : 2);
   static constexpr int OUT2_BUF = EPI == Epi::UpFused ? 32 * ECOLS : 0;
   static constexpr int SLOT = OUT_BUF + OUT2_BUF;  // one output staging slot (two per epilogue warp)
@@ -82,13 +95,13 @@ struct GemmCfg {
   // DPre: each epilogue warp keeps the post block of a whole tile (NCHUNK
   // chunks of 32x32) in its own ring, loaded one tile ahead
   static constexpr int AUX_CHUNK = EPI == Epi::DPre ? 32 * ECOLS * 2 : 0;
-  static constexpr int AUX_WARP = AUX_CHUNK * NCHUNK;
-  static constexpr int NAUX = EPI == Epi::DPre ? NCHUNK : 0;
+  static constexpr int AUX_WARP = AUX_CHUNK * NCH_W;
+  static constexpr int NAUX = EPI == Epi::DPre ? NCH_W : 0;
   static constexpr int TMEM_COLS = 512;
   static_assert(2 * BN <= TMEM_COLS, "two accumulators");
-  static constexpr int NUM_BARS = 2 * STAGES + 4 + 4 * NAUX + 1;
-  static constexpr int SMEM_BYTES =
-      1024 /*alignment slack*/ + STAGES * (A_BYTES + B_BYTES) + 8 * SLOT + 4 * AUX_WARP + NUM_BARS * 8 + 16;
+  static constexpr int NUM_BARS = 2 * STAGES + 4 + NEPI * NAUX + 1;
+  static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * (A_BYTES + B_BYTES) + 2 * NEPI * SLOT +
+                                    NEPI * AUX_WARP + NUM_BARS * 8 + 16;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
@@ -113,27 +126,32 @@ __device__ __forceinline__ void store_row_bf16(uint32_t base, int lane, const ui
 }  // namespace dev
 
 template <class C>
-__global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_constant__ GemmParams p) {
   using namespace dev;
+  constexpr int CG = C::CG;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   uint8_t* sA = smem;
   uint8_t* sB = sA + C::STAGES * C::A_BYTES;
   uint8_t* sEpi = sB + C::STAGES * C::B_BYTES;
-  uint8_t* sAux = sEpi + 8 * C::SLOT;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sAux + 4 * C::AUX_WARP);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + C::STAGES;
+  uint8_t* sAux = sEpi + 2 * C::NEPI * C::SLOT;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sAux + C::NEPI * C::AUX_WARP);
+  uint64_t* full = bars;                // [STAGES] (the leader's are used)
+  uint64_t* empty = bars + C::STAGES;   // [STAGES]
   uint64_t* tfull = bars + 2 * C::STAGES;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* auxb = tempty + 2;  // [4 warps][NAUX chunks]
-  uint64_t* fin = auxb + 4 * C::NAUX;
+  uint64_t* tempty = tfull + 2;         // the leader's count both CTAs' epilogues
+  uint64_t* auxb = tempty + 2;          // [NEPI warps][NAUX chunks]
+  uint64_t* fin = auxb + C::NEPI * C::NAUX;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(fin + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;  // position in the CTA pair
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(blockIdx.x) / CG;
+  const int npairs = static_cast<int>(gridDim.x) / CG;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -142,19 +160,20 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 32 * C::NEPI * CG);
     }
-    for (int i = 0; i < 4 * C::NAUX; ++i) mbar_init(&auxb[i], 1);
+    for (int i = 0; i < C::NEPI * C::NAUX; ++i) mbar_init(&auxb[i], 1);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, C::TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc<CG>(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish<CG>();
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (CG == 2) cluster_sync();  // the peer's barriers are initialised
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const WaitCtx w{p.status, abort_flag, p.timeout_ns};
@@ -172,11 +191,11 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
       }
       uint32_t stage = 0, phase = 0;
       long long issued = 0;
-      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      for (int t = pair; t < num_tiles; t += npairs) {
         const int g = t / tiles_per_group;
         const int tt = t - g * tiles_per_group;
-        const int m0 = (tt / p.tiles_n) * C::BM;
-        const int n0 = (tt % p.tiles_n) * C::BN;
+        const int m0 = (tt / p.tiles_n) * C::TILE_M + static_cast<int>(rank) * C::BM;  // this CTA's A rows
+        const int n0 = (tt % p.tiles_n) * C::BN + static_cast<int>(rank) * C::B_ROWS;  // this CTA's B rows
         const CUtensorMap* mA = &p.tmA[g];
         const CUtensorMap* mB = &p.tmB[g];
         bool ok = true;
@@ -185,21 +204,40 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES);
           uint8_t* a = sA + stage * C::A_BYTES;
           uint8_t* b = sB + stage * C::B_BYTES;
           const int k0 = kb * C::BK;
-          if constexpr (C::A_MN) {
+          if constexpr (CG == 1) {
+            mbar_arrive_expect_tx(&full[stage], C::STAGE_TX);
+            if constexpr (C::A_MN) {
 #pragma unroll
-            for (int i = 0; i < C::BM / 64; ++i) tma_load_2d(a + i * C::BK * 128, mA, &full[stage], m0 + i * 64, k0);
-          } else {
-            tma_load_2d(a, mA, &full[stage], k0, m0);
-          }
-          if constexpr (C::B_MN) {
+              for (int i = 0; i < C::BM / 64; ++i) tma_load_2d(a + i * C::BK * 128, mA, &full[stage], m0 + i * 64, k0);
+            } else {
+              tma_load_2d(a, mA, &full[stage], k0, m0);
+            }
+            if constexpr (C::B_MN) {
 #pragma unroll
-            for (int i = 0; i < C::BN / 64; ++i) tma_load_2d(b + i * C::BK * 128, mB, &full[stage], n0 + i * 64, k0);
+              for (int i = 0; i < C::B_ROWS / 64; ++i)
+                tma_load_2d(b + i * C::BK * 128, mB, &full[stage], n0 + i * 64, k0);
+            } else {
+              tma_load_2d(b, mB, &full[stage], k0, n0);
+            }
           } else {
-            tma_load_2d(b, mB, &full[stage], k0, n0);
+            // both CTAs' copies complete on the leader's full barrier
+            if (leader) mbar_arrive_expect_tx(&full[stage], C::STAGE_TX);
+            const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+            if constexpr (C::A_MN) {
+#pragma unroll
+              for (int i = 0; i < C::BM / 64; ++i) tma_load_2d_cg2(a + i * C::BK * 128, mA, fb, m0 + i * 64, k0);
+            } else {
+              tma_load_2d_cg2(a, mA, fb, k0, m0);
+            }
+            if constexpr (C::B_MN) {
+#pragma unroll
+              for (int i = 0; i < C::B_ROWS / 64; ++i) tma_load_2d_cg2(b + i * C::BK * 128, mB, fb, n0 + i * 64, k0);
+            } else {
+              tma_load_2d_cg2(b, mB, fb, k0, n0);
+            }
           }
           ++issued;
           if (++stage == C::STAGES) {
@@ -209,18 +247,21 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
         }
         if (!ok) break;
       }
-      // drain: the last issue into each stage must have landed before exit
-      const long long n_drain = issued < C::STAGES ? issued : C::STAGES;
-      for (long long i = 0; i < n_drain; ++i) {
-        const long long n = issued - 1 - i;
-        mbar_wait_drain(&full[n % C::STAGES], static_cast<uint32_t>((n / C::STAGES) & 1), p.timeout_ns);
+      // drain: the last copy into each stage must have landed before exit
+      // (the leader's barrier sees both CTAs' copies)
+      if (leader) {
+        const long long n_drain = issued < C::STAGES ? issued : C::STAGES;
+        for (long long i = 0; i < n_drain; ++i) {
+          const long long n = issued - 1 - i;
+          mbar_wait_drain(&full[n % C::STAGES], static_cast<uint32_t>((n / C::STAGES) & 1), p.timeout_ns);
+        }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (the pair's leader)
+    if (lane == 0 && leader) {
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
-      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      for (int t = pair; t < num_tiles; t += npairs) {
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, w)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * C::BN;
@@ -237,33 +278,43 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
           for (int k = 0; k < C::BK / C::UMMA_K; ++k) {
             const uint64_t ad = smem_desc(a0 + k * C::A_KSTEP, C::A_LBO, C::SBO);
             const uint64_t bd = smem_desc(b0 + k * C::B_KSTEP, C::B_LBO, C::SBO);
-            const uint32_t accum = (kb | k) != 0;
-            if constexpr (C::FP8)
-              umma_f8(d_tmem, ad, bd, C::IDESC, accum);
-            else
-              umma_f16(d_tmem, ad, bd, C::IDESC, accum);
+            umma<CG, C::FP8>(d_tmem, ad, bd, C::IDESC, (kb | k) != 0 ? 1u : 0u);
           }
-          tc_commit(&empty[stage]);
+          if constexpr (CG == 1)
+            tc_commit(&empty[stage]);
+          else
+            tc_commit_cg2_mc(&empty[stage], 0x3);  // frees the stage in both CTAs
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(&tfull[acc]);
+        if constexpr (CG == 1)
+          tc_commit(&tfull[acc]);
+        else
+          tc_commit_cg2_mc(&tfull[acc], 0x3);  // accumulator ready in both CTAs
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
       // every UMMA this thread issued must be complete before TMEM is freed
-      tc_commit(fin);
+      if constexpr (CG == 1)
+        tc_commit(fin);
+      else
+        tc_commit_cg2(fin);
       mbar_wait_drain(fin, 0, p.timeout_ns);
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter == row block of 32 within the tile
+    const int q = warp & 3;  // TMEM lane quarter == row block of 32 within this CTA's rows
+    const int e = warp - 2;  // epilogue warp index
+    const int half = e / 4;  // which column group of the tile this warp drains (< EPI_SPLIT)
+    const int c_begin = half * C::NCH_W;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    // arrivals that free an accumulator go to the leader's barrier
+    const uint32_t tempty_addr0 = CG == 2 ? mapa_shared(smem_u32(&tempty[0]), 0) : 0u;
     uint32_t acc = 0, acc_phase = 0, ctr = 0;
     float s_up = 0.f, comb = 1.f;
     if constexpr (C::EPI == Epi::UpFused) {
@@ -273,50 +324,56 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
     // DPre: rounds of post prefetch started (one round = a tile's NAUX chunks,
     // ring slot c = chunk c) and how many slots the latest round has reached
     uint32_t aux_rounds = 0, aux_last = 0;
-    uint8_t* aux_ring = sAux + q * C::AUX_WARP;
-    auto issue_post_tile = [&](int tile) {
-      if constexpr (C::EPI == Epi::DPre) {
-        const int g2 = tile / tiles_per_group;
-        const int t2 = tile - g2 * tiles_per_group;
-        const int r0 = (t2 / p.tiles_n) * C::BM + q * 32;
-        const int c0 = (t2 % p.tiles_n) * C::BN;
-        for (int c = 0; c < C::NAUX; ++c) {
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&auxb[q * C::NAUX + c], C::AUX_CHUNK);
-            tma_load_2d(aux_ring + c * C::AUX_CHUNK, &p.tmAux, &auxb[q * C::NAUX + c], c0 + c * C::ECOLS, r0);
+    uint8_t* aux_ring = sAux + e * C::AUX_WARP;
+    uint64_t* my_auxb = auxb + e * C::NAUX;
+    auto tile_rows = [&](int tile) {  // first row of this warp's 32 rows in `tile`
+      const int tt2 = tile - (tile / tiles_per_group) * tiles_per_group;
+      return (tt2 / p.tiles_n) * C::TILE_M + static_cast<int>(rank) * C::BM + q * 32;
+    };
+    auto tile_cols = [&](int tile) {
+      const int tt2 = tile - (tile / tiles_per_group) * tiles_per_group;
+      return (tt2 % p.tiles_n) * C::BN;
+    };
+    if constexpr (C::EPI == Epi::DPre) {
+      if (pair < num_tiles) {
+        const int r0 = tile_rows(pair), c0 = tile_cols(pair);
+        if (lane == 0) {
+          for (int c = 0; c < C::NAUX; ++c) {
+            mbar_arrive_expect_tx(&my_auxb[c], C::AUX_CHUNK);
+            tma_load_2d(aux_ring + c * C::AUX_CHUNK, &p.tmAux, &my_auxb[c], c0 + (c_begin + c) * C::ECOLS, r0);
           }
         }
         aux_rounds = 1;
         aux_last = C::NAUX;
       }
-    };
-    uint32_t iter = 0;  // tiles processed by this CTA
-    if constexpr (C::EPI == Epi::DPre) {
-      if (static_cast<int>(blockIdx.x) < num_tiles) issue_post_tile(blockIdx.x);
     }
+    uint32_t iter = 0;  // tiles processed by this CTA
 
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+    for (int t = pair; t < num_tiles; t += npairs) {
       const int g = t / tiles_per_group;
       const int tt = t - g * tiles_per_group;
       const int mb = tt / p.tiles_n, nb = tt % p.tiles_n;
-      const int m0 = mb * C::BM, n0 = nb * C::BN;
-      const int row0 = m0 + q * 32;
-
-      const int next_tile = t + static_cast<int>(gridDim.x);
+      const int row0 = tile_rows(t);
+      const int n0 = nb * C::BN;
+      const int next_tile = t + npairs;
       if (!mbar_wait(&tfull[acc], acc_phase, w)) break;
       tc_fence_after();
       float tmax = 0.f;
       bool ok = true;
 #pragma unroll 1
-      for (int c = 0; c < C::NCHUNK; ++c) {
+      for (int cw = 0; cw < C::NCH_W; ++cw) {
+        const int c = c_begin + cw;  // chunk within the tile
         uint32_t v[32];
         tmem_ld32(tmem_base + lane_base + acc * C::BN + c * C::ECOLS, v);
-        if (c == C::NCHUNK - 1) {
+        if (cw == C::NCH_W - 1) {
           tc_fence_before();
-          mbar_arrive(&tempty[acc]);
+          if constexpr (CG == 1)
+            mbar_arrive(&tempty[acc]);
+          else
+            mbar_arrive_cluster(tempty_addr0 + acc * 8u);
         }
         const uint32_t b = ctr & 1u;
-        uint8_t* slot = sEpi + (q * 2 + b) * C::SLOT;
+        uint8_t* slot = sEpi + (e * 2 + b) * C::SLOT;
         const uint32_t sbase = smem_u32(slot);
         if (lane == 0) bulk_wait_read<1>();  // the store issued from this slot two chunks ago has read it
         __syncwarp();
@@ -332,16 +389,16 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
             tmax = fmaxf(tmax, fmaxf(sa, sb));
             pk[i] = pack_bf16x2(sa, sb);
           }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint32_t q0 = pack_e4m3x2(__fmul_rn(bf16lo_to_f32(pk[2 * i]), s_up),
-                                            __fmul_rn(bf16hi_to_f32(pk[2 * i]), s_up));
-            const uint32_t q1 = pack_e4m3x2(__fmul_rn(bf16lo_to_f32(pk[2 * i + 1]), s_up),
-                                            __fmul_rn(bf16hi_to_f32(pk[2 * i + 1]), s_up));
-            qk[i] = q0 | (q1 << 16);
-          }
           store_row_bf16<64>(sbase, lane, pk);
           if (p.write_q) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint32_t q0 = pack_e4m3x2(__fmul_rn(bf16lo_to_f32(pk[2 * i]), s_up),
+                                              __fmul_rn(bf16hi_to_f32(pk[2 * i]), s_up));
+              const uint32_t q1 = pack_e4m3x2(__fmul_rn(bf16lo_to_f32(pk[2 * i + 1]), s_up),
+                                              __fmul_rn(bf16hi_to_f32(pk[2 * i + 1]), s_up));
+              qk[i] = q0 | (q1 << 16);
+            }
             const uint32_t qb = sbase + C::OUT_BUF;
 #pragma unroll
             for (int j = 0; j < 2; ++j)
@@ -370,10 +427,10 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
           store_row_bf16<64>(sbase, lane, pk);
         } else if constexpr (C::EPI == Epi::DPre) {
           // post of this chunk was loaded one tile ahead into ring slot c
-          if (!mbar_wait(&auxb[q * C::NAUX + c], iter & 1u, w)) {
+          if (!mbar_wait(&my_auxb[cw], iter & 1u, w)) {
             ok = false;
           } else {
-            const uint32_t ab = smem_u32(aux_ring + c * C::AUX_CHUNK);
+            const uint32_t ab = smem_u32(aux_ring + cw * C::AUX_CHUNK);
             uint32_t pp[16], pk[16];
 #pragma unroll
             for (int j = 0; j < 4; ++j)
@@ -381,15 +438,13 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
             __syncwarp();
             // ring slot c is free again: fetch the next tile's chunk c into it
             if (next_tile < num_tiles) {
-              const int g2 = next_tile / tiles_per_group;
-              const int t2 = next_tile - g2 * tiles_per_group;
               if (lane == 0) {
-                mbar_arrive_expect_tx(&auxb[q * C::NAUX + c], C::AUX_CHUNK);
-                tma_load_2d(aux_ring + c * C::AUX_CHUNK, &p.tmAux, &auxb[q * C::NAUX + c],
-                            (t2 % p.tiles_n) * C::BN + c * C::ECOLS, (t2 / p.tiles_n) * C::BM + q * 32);
+                mbar_arrive_expect_tx(&my_auxb[cw], C::AUX_CHUNK);
+                tma_load_2d(aux_ring + cw * C::AUX_CHUNK, &p.tmAux, &my_auxb[cw],
+                            tile_cols(next_tile) + c * C::ECOLS, tile_rows(next_tile));
               }
-              if (c == 0) aux_rounds = iter + 2;
-              aux_last = c + 1;
+              if (cw == 0) aux_rounds = iter + 2;
+              aux_last = cw + 1;
             }
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -420,7 +475,9 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
       if constexpr (C::EPI == Epi::UpFused) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
-        if (lane == 0) p.partial_amax[(mb * 4 + q) * p.tiles_n + nb] = round_bf16(tmax);
+        if (lane == 0)
+          p.partial_amax[((mb * CG + static_cast<int>(rank)) * 4 + q) * (p.tiles_n * C::EPI_SPLIT) +
+                         nb * C::EPI_SPLIT + half] = round_bf16(tmax);
       }
       if (++acc == 2) {
         acc = 0;
@@ -433,7 +490,7 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
         // the last load issued into each ring slot must have landed before exit
         for (int c = 0; c < C::NAUX; ++c) {
           const uint32_t n = static_cast<uint32_t>(c) < aux_last ? aux_rounds : aux_rounds - 1u;
-          if (n > 0) mbar_wait_drain(&auxb[q * C::NAUX + c], (n - 1u) & 1u, p.timeout_ns);
+          if (n > 0) mbar_wait_drain(&my_auxb[c], (n - 1u) & 1u, p.timeout_ns);
         }
       }
       bulk_wait<0>();
@@ -441,11 +498,15 @@ __global__ void __launch_bounds__(192, 1) gemm_sm100_kernel(const __grid_constan
     __syncwarp();
   }
 
+  __syncwarp();
   __syncthreads();
+  // no CTA of a pair leaves while its peer may still read its shared memory
+  // or arrive on its barriers; TMEM is freed by both CTAs together
+  if constexpr (CG == 2) cluster_sync();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    tmem_dealloc<CG>(tmem_base, C::TMEM_COLS);
   }
 }
 

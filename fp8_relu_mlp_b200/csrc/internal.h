@@ -17,8 +17,13 @@ enum class GemmKind : int {
   DPre = 3,     // K5: dOut . W2^T -> dPre with the 2 sqrt(post) epilogue
   DW = 4,       // K7/K8: dPre^T . x and post^T . dOut (BF16, MN-major A/B), fp32 out
 };
-constexpr int kGemmBM = 128;
-constexpr int kGemmBN = 256;
+constexpr int kGemmBM = 128;  // accumulator rows per CTA
+constexpr int kGemmBN = 256;  // output tile columns
+
+// rows of one output tile of `kind` (128 per CTA times the CTA-group size)
+int gemm_tile_m(GemmKind kind);
+// columns of post covered by one partial-amax entry
+int up_partial_cols();
 
 struct DeviceInfo {
   int device = -1;

@@ -114,10 +114,11 @@ typedef struct fp8mlp_scale_state {
  *
  *   post[m,i]     = bf16( fp32(r*r) ),  r = max(fp32(x[m,:] . W1[i,:]), 0)
  *   post_fp8[m,i] = e4m3_satfinite( fp32(post[m,i] * st->scale) )
- *   partial_amax  = max of post over blocks of 32 rows x 256 columns,
- *                   fp32, laid out [4*ceil(M/128)][ceil(h/256)]; blocks
- *                   that lie wholly past row M hold 0
- *                   (see fp8mlp_partial_amax_shape)
+ *   partial_amax  = max of post over blocks of block_rows x block_cols
+ *                   (32 x 128), fp32, row-major [row_blocks][col_blocks]
+ *                   with the sizes of fp8mlp_partial_amax_shape
+ *                   (8*ceil(M/256) x 2*ceil(h/256)); blocks that lie
+ *                   wholly past row M or column h hold 0
  *   pre_debug     = optional fp32 pre [M,h] (NULL to skip; slow, for tests)
  *
  * st->scale is read on the device; the host never waits for it.
