@@ -56,6 +56,7 @@ _SIGS = {
     "fp8mlp_scale_state_init": [_p, _f, _f, _p],
     "fp8mlp_amax_reduce_update_scale": [_p, _i, _p, _p],
     "fp8mlp_w2_fp8_cache_refresh": [_i, _i, _p, _p, _p, _p, _p],
+    "fp8mlp_w2_fp8_cache_refresh_noalloc": [_i, _i, _p, _p, _p, _p],
     "fp8mlp_bwd_dpre": [_i, _i, _i, _p, _p, _p, _p, _p],
     "fp8mlp_bwd_dx": [_i, _i, _i, _p, _p, _p, _p],
     "fp8mlp_bwd_dw": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p],
@@ -169,6 +170,13 @@ def fp8mlp_amax_reduce_update_scale(partial_amax, n, st, stream=None):
 
 def fp8mlp_w2_fp8_cache_refresh(h, d, W2, W2q_t, w2_scale_inv, workspace, stream=None):
     return _call("fp8mlp_w2_fp8_cache_refresh", h, d, _ptr(W2), _ptr(W2q_t), _ptr(w2_scale_inv), _ptr(workspace),
+                 _stream(stream))
+
+
+def fp8mlp_w2_fp8_cache_refresh_noalloc(h, d, W2, W2q_t, w2_scale_inv, stream=None):
+    """W2 cache refresh without a workspace: for callers that cannot hand the
+    library device memory (see include/fp8mlp.h)."""
+    return _call("fp8mlp_w2_fp8_cache_refresh_noalloc", h, d, _ptr(W2), _ptr(W2q_t), _ptr(w2_scale_inv),
                  _stream(stream))
 
 

@@ -137,6 +137,8 @@ int launch(GemmKind k, const GemmParams& p, const DeviceInfo* di, cudaStream_t s
 
 void count_launches(unsigned long long n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
+void set_error_detail(const char* what) { g_detail = what; }
+
 int current_device(DeviceInfo** info) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);

@@ -48,6 +48,9 @@ cudaError_t launch_rmsnorm_bwd(int M, int d, const uint16_t* r, const float* rst
 cudaError_t launch_residual_add(int M, int d, const uint16_t* r, const uint16_t* out, uint16_t* r_next,
                                 int num_sms, cudaStream_t s);
 
+// set the text returned by fp8mlp_last_error_detail() on this thread
+void set_error_detail(const char* what);
+
 // number of kernels this library has launched (all devices, all threads)
 void count_launches(unsigned long long n);
 

@@ -200,6 +200,28 @@ int fp8mlp_amax_reduce_update_scale(const float* partial_amax, int n, fp8mlp_sca
 int fp8mlp_w2_fp8_cache_refresh(int h, int d, const uint16_t* W2, uint8_t* W2q_t, float* w2_scale_inv,
                                 void* workspace, fp8mlp_stream_t stream);
 
+/*
+ * The same refresh for callers that cannot allocate device memory.  The paper
+ * has no counterpart: this entry point exists for integration only.  Some
+ * callers cannot provide a workspace: code inside another framework's
+ * operator hook that owns every device allocation through its own pool and
+ * exposes none to the op, or a runtime that forbids cudaMalloc/cudaFree on its
+ * hot path because they can synchronise the whole device.  Results equal
+ * fp8mlp_w2_fp8_cache_refresh's bit for bit.
+ *   - Scratch: a fixed 8 KiB device array owned by the library (2048 partial
+ *     maxima, one per 8192 elements of W2); every GPU that loads the library
+ *     holds it until the process exits.  h*d above 16,777,216 elements is
+ *     rejected with FP8MLP_ERR_UNSUPPORTED_SHAPE (use the workspace version).
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents; no
+ *     entry needs to start at zero (each call writes every entry it reads).
+ *     Calls that overlap on the GPU (other streams, other host threads) race.
+ *   - No cudaMalloc, cudaFree or other allocating call is made.
+ */
+int fp8mlp_w2_fp8_cache_refresh_noalloc(int h, int d, const uint16_t* W2, uint8_t* W2q_t, float* w2_scale_inv,
+                                        fp8mlp_stream_t stream);
+
 /* Device workspace in bytes needed by the calls that take one. */
 size_t fp8mlp_workspace_size(int M, int d, int h);
 
