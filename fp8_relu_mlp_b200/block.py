@@ -101,3 +101,50 @@ class MLPBlock:
         """numpy uint16 BF16 bit patterns -> torch bf16 device tensor."""
         import numpy as np
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+class MLPStack:
+    """L residual layers of ``r_{l+1} = r_l + MLP_l(RMSNorm(r_l))`` (the 9-layer,
+    768-dim ReLU^2 stacks of the nanochat runs), forward and backward, all
+    through the C ABI.  Each layer keeps its own block buffers (post, x, its
+    delayed-scale state and W2 cache); the residual stream r_l and the RMSNorm
+    statistics are kept per layer for the backward."""
+
+    def __init__(self, L: int, M: int, d: int, h: int, device="cuda", margin: float = 2.0,
+                 initial_scale: float = 1.0, stream=None):
+        self.L, self.M, self.d, self.h = L, M, d, h
+        self.device = torch.device(device)
+        self.stream = stream
+        self.blocks = [MLPBlock(M, d, h, device, margin, initial_scale, stream=stream) for _ in range(L)]
+        self.r = [torch.zeros(M, d, dtype=torch.bfloat16, device=self.device) for _ in range(L + 1)]
+        self.rstd = [torch.empty(M, dtype=torch.float32, device=self.device) for _ in range(L)]
+        self.dr = torch.zeros(M, d, dtype=torch.bfloat16, device=self.device)
+
+    def refresh_w2_caches(self):
+        for b in self.blocks:
+            b.refresh_w2_cache()
+
+    def calibrate(self):
+        for l, b in enumerate(self.blocks):
+            A.fp8mlp_rmsnorm_fwd(self.M, self.d, self.r[l], b.x, self.rstd[l], self.stream)
+            b.calibrate()
+            b.forward()
+            A.fp8mlp_residual_add(self.M, self.d, self.r[l], b.out, self.r[l + 1], self.stream)
+
+    def forward(self):
+        for l, b in enumerate(self.blocks):
+            A.fp8mlp_rmsnorm_fwd(self.M, self.d, self.r[l], b.x, self.rstd[l], self.stream)
+            b.forward()
+            A.fp8mlp_residual_add(self.M, self.d, self.r[l], b.out, self.r[l + 1], self.stream)
+
+    def backward(self):
+        """``self.dr`` holds dL/dr_L on entry and dL/dr_0 on exit."""
+        M, d, h = self.M, self.d, self.h
+        for l in range(self.L - 1, -1, -1):
+            b = self.blocks[l]
+            A.fp8mlp_mlp_bwd(M, d, h, b.x, b.W1, b.W2, b.post, self.dr, b.dPre, b.dX, b.dW1, b.dW2, self.stream)
+            A.fp8mlp_rmsnorm_bwd(M, d, self.r[l], self.rstd[l], b.dX, self.dr, self.dr, self.stream)
+
+    def update_scales(self):
+        for b in self.blocks:
+            b.update_scale()

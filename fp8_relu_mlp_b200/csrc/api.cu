@@ -192,9 +192,11 @@ int fp8mlp_partial_amax_shape(int M, int h, int* row_blocks, int* col_blocks, in
 
 size_t fp8mlp_workspace_size(int M, int d, int h) {
   (void)M;
-  (void)d;
-  (void)h;
-  return 256;
+  if (d <= 0 || h <= 0) return 256;
+  // W2 cache refresh: one 4-byte partial maximum per kW2ElemsPerBlock elements
+  const long long n = static_cast<long long>(h) * d;
+  const size_t need = 4 * static_cast<size_t>((n + kW2ElemsPerBlock - 1) / kW2ElemsPerBlock);
+  return need < 256 ? 256 : ((need + 255) / 256) * 256;
 }
 
 int fp8mlp_up_proj_fused(int M, int d, int h, const uint16_t* x, const uint16_t* W1, const fp8mlp_scale_state* st,

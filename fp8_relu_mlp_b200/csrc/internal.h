@@ -39,8 +39,11 @@ cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int num_tiles, int n
 // small kernels
 cudaError_t launch_state_init(fp8mlp_scale_state* st, float margin, float s0, cudaStream_t s);
 cudaError_t launch_amax_scale(const float* pa, int n, fp8mlp_scale_state* st, unsigned int* status, cudaStream_t s);
+// the W2 cache refresh reduces |W2| in blocks of kW2ElemsPerBlock elements,
+// one partial maximum per block in the caller's workspace
+constexpr int kW2ElemsPerBlock = 8192;
 cudaError_t launch_w2_cache(int h, int d, const uint16_t* W2, uint8_t* W2q_t, float* w2_scale_inv,
-                            unsigned int* amax_word, unsigned int* status, int num_sms, cudaStream_t s);
+                            unsigned int* partial, unsigned int* status, int num_sms, cudaStream_t s);
 cudaError_t launch_rmsnorm_fwd(int M, int d, const uint16_t* r, uint16_t* x, float* rstd, int num_sms,
                                cudaStream_t s);
 cudaError_t launch_rmsnorm_bwd(int M, int d, const uint16_t* r, const float* rstd, const uint16_t* dx,

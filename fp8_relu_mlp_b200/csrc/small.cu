@@ -35,12 +35,20 @@ __global__ void __launch_bounds__(1024) amax_scale_kernel(const float* __restric
   __shared__ int snan[32];
   float m = 0.f;
   int nan = 0;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const float v = pa[i];
-    if (v != v)
-      nan = 1;
-    else
-      m = fmaxf(m, v);
+  // eight independent loads in flight per thread per round (the partials are
+  // a few thousand floats: latency, not bandwidth, is the cost)
+  for (int base = 0; base < n; base += 8 * 1024) {
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = base + k * 1024 + threadIdx.x;
+      v[k] = i < n ? __ldg(pa + i) : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      nan |= (v[k] != v[k]);
+      m = fmaxf(m, v[k]);
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -83,22 +91,36 @@ __global__ void __launch_bounds__(1024) amax_scale_kernel(const float* __restric
 }
 
 // max |W2| over BF16 bit patterns: the magnitude bits order like the values
-// (NaN patterns above infinity), so an integer max is exact.
-__global__ void w2_amax_kernel(const uint4* __restrict__ W, size_t n_vec, unsigned int* amax_word) {
+// (NaN patterns above infinity), so an integer max is exact.  Block b covers
+// elements [b*kW2ElemsPerBlock, (b+1)*kW2ElemsPerBlock) and writes its max to
+// partial[b]; the quantising kernel reduces the partials.
+__global__ void __launch_bounds__(256) w2_amax_kernel(const uint4* __restrict__ W, long long n_vec,
+                                                      unsigned int* __restrict__ partial) {
+  __shared__ unsigned int wmax[8];
+  const long long base = static_cast<long long>(blockIdx.x) * (kW2ElemsPerBlock / 8);
   unsigned int m = 0;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n_vec;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const uint4 v = W[i];
-    const unsigned int w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      m = max(m, w4[k] & 0x7FFFu);
-      m = max(m, (w4[k] >> 16) & 0x7FFFu);
+  for (int k = 0; k < kW2ElemsPerBlock / 8 / 256; ++k) {
+    const long long i = base + k * 256 + threadIdx.x;
+    if (i < n_vec) {
+      const uint4 v = W[i];
+      const unsigned int w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        m = max(m, w4[j] & 0x7FFFu);
+        m = max(m, (w4[j] >> 16) & 0x7FFFu);
+      }
     }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((threadIdx.x & 31) == 0 && m != 0) atomicMax(amax_word, m);
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned int r = 0;
+    for (int w = 0; w < 8; ++w) r = max(r, wmax[w]);
+    partial[blockIdx.x] = r;
+  }
 }
 
 __device__ __forceinline__ float w2_scale_from(unsigned int amax_bits, bool* degenerate) {
@@ -114,12 +136,22 @@ __device__ __forceinline__ float w2_scale_from(unsigned int amax_bits, bool* deg
 // W2q_t[j, i] = e4m3(W2[i, j] * s_w); 64x64 tiles through shared memory.
 __global__ void __launch_bounds__(256) w2_quant_t_kernel(int h, int d, const uint16_t* __restrict__ W2,
                                                          uint8_t* __restrict__ W2q_t, float* w2_scale_inv,
-                                                         const unsigned int* amax_word, unsigned int* status) {
+                                                         const unsigned int* __restrict__ partial, int nparts,
+                                                         unsigned int* status) {
   __shared__ float tile[64][65];
+  __shared__ unsigned int wmax[8];
   const int i0 = blockIdx.y * 64;  // rows of W2 (h)
   const int j0 = blockIdx.x * 64;  // cols of W2 (d)
+  unsigned int am = 0;
+  for (int i = threadIdx.x; i < nparts; i += 256) am = max(am, partial[i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, o));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = am;
+  __syncthreads();
+  am = 0;
+  for (int w = 0; w < 8; ++w) am = max(am, wmax[w]);
   bool degenerate;
-  const float s_w = w2_scale_from(*amax_word, &degenerate);
+  const float s_w = w2_scale_from(am, &degenerate);
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
     w2_scale_inv[0] = __fdiv_rn(1.f, s_w);
     if (degenerate) atomicOr(status, STATUS_W2_DEGENERATE);
@@ -262,17 +294,16 @@ cudaError_t launch_amax_scale(const float* pa, int n, fp8mlp_scale_state* st, un
 }
 
 cudaError_t launch_w2_cache(int h, int d, const uint16_t* W2, uint8_t* W2q_t, float* w2_scale_inv,
-                            unsigned int* amax_word, unsigned int* status, int num_sms, cudaStream_t s) {
-  cudaError_t e = cudaMemsetAsync(amax_word, 0, sizeof(unsigned int), s);
-  if (e != cudaSuccess) return e;
-  const size_t n_vec = static_cast<size_t>(h) * d / 8;
-  w2_amax_kernel<<<grid_for(n_vec, 256, num_sms, 4), 256, 0, s>>>(reinterpret_cast<const uint4*>(W2), n_vec,
-                                                                   amax_word);
+                            unsigned int* partial, unsigned int* status, int num_sms, cudaStream_t s) {
+  (void)num_sms;
+  const long long n = static_cast<long long>(h) * d;
+  const int nparts = static_cast<int>((n + kW2ElemsPerBlock - 1) / kW2ElemsPerBlock);
+  w2_amax_kernel<<<nparts, 256, 0, s>>>(reinterpret_cast<const uint4*>(W2), n / 8, partial);
   count_launches(1);
-  e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 grid((d + 63) / 64, (h + 63) / 64);
-  w2_quant_t_kernel<<<grid, 256, 0, s>>>(h, d, W2, W2q_t, w2_scale_inv, amax_word, status);
+  w2_quant_t_kernel<<<grid, 256, 0, s>>>(h, d, W2, W2q_t, w2_scale_inv, partial, nparts, status);
   count_launches(1);
   return cudaGetLastError();
 }

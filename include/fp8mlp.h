@@ -194,8 +194,8 @@ int fp8mlp_amax_reduce_update_scale(const float* partial_amax, int n, fp8mlp_sca
  *   s_w = fp32(448 / max|W2|)   (1 if max|W2| is 0 or not finite)
  *   W2q_t[j,i] = e4m3_satfinite( fp32(W2[i,j] * s_w) ),  w2_scale_inv[0] = fp32(1/s_w)
  * W2 [h,d] bf16, W2q_t [d,h] e4m3.  workspace: at least
- * fp8mlp_workspace_size(0,d,h) bytes of caller-owned device memory (a
- * reduction word; cleared by the call).
+ * fp8mlp_workspace_size(0,d,h) bytes of caller-owned device memory (one
+ * partial maximum per 8192 elements of W2; no initial contents needed).
  */
 int fp8mlp_w2_fp8_cache_refresh(int h, int d, const uint16_t* W2, uint8_t* W2q_t, float* w2_scale_inv,
                                 void* workspace, fp8mlp_stream_t stream);

@@ -534,3 +534,41 @@ def test_graph_replay_matches_eager():
     torch.cuda.synchronize()
     for k in ("post", "post_fp8", "out", "dPre", "dX", "dW1", "dW2", "W2q_t", "state", "partial_amax"):
         assert torch.equal(getattr(e, k), getattr(g, k)), k
+
+
+# ---------------------------------------------------------------------------
+# layer stack: RMSNorm + block + residual, forward and backward
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("L,M,d,h", [(3, 300, 128, 512), (2, 1024, 768, 3072)])
+def test_stack_vs_oracle(L, M, d, h):
+    from fp8_relu_mlp_b200.block import MLPBlock, MLPStack
+    g = np.random.default_rng(L * 100 + M)
+    r0 = synth.to_bf16_bits(g.standard_normal((M, d)).astype(np.float32))
+    dtop = synth.to_bf16_bits(g.standard_normal((M, d)).astype(np.float32))
+    layers, scales = [], []
+    S = MLPStack(L, M, d, h)
+    for l in range(L):
+        P = synth.make_problem(1, d, h, seed=500 + l)
+        W2q_t, s_w, s_wi = ref.w2_cache(P["W2"])
+        layers.append(dict(W1=P["W1"], W2=P["W2"], W2q_t=W2q_t, w2_scale_inv=s_wi))
+        s = np.float32(30.0 + 5 * l)
+        scales.append((s, np.float32(np.float32(1) / s)))
+        b = S.blocks[l]
+        b.W1.copy_(MLPBlock.bits_to_bf16(P["W1"], b.device))
+        b.W2.copy_(MLPBlock.bits_to_bf16(P["W2"], b.device))
+        A.fp8mlp_scale_state_init(b.state, 2.0, float(s))
+    S.refresh_w2_caches()
+    S.r[0].copy_(MLPBlock.bits_to_bf16(r0, S.device))
+    S.forward()
+    S.dr.copy_(MLPBlock.bits_to_bf16(dtop, S.device))
+    S.backward()
+    torch.cuda.synchronize()
+    saved, rL = ref.stack_forward(r0, layers, scales)
+    dr0, grads = ref.stack_backward(saved, layers, dtop)
+    assert rel_fro(ref.bf16_to_f64(host_bits(S.r[L])), ref.bf16_to_f64(rL)) < 2e-2
+    assert rel_fro(ref.bf16_to_f64(host_bits(S.dr)), ref.bf16_to_f64(dr0)) < 2e-2
+    for l in range(L):
+        assert rel_fro(host_bits(S.blocks[l].dW1), grads[l][0]) < 2e-2, l
+        assert rel_fro(host_bits(S.blocks[l].dW2), grads[l][1]) < 2e-2, l
+    assert A.fp8mlp_get_device_status() == 0
