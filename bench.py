@@ -47,12 +47,14 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="step16k", choices=["step16k", "train49k", "heavytail"])
+    ap.add_argument("--workload", default="step16k", choices=["step16k", "train49k", "heavytail", "stack9"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
     ap.add_argument("--eager", action="store_true", help="launch every call from the host instead of replaying a CUDA graph")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with N>1, run independent replicas (no partial-amax / dW all-reduce)")
     return ap.parse_args()
 
 
@@ -198,6 +200,24 @@ def oracle_step_timer(W, tokens, seed=0):
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:  # pragma: no cover
         threads = 1
+    if W.layers > 1:
+        g = synth.rng(seed)
+        r0 = synth.to_bf16_bits(synth.make_x(g, tokens, W.d, "normal"))
+        dtop = synth.to_bf16_bits(synth.make_x(g, tokens, W.d, "normal"))
+        Ps = [synth.make_problem(1, W.d, W.h, seed=l) for l in range(W.layers)]
+        st = {"s": [ref.scale_state_init(W.margin, 1.0) for _ in range(W.layers)]}
+
+        def step():
+            layers = []
+            for P in Ps:
+                W2q_t, s_w, s_wi = ref.w2_cache(P["W2"])
+                layers.append(dict(W1=P["W1"], W2=P["W2"], W2q_t=W2q_t, w2_scale_inv=s_wi))
+            scales = [(x["scale"], x["scale_inv"]) for x in st["s"]]
+            saved, _ = ref.stack_forward(r0, layers, scales)
+            ref.stack_backward(saved, layers, dtop)
+            st["s"] = [ref.scale_update(x, sv["amax"]) for x, sv in zip(st["s"], saved)]
+            return np
+        return step, threads
     P = synth.make_problem(tokens, W.d, W.h, seed=seed)
     st = {"s": ref.scale_state_init(W.margin, 1.0)}
 
@@ -211,6 +231,8 @@ def oracle_step_timer(W, tokens, seed=0):
 
 
 def cpu_baseline(W, seconds, tokens=512):
+    if W.layers > 1:
+        tokens = 128
     step, threads = oracle_step_timer(W, tokens)
     t0 = time.perf_counter()
     reps = 0
@@ -222,13 +244,13 @@ def cpu_baseline(W, seconds, tokens=512):
             break
     return {"value": tokens * reps / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"{reps} oracle steps of {tokens} tokens of the {W.name} workload "
-                      f"(d={W.d}, h={W.h}; fwd+bwd+scale+W2 cache), {el:.1f} s"}
+                      f"(d={W.d}, h={W.h}, {W.layers} layer(s); fwd+bwd+scale+W2 cache), {el:.1f} s"}
 
 
 def run_reference(a, W, world, rank):
     if rank != 0:
         return
-    tokens = 256
+    tokens = 256 if W.layers == 1 else 32
     step, threads = oracle_step_timer(W, tokens)
     for _ in range(a.warmup):
         step()
@@ -305,6 +327,9 @@ def run_ours(a, W, world, rank, local_rank):
         mark(6)
         blk.refresh_w2_cache()
         mark(7)
+
+    if world > 1 and not a.replicas:
+        return run_dp(a, W, world, rank, local_rank, blk, flush, dist, peaks, fp8_peak, fp8_src)
 
     # one step = one CUDA-graph replay of the whole call sequence.  A first,
     # untimed pass with an event between every kernel gives the per-kernel
@@ -432,6 +457,243 @@ def run_ours(a, W, world, rank, local_rank):
     return line
 
 
+def run_dp(a, W, world, rank, local_rank, blk, flush, dist, peaks, fp8_peak, fp8_src):
+    """Data-parallel training step on N ranks: each rank its own M tokens; the
+    partial amax is all-reduced (MAX) and dW1/dW2 all-reduced (mean) over
+    NCCL on a side stream that overlaps the dX GEMM (fp8_relu_mlp_b200.dp).
+    Steps are issued eagerly; the time is the max over ranks."""
+    import torch
+    from fp8_relu_mlp_b200 import _abi as A
+    from fp8_relu_mlp_b200.dp import DataParallelStep
+    M, d, h = W.M, W.d, W.h
+    stepper = DataParallelStep(blk)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for _ in range(max(a.warmup, 3)):
+        flush.zero_()
+        stepper()
+    torch.cuda.synchronize()
+    A.fp8mlp_clear_device_status()
+    dist.barrier()
+    torch.cuda.synchronize()
+    step_ms, dom_ms = [], []
+    n0 = A.fp8mlp_kernel_launch_count()
+    with ClockSampler(local_rank) as clk:
+        for _ in range(a.steps):
+            flush.zero_()
+            stepper(mark=lambda i: ev[i].record())
+            ev[3].synchronize()
+            step_ms.append(ev[0].elapsed_time(ev[3]))
+            dom_ms.append(ev[1].elapsed_time(ev[2]))
+    launches = A.fp8mlp_kernel_launch_count() - n0
+    dist.barrier()
+    status = A.fp8mlp_get_device_status()
+    total_s = sum(step_ms) * 1e-3
+    t = torch.tensor([total_s], device=blk.device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_s = float(t.item())
+    value = M * world * a.steps / total_s
+    work = kernel_work(M, d, h)
+    dom_s = statistics.mean(dom_ms) * 1e-3
+    achieved = work["bwd_dw"]["bf16"] / dom_s / 1e12
+    roof_t = 0.0
+    for n, w in work.items():
+        roof_t += max(w["bf16"] / (peaks["bf16_tflops"] * 1e12) + w["fp8"] / (fp8_peak * 1e12),
+                      w["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": total_s / a.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16+e4m3 (fp32 accumulate)",
+            "data": "synthetic (seeded; shapes of the 768-dim GPT-2-small / nanochat MLP)",
+            "config": dict(config_of(W), parallelism=f"dp{world}: NCCL all-reduce of partial amax (MAX) "
+                                                     f"and dW1/dW2 (mean), overlapped with dX"),
+            "roofline": {"bound": "tensor", "kernel": "bwd_dw", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "traffic": load_traffic(W.name).get("bwd_dw"),
+                         "peak_source": f"bf16_tflops burst of {peaks['source']} peaks"},
+            "step_roofline": {"roofline_ms": roof_t * 1e3, "measured_ms": total_s / a.steps * 1e3,
+                              "frac": roof_t / (total_s / a.steps)},
+            "clocks": clk.summary(), "gpu_launches": int(launches), "device_status": status,
+            "launch_mode": "eager",
+        }
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
+    return None
+
+
+def run_stack(a, W, world, rank, local_rank):
+    """The 9-layer stack workload: per step, forward through every layer
+    (RMSNorm, block, residual), backward through every layer, the scale
+    updates and the W2 cache refreshes, replayed as one CUDA graph."""
+    import numpy as np
+    import torch
+    from fp8_relu_mlp_b200 import _abi as A
+    from fp8_relu_mlp_b200 import synth
+    from fp8_relu_mlp_b200.block import MLPBlock, MLPStack
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    L, M, d, h = W.layers, W.M, W.d, W.h
+    peaks = load_peaks()
+    fp8_peak, fp8_src = measure_fp8_peak(torch, peaks["bf16_tflops"])
+    S = MLPStack(L, M, d, h, device=dev, margin=W.margin)
+    g = synth.rng(1000 + rank)
+    r0 = synth.to_bf16_bits(synth.make_x(g, M, d, "normal"))
+    dtop = synth.to_bf16_bits(synth.make_x(g, M, d, "normal"))
+    for l, b in enumerate(S.blocks):
+        P = synth.make_problem(1, d, h, seed=100 * rank + l)
+        b.W1.copy_(MLPBlock.bits_to_bf16(P["W1"], dev))
+        b.W2.copy_(MLPBlock.bits_to_bf16(P["W2"], dev))
+    S.r[0].copy_(MLPBlock.bits_to_bf16(r0, dev))
+    dtop_d = MLPBlock.bits_to_bf16(dtop, dev)
+    S.refresh_w2_caches()
+    S.calibrate()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    last = S.blocks[L - 1]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record()
+        mark(0)
+        S.forward()
+        S.dr.copy_(dtop_d)
+        # backward of the top layer, with its dW launch marked
+        A.fp8mlp_bwd_dpre(M, d, h, S.dr, last.W2, last.post, last.dPre)
+        A.fp8mlp_bwd_dx(M, d, h, last.dPre, last.W1, last.dX)
+        mark(1)
+        A.fp8mlp_bwd_dw(M, d, h, last.x, last.dPre, last.post, S.dr, last.dW1, last.dW2)
+        mark(2)
+        A.fp8mlp_rmsnorm_bwd(M, d, S.r[L - 1], S.rstd[L - 1], last.dX, S.dr, S.dr)
+        for l in range(L - 2, -1, -1):
+            b = S.blocks[l]
+            A.fp8mlp_mlp_bwd(M, d, h, b.x, b.W1, b.W2, b.post, S.dr, b.dPre, b.dX, b.dW1, b.dW2)
+            A.fp8mlp_rmsnorm_bwd(M, d, S.r[l], S.rstd[l], b.dX, S.dr, S.dr)
+        S.update_scales()
+        S.refresh_w2_caches()
+        mark(3)
+
+    step()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True, external=not a.eager) for _ in range(4)]
+    n_cap0 = A.fp8mlp_kernel_launch_count()
+    graph = None if a.eager else S.blocks[0].capture(lambda: step(ev))
+    kernels_per_step = A.fp8mlp_kernel_launch_count() - n_cap0
+
+    def run():
+        if graph is not None:
+            graph.replay()
+        else:
+            step(ev)
+
+    for _ in range(max(a.warmup, 3)):
+        flush.zero_()
+        run()
+    torch.cuda.synchronize()
+    A.fp8mlp_clear_device_status()
+    if dist:
+        dist.barrier()
+    step_ms, dom_ms = [], []
+    n0 = A.fp8mlp_kernel_launch_count()
+    with ClockSampler(local_rank) as clk:
+        for _ in range(a.steps):
+            flush.zero_()
+            run()
+            ev[3].synchronize()
+            step_ms.append(ev[0].elapsed_time(ev[3]))
+            dom_ms.append(ev[1].elapsed_time(ev[2]))
+    launches = kernels_per_step * a.steps if graph is not None else A.fp8mlp_kernel_launch_count() - n0
+    status = A.fp8mlp_get_device_status()
+    total_s = sum(step_ms) * 1e-3
+    if dist:
+        t = torch.tensor([total_s], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_s = float(t.item())
+    value = M * world * a.steps / total_s
+    work = kernel_work(M, d, h)
+    # per layer: the five GEMMs and the small kernels, plus RMSNorm fwd (read r,
+    # write x), residual add (read r, out; write r'), RMSNorm bwd (read r, dX,
+    # dr; write dr) and the dr copy
+    norm_bytes = (2 + 3 + 4) * 2 * M * d
+    roof_t = 0.0
+    for n, w in work.items():
+        roof_t += max(w["bf16"] / (peaks["bf16_tflops"] * 1e12) + w["fp8"] / (fp8_peak * 1e12),
+                      w["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    roof_t = L * (roof_t + norm_bytes / (peaks["hbm_gbs"] * 1e9)) + 4 * M * d / (peaks["hbm_gbs"] * 1e9)
+    dom_s = statistics.mean(dom_ms) * 1e-3
+    achieved = work["bwd_dw"]["bf16"] / dom_s / 1e12
+    # a step of tens of milliseconds runs under the power cap: the kernel is
+    # compared with the sustained BF16 figure
+    peak_sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    e2e = None
+    if not a.no_e2e:
+        r0h = torch.from_numpy(r0.view(np.int16)).view(torch.bfloat16).pin_memory()
+        dth = torch.from_numpy(dtop.view(np.int16)).view(torch.bfloat16).pin_memory()
+        rLh = torch.empty(M, d, dtype=torch.bfloat16).pin_memory()
+        dr0h = torch.empty(M, d, dtype=torch.bfloat16).pin_memory()
+
+        def body():
+            S.r[0].copy_(r0h, non_blocking=True)
+            dtop_d.copy_(dth, non_blocking=True)
+            step()
+            rLh.copy_(S.r[L], non_blocking=True)
+            dr0h.copy_(S.dr, non_blocking=True)
+
+        body()
+        torch.cuda.synchronize()
+        g2 = None if a.eager else S.blocks[0].capture(body)
+        for _ in range(2):
+            g2.replay() if g2 is not None else body()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+        e0.record()
+        for _ in range(a.steps):
+            g2.replay() if g2 is not None else body()
+        e1.record()
+        e1.synchronize()
+        t2 = e0.elapsed_time(e1) * 1e-3
+        if dist:
+            tt = torch.tensor([t2], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            t2 = float(tt.item())
+        e2e = {"value": M * world * a.steps / t2, "unit": "tokens/s", "h2d_bytes_per_step": 4 * M * d,
+               "d2h_bytes_per_step": 4 * M * d}
+    if rank == 0:
+        traffic = load_traffic(W.name).get("bwd_dw")
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": total_s / a.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16+e4m3 (fp32 accumulate)",
+            "data": "synthetic (seeded; 9-layer 768-dim ReLU^2 stack of the nanochat runs)",
+            "config": dict(config_of(W), layers=L, parallelism=f"dp{world} replicas" if world > 1 else "single GPU"),
+            "roofline": {"bound": "tensor", "kernel": "bwd_dw (top layer)", "achieved": achieved,
+                         "peak": peak_sus, "unit": "TFLOP/s", "frac": achieved / peak_sus,
+                         "traffic": traffic,
+                         "peak_source": f"bf16_tflops_sustained of {peaks['source']} peaks (long step, power cap)"},
+            "step_roofline": {"roofline_ms": roof_t * 1e3, "measured_ms": total_s / a.steps * 1e3,
+                              "frac": roof_t / (total_s / a.steps),
+                              "peaks": {"bf16_tflops": peaks["bf16_tflops"], "fp8_tflops": fp8_peak,
+                                        "hbm_gbs": peaks["hbm_gbs"]}},
+            "clocks": clk.summary(), "gpu_launches": int(launches), "device_status": status,
+            "launch_mode": "eager" if graph is None else "cuda_graph",
+        }
+        if e2e:
+            line["e2e"] = e2e
+        if not a.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(W, a.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if dist:
+        del graph
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def measure_e2e(a, blk, P, torch, dev, stream, M, world, dist):
     """Same step through the public API with host buffers: the step's inputs
     (x, dOut) come from pinned host memory and its results (out, dX) go back
@@ -494,7 +756,10 @@ def main():
     if a.impl == "reference":
         run_reference(a, W, world, rank)
         return 0
-    run_ours(a, W, world, rank, local_rank)
+    if W.layers > 1:
+        run_stack(a, W, world, rank, local_rank)
+    else:
+        run_ours(a, W, world, rank, local_rank)
     return 0
 
 

@@ -572,3 +572,45 @@ def test_stack_vs_oracle(L, M, d, h):
         assert rel_fro(host_bits(S.blocks[l].dW1), grads[l][0]) < 2e-2, l
         assert rel_fro(host_bits(S.blocks[l].dW2), grads[l][1]) < 2e-2, l
     assert A.fp8mlp_get_device_status() == 0
+
+
+# ---------------------------------------------------------------------------
+# the data-parallel step on a one-rank NCCL group equals the plain step
+# ---------------------------------------------------------------------------
+
+def test_data_parallel_step_single_rank():
+    import os
+    import socket
+    import torch.distributed as dist
+    from fp8_relu_mlp_b200.block import MLPBlock
+    from fp8_relu_mlp_b200.dp import DataParallelStep
+    M, d, h = 1000, 768, 3072
+    P = synth.make_problem(M, d, h, seed=91)
+
+    def make():
+        b = MLPBlock(M, d, h)
+        for k in ("x", "W1", "W2", "dOut"):
+            getattr(b, k).copy_(MLPBlock.bits_to_bf16(P[k], b.device))
+        b.refresh_w2_cache()
+        b.calibrate()
+        return b
+
+    plain = make()
+    plain.forward()
+    plain.backward()
+    plain.update_scale()
+    plain.refresh_w2_cache()
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("nccl", rank=0, world_size=1)
+    try:
+        b = make()
+        DataParallelStep(b)()
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    for k in ("post", "post_fp8", "out", "dPre", "dX", "dW1", "dW2", "state", "W2q_t"):
+        assert torch.equal(getattr(plain, k), getattr(b, k)), k
