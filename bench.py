@@ -53,6 +53,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
     ap.add_argument("--eager", action="store_true", help="launch every call from the host instead of replaying a CUDA graph")
+    ap.add_argument("--no-pdl", action="store_true", help="launch without programmatic dependent launch")
     ap.add_argument("--replicas", action="store_true",
                     help="with N>1, run independent replicas (no partial-amax / dW all-reduce)")
     return ap.parse_args()
@@ -292,6 +293,7 @@ def run_ours(a, W, world, rank, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    A.fp8mlp_set_programmatic_launch(not a.no_pdl)
     M, d, h = W.M, W.d, W.h
     peaks = load_peaks()
     fp8_peak, fp8_src = measure_fp8_peak(torch, peaks["bf16_tflops"])
@@ -421,6 +423,9 @@ def run_ours(a, W, world, rank, local_rank):
     e2e = None
     if not a.no_e2e:
         e2e = measure_e2e(a, blk, P, torch, dev, stream, M, world, dist)
+    schedule = None
+    if W.spike_steps and rank == 0:
+        schedule = spike_schedule(W, blk, P, torch, dev)
 
     line = None
     if rank == 0:
@@ -444,10 +449,12 @@ def run_ours(a, W, world, rank, local_rank):
             "kernels_ms": breakdown,
             "kernels_ms_note": "median of 5 untimed steps with an event between every kernel",
             "clocks": clocks, "gpu_launches": int(launches), "device_status": status,
-            "launch_mode": "eager" if g_t is None else "cuda_graph",
+            "launch_mode": ("eager" if g_t is None else "cuda_graph") + ("" if a.no_pdl else " + programmatic dependent launch"),
         }
         if e2e:
             line["e2e"] = e2e
+        if schedule:
+            line["spike_schedule"] = schedule
         if not a.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(W, a.cpu_seconds)
         print(json.dumps(line), flush=True)
@@ -455,6 +462,27 @@ def run_ours(a, W, world, rank, local_rank):
         dist.barrier()
         dist.destroy_process_group()
     return line
+
+
+def spike_schedule(W, blk, P, torch, dev):
+    """Run the workload's step schedule (x doubled at the spike steps) and
+    report, per step, the delayed scale used, the amax measured and the
+    fraction of FP8 codes that saturated at +-448."""
+    from fp8_relu_mlp_b200 import _abi as A
+    from fp8_relu_mlp_b200.block import MLPBlock
+    x0 = MLPBlock.bits_to_bf16(P["x"], dev)
+    A.fp8mlp_scale_state_init(blk.state, W.margin, 1.0)
+    blk.x.copy_(x0)
+    blk.calibrate()
+    steps = []
+    for t in range(W.steps):
+        blk.x.copy_(x0 * W.spike_factor if t in W.spike_steps else x0)
+        s_used = blk.read_state()["scale"]
+        blk.train_step()
+        st = blk.read_state()
+        sat = float(((blk.post_fp8 & 0x7F) == 0x7E).float().mean())
+        steps.append({"step": t, "scale": s_used, "amax": st["amax_prev"], "saturated_frac": sat})
+    return {"spike_steps": list(W.spike_steps), "x_factor": W.spike_factor, "steps": steps}
 
 
 def run_dp(a, W, world, rank, local_rank, blk, flush, dist, peaks, fp8_peak, fp8_src):
@@ -539,6 +567,7 @@ def run_stack(a, W, world, rank, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    A.fp8mlp_set_programmatic_launch(not a.no_pdl)
     L, M, d, h = W.layers, W.M, W.d, W.h
     peaks = load_peaks()
     fp8_peak, fp8_src = measure_fp8_peak(torch, peaks["bf16_tflops"])

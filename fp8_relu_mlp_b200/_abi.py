@@ -68,6 +68,7 @@ _SIGS = {
     "fp8mlp_clear_device_status": [_p],
     "fp8mlp_set_wait_timeout_ns": [_u64],
     "fp8mlp_set_debug_flags": [_i],
+    "fp8mlp_set_programmatic_launch": [_i],
 }
 for _n, _a in _SIGS.items():
     _fn = getattr(lib, _n)
@@ -227,6 +228,10 @@ def fp8mlp_clear_device_status(stream=None):
 
 def fp8mlp_set_wait_timeout_ns(ns):
     return _call("fp8mlp_set_wait_timeout_ns", int(ns))
+
+
+def fp8mlp_set_programmatic_launch(enable):
+    return _call("fp8mlp_set_programmatic_launch", int(bool(enable)))
 
 
 def fp8mlp_set_debug_flags(flags):

@@ -17,6 +17,7 @@ thread_local std::string g_detail;
 std::atomic<unsigned long long> g_launches{0};
 std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
 std::atomic<int> g_debug_flags{0};
+std::atomic<int> g_pdl{1};
 
 int fail(int code, const std::string& what) {
   g_detail = what;
@@ -138,6 +139,8 @@ int launch(GemmKind k, const GemmParams& p, const DeviceInfo* di, cudaStream_t s
 void count_launches(unsigned long long n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
 void set_error_detail(const char* what) { g_detail = what; }
+
+bool pdl_enabled() { return g_pdl.load(std::memory_order_relaxed) != 0; }
 
 int current_device(DeviceInfo** info) {
   int dev = -1;
@@ -492,6 +495,11 @@ int fp8mlp_clear_device_status(fp8mlp_stream_t stream) {
 int fp8mlp_set_wait_timeout_ns(unsigned long long ns) {
   if (ns == 0) return fail(FP8MLP_ERR_INVALID_ARG, "timeout must be > 0");
   g_timeout_ns.store(ns);
+  return FP8MLP_OK;
+}
+
+int fp8mlp_set_programmatic_launch(int enable) {
+  g_pdl.store(enable ? 1 : 0);
   return FP8MLP_OK;
 }
 

@@ -176,6 +176,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
   if constexpr (CG == 2) cluster_sync();  // the peer's barriers are initialised
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // the set-up above overlaps the previous kernel's tail; from here on global
+  // memory is read and written
+  pdl_wait();
+  if (threadIdx.x == 0) pdl_launch_dependents();
   const WaitCtx w{p.status, abort_flag, p.timeout_ns};
 
   const int tiles_per_group = p.tiles_m * p.tiles_n;

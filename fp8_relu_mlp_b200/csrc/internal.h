@@ -57,6 +57,27 @@ void set_error_detail(const char* what);
 // number of kernels this library has launched (all devices, all threads)
 void count_launches(unsigned long long n);
 
+// programmatic dependent launch on/off (fp8mlp_set_programmatic_launch)
+bool pdl_enabled();
+
+// Launch `k` with the programmatic stream-serialisation attribute (when
+// enabled): the kernel may start while the previous kernel on the stream
+// finishes, and waits for it with pdl_wait() before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, static_cast<KArgs>(args)...);
+}
+
 // status word symbol address on the current device
 cudaError_t status_word_address(unsigned int** ptr);
 

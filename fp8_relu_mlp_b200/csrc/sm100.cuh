@@ -90,6 +90,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
 }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialisation attribute may start before the previous kernel on the
+// stream has finished; it must wait (pdl_wait) before touching global memory
+// the previous kernel writes or reads.  pdl_launch_dependents lets the next
+// kernel start launching once every CTA of this grid has issued it (or
+// exited), so no CTA of this grid is left waiting for an SM.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // clusters (pairs of CTAs sharing one 2-CTA UMMA)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {

@@ -18,6 +18,8 @@ namespace {
 using namespace dev;
 
 __global__ void state_init_kernel(fp8mlp_scale_state* st, float margin, float s0) {
+  pdl_wait();
+  pdl_launch_dependents();
   st->amax_prev = 0.f;
   st->scale = s0;
   st->scale_inv = __fdiv_rn(1.f, s0);
@@ -31,6 +33,8 @@ __global__ void state_init_kernel(fp8mlp_scale_state* st, float margin, float s0
 // A = max(partial amax); s = 448 / (margin * A); see fp8mlp_amax_reduce_update_scale.
 __global__ void __launch_bounds__(1024) amax_scale_kernel(const float* __restrict__ pa, int n,
                                                           fp8mlp_scale_state* st, unsigned int* status) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ float smax[32];
   __shared__ int snan[32];
   float m = 0.f;
@@ -96,6 +100,8 @@ __global__ void __launch_bounds__(1024) amax_scale_kernel(const float* __restric
 // partial[b]; the quantising kernel reduces the partials.
 __global__ void __launch_bounds__(256) w2_amax_kernel(const uint4* __restrict__ W, long long n_vec,
                                                       unsigned int* __restrict__ partial) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ unsigned int wmax[8];
   const long long base = static_cast<long long>(blockIdx.x) * (kW2ElemsPerBlock / 8);
   unsigned int m = 0;
@@ -139,6 +145,8 @@ __global__ void __launch_bounds__(256) w2_quant_t_kernel(int h, int d, const uin
                                                          const unsigned int* __restrict__ partial, int nparts,
                                                          unsigned int* status) {
   __shared__ float tile[64][65];
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ unsigned int wmax[8];
   const int i0 = blockIdx.y * 64;  // rows of W2 (h)
   const int j0 = blockIdx.x * 64;  // cols of W2 (d)
@@ -185,6 +193,8 @@ __global__ void __launch_bounds__(256) w2_quant_t_kernel(int h, int d, const uin
 // One warp per row.  d is a multiple of 16; each lane handles 8-element groups.
 __global__ void rmsnorm_fwd_kernel(int M, int d, const uint16_t* __restrict__ r, uint16_t* __restrict__ x,
                                    float* __restrict__ rstd) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
   for (int row = blockIdx.x * warps + (threadIdx.x >> 5); row < M; row += gridDim.x * warps) {
@@ -219,6 +229,8 @@ __global__ void rmsnorm_fwd_kernel(int M, int d, const uint16_t* __restrict__ r,
 
 __global__ void rmsnorm_bwd_kernel(int M, int d, const uint16_t* __restrict__ r, const float* __restrict__ rstd,
                                    const uint16_t* __restrict__ dx, const uint16_t* dr_in, uint16_t* dr_out) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
   for (int row = blockIdx.x * warps + (threadIdx.x >> 5); row < M; row += gridDim.x * warps) {
@@ -259,6 +271,8 @@ __global__ void rmsnorm_bwd_kernel(int M, int d, const uint16_t* __restrict__ r,
 
 __global__ void residual_add_kernel(size_t n_vec, const uint4* __restrict__ r, const uint4* __restrict__ o,
                                     uint4* __restrict__ rn) {
+  pdl_wait();
+  pdl_launch_dependents();
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n_vec;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const uint4 a = r[i], b = o[i];
@@ -282,15 +296,15 @@ int grid_for(size_t work, int per_block, int num_sms, int blocks_per_sm) {
 }  // namespace
 
 cudaError_t launch_state_init(fp8mlp_scale_state* st, float margin, float s0, cudaStream_t s) {
-  state_init_kernel<<<1, 1, 0, s>>>(st, margin, s0);
+  const cudaError_t e = launch_pdl(state_init_kernel, dim3(1), dim3(1), 0, s, st, margin, s0);
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_amax_scale(const float* pa, int n, fp8mlp_scale_state* st, unsigned int* status, cudaStream_t s) {
-  amax_scale_kernel<<<1, 1024, 0, s>>>(pa, n, st, status);
+  const cudaError_t e = launch_pdl(amax_scale_kernel, dim3(1), dim3(1024), 0, s, pa, n, st, status);
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_w2_cache(int h, int d, const uint16_t* W2, uint8_t* W2q_t, float* w2_scale_inv,
@@ -298,38 +312,41 @@ cudaError_t launch_w2_cache(int h, int d, const uint16_t* W2, uint8_t* W2q_t, fl
   (void)num_sms;
   const long long n = static_cast<long long>(h) * d;
   const int nparts = static_cast<int>((n + kW2ElemsPerBlock - 1) / kW2ElemsPerBlock);
-  w2_amax_kernel<<<nparts, 256, 0, s>>>(reinterpret_cast<const uint4*>(W2), n / 8, partial);
+  cudaError_t e = launch_pdl(w2_amax_kernel, dim3(nparts), dim3(256), 0, s, reinterpret_cast<const uint4*>(W2),
+                             n / 8, partial);
   count_launches(1);
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 grid((d + 63) / 64, (h + 63) / 64);
-  w2_quant_t_kernel<<<grid, 256, 0, s>>>(h, d, W2, W2q_t, w2_scale_inv, partial, nparts, status);
+  e = launch_pdl(w2_quant_t_kernel, grid, dim3(256), 0, s, h, d, W2, W2q_t, w2_scale_inv,
+                 static_cast<const unsigned int*>(partial), nparts, status);
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_rmsnorm_fwd(int M, int d, const uint16_t* r, uint16_t* x, float* rstd, int num_sms,
                                cudaStream_t s) {
-  rmsnorm_fwd_kernel<<<grid_for(static_cast<size_t>(M), 8, num_sms, 8), 256, 0, s>>>(M, d, r, x, rstd);
+  const cudaError_t e = launch_pdl(rmsnorm_fwd_kernel, dim3(grid_for(static_cast<size_t>(M), 8, num_sms, 8)),
+                                   dim3(256), 0, s, M, d, r, x, rstd);
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_rmsnorm_bwd(int M, int d, const uint16_t* r, const float* rstd, const uint16_t* dx,
                                const uint16_t* dr_in, uint16_t* dr_out, int num_sms, cudaStream_t s) {
-  rmsnorm_bwd_kernel<<<grid_for(static_cast<size_t>(M), 8, num_sms, 8), 256, 0, s>>>(M, d, r, rstd, dx, dr_in,
-                                                                                      dr_out);
+  const cudaError_t e = launch_pdl(rmsnorm_bwd_kernel, dim3(grid_for(static_cast<size_t>(M), 8, num_sms, 8)),
+                                   dim3(256), 0, s, M, d, r, rstd, dx, dr_in, dr_out);
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_residual_add(int M, int d, const uint16_t* r, const uint16_t* out, uint16_t* r_next,
                                 int num_sms, cudaStream_t s) {
   const size_t n_vec = static_cast<size_t>(M) * d / 8;
-  residual_add_kernel<<<grid_for(n_vec, 256, num_sms, 8), 256, 0, s>>>(
-      n_vec, reinterpret_cast<const uint4*>(r), reinterpret_cast<const uint4*>(out), reinterpret_cast<uint4*>(r_next));
+  const cudaError_t e =
+      launch_pdl(residual_add_kernel, dim3(grid_for(n_vec, 256, num_sms, 8)), dim3(256), 0, s, n_vec,
+                 reinterpret_cast<const uint4*>(r), reinterpret_cast<const uint4*>(out), reinterpret_cast<uint4*>(r_next));
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace fp8mlp

@@ -281,6 +281,12 @@ int fp8mlp_residual_add(int M, int d, const uint16_t* r, const uint16_t* out, ui
 int fp8mlp_get_device_status(unsigned int* status, fp8mlp_stream_t stream);
 /* Clear the device status word (enqueued on `stream`). */
 int fp8mlp_clear_device_status(fp8mlp_stream_t stream);
+/* Programmatic dependent launch (default on): every kernel of the library is
+ * launched so that it may start while the previous kernel on the stream is
+ * finishing (its set-up overlaps that kernel's tail); each kernel waits for
+ * the previous one to complete before it touches global memory, so results
+ * do not depend on this setting.  0 turns it off for later launches. */
+int fp8mlp_set_programmatic_launch(int enable);
 /* Per-wait limit of the kernels' bounded waits, in ns (default 2e9). */
 int fp8mlp_set_wait_timeout_ns(unsigned long long ns);
 /* Test hook: FP8MLP_DEBUG_STALL_PRODUCER makes the next GEMM launches'
