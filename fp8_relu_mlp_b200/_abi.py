@@ -58,6 +58,10 @@ _SIGS = {
     "fp8mlp_w2_fp8_cache_refresh": [_i, _i, _p, _p, _p, _p, _p],
     "fp8mlp_w2_fp8_cache_refresh_noalloc": [_i, _i, _p, _p, _p, _p],
     "fp8mlp_bwd_dpre": [_i, _i, _i, _p, _p, _p, _p, _p],
+    "fp8mlp_quantize_x": [_i, _i, _p, _p, _p, _p, _p],
+    "fp8mlp_x_partial_amax_count": [_i, _i],
+    "fp8mlp_w1_fp8_cache_refresh": [_i, _i, _p, _p, _p, _p, _p],
+    "fp8mlp_up_proj_fused_fp8": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _p],
     "fp8mlp_bwd_dx": [_i, _i, _i, _p, _p, _p, _p],
     "fp8mlp_bwd_dw": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p],
     "fp8mlp_mlp_bwd": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p],
@@ -183,6 +187,25 @@ def fp8mlp_w2_fp8_cache_refresh_noalloc(h, d, W2, W2q_t, w2_scale_inv, stream=No
 
 def fp8mlp_workspace_size(M, d, h):
     return int(lib.fp8mlp_workspace_size(M, d, h))
+
+
+def fp8mlp_quantize_x(M, d, x, st_x, x_fp8, partial_amax_x, stream=None):
+    return _call("fp8mlp_quantize_x", M, d, _ptr(x), _ptr(st_x), _ptr(x_fp8), _ptr(partial_amax_x), _stream(stream))
+
+
+def fp8mlp_x_partial_amax_count(M, d):
+    return int(lib.fp8mlp_x_partial_amax_count(M, d))
+
+
+def fp8mlp_w1_fp8_cache_refresh(h, d, W1, W1q, w1_scale_inv, workspace, stream=None):
+    return _call("fp8mlp_w1_fp8_cache_refresh", h, d, _ptr(W1), _ptr(W1q), _ptr(w1_scale_inv), _ptr(workspace),
+                 _stream(stream))
+
+
+def fp8mlp_up_proj_fused_fp8(M, d, h, x_fp8, W1q, w1_scale_inv, st_x, st, post, post_fp8, partial_amax,
+                             pre_debug=None, flags=0, stream=None):
+    return _call("fp8mlp_up_proj_fused_fp8", M, d, h, _ptr(x_fp8), _ptr(W1q), _ptr(w1_scale_inv), _ptr(st_x),
+                 _ptr(st), _ptr(post), _ptr(post_fp8), _ptr(partial_amax), _ptr(pre_debug), flags, _stream(stream))
 
 
 def fp8mlp_bwd_dpre(M, d, h, dOut, W2, post, dPre, stream=None):

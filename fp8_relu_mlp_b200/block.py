@@ -21,8 +21,12 @@ from . import _abi as A
 
 class MLPBlock:
     def __init__(self, M: int, d: int, h: int, device="cuda", margin: float = 2.0, initial_scale: float = 1.0,
-                 with_backward: bool = True, stream=None):
+                 with_backward: bool = True, stream=None, fp8_up: bool = False):
+        """``fp8_up``: run the up-projection on e4m3 copies of x (delayed scale
+        of its own) and W1 (exact cache scale) as well; the backward keeps the
+        BF16 x and W1."""
         self.M, self.d, self.h = M, d, h
+        self.fp8_up = fp8_up
         self.device = torch.device(device)
         self.stream = stream
         dev = self.device
@@ -46,19 +50,55 @@ class MLPBlock:
             self.dW1 = torch.empty(h, d, dtype=f32, device=dev)
             self.dW2 = torch.empty(h, d, dtype=f32, device=dev)
         A.fp8mlp_scale_state_init(self.state, margin, initial_scale, self.stream)
+        if fp8_up:
+            self.x_fp8 = torch.empty(M, d, dtype=u8, device=dev)
+            self.W1q = torch.zeros(h, d, dtype=u8, device=dev)
+            self.w1_scale_inv = torch.ones(4, dtype=f32, device=dev)
+            self.state_x = torch.zeros(8, dtype=f32, device=dev)
+            self.partial_amax_x = torch.zeros(max(1, A.fp8mlp_x_partial_amax_count(M, d)), dtype=f32, device=dev)
+            A.fp8mlp_scale_state_init(self.state_x, margin, initial_scale, self.stream)
 
     # ------------------------------------------------------------------ calls
+    def refresh_w1_cache(self):
+        A.fp8mlp_w1_fp8_cache_refresh(self.h, self.d, self.W1, self.W1q, self.w1_scale_inv, self.workspace,
+                                      self.stream)
+
+    def _quantize_x(self):
+        A.fp8mlp_quantize_x(self.M, self.d, self.x, self.state_x, self.x_fp8, self.partial_amax_x, self.stream)
+
+    def _update_x_scale(self):
+        A.fp8mlp_amax_reduce_update_scale(self.partial_amax_x, A.fp8mlp_x_partial_amax_count(self.M, self.d),
+                                          self.state_x, self.stream)
+
+    def _up_fp8(self, flags):
+        A.fp8mlp_up_proj_fused_fp8(self.M, self.d, self.h, self.x_fp8, self.W1q, self.w1_scale_inv, self.state_x,
+                                   self.state, self.post, self.post_fp8 if flags == 0 else None,
+                                   self.partial_amax, None, flags, self.stream)
     def refresh_w2_cache(self):
         A.fp8mlp_w2_fp8_cache_refresh(self.h, self.d, self.W2, self.W2q_t, self.w2_scale_inv, self.workspace,
                                       self.stream)
 
     def calibrate(self):
-        """Step 0: post and partial amax only, then the first scale."""
+        """Step 0: post and partial amax only, then the first scale (with the
+        FP8 up-projection, first the x-scale from x's own amax)."""
+        if self.fp8_up:
+            self._quantize_x()
+            self._update_x_scale()
+            self._quantize_x()
+            self._up_fp8(A.FWD_CALIBRATE)
+            A.fp8mlp_amax_reduce_update_scale(self.partial_amax, self.partial_amax.numel(), self.state, self.stream)
+            return
         A.fp8mlp_mlp_fwd(self.M, self.d, self.h, self.x, self.W1, None, None, None, self.state, self.post, None,
                          self.partial_amax, None, None, A.FWD_CALIBRATE, self.stream)
         self.update_scale()
 
     def forward(self, eval_bf16: bool = False, pre_debug=None):
+        if self.fp8_up and not eval_bf16:
+            self._quantize_x()
+            self._up_fp8(0)
+            A.fp8mlp_down_proj_fp8(self.M, self.d, self.h, self.post_fp8, self.W2q_t, self.w2_scale_inv, self.state,
+                                   self.out, self.stream)
+            return
         flags = A.FWD_EVAL_BF16 if eval_bf16 else 0
         A.fp8mlp_mlp_fwd(self.M, self.d, self.h, self.x, self.W1, self.W2q_t, self.w2_scale_inv, self.W2,
                          self.state, self.post, None if eval_bf16 else self.post_fp8, self.partial_amax, self.out,
@@ -66,6 +106,8 @@ class MLPBlock:
 
     def update_scale(self):
         A.fp8mlp_amax_reduce_update_scale(self.partial_amax, self.partial_amax.numel(), self.state, self.stream)
+        if self.fp8_up:
+            self._update_x_scale()
 
     def backward(self):
         A.fp8mlp_mlp_bwd(self.M, self.d, self.h, self.x, self.W1, self.W2, self.post, self.dOut, self.dPre,
@@ -90,8 +132,8 @@ class MLPBlock:
         return g
 
     # --------------------------------------------------------------- helpers
-    def read_state(self) -> dict:
-        s = self.state.cpu()
+    def read_state(self, state=None) -> dict:
+        s = (self.state if state is None else state).cpu()
         i = s.view(torch.int32)
         return dict(amax_prev=float(s[0]), scale=float(s[1]), scale_inv=float(s[2]), margin=float(s[3]),
                     step=int(i[4]), flags=int(i[5]))

@@ -340,6 +340,82 @@ int fp8mlp_w2_fp8_cache_refresh(int h, int d, const uint16_t* W2, uint8_t* W2q_t
   return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "w2_fp8_cache_refresh launch");
 }
 
+int fp8mlp_x_partial_amax_count(int M, int d) {
+  if (M < 0 || d < 0) return 0;
+  const long long n = static_cast<long long>(M) * d;
+  return static_cast<int>((n + kXElemsPerBlock - 1) / kXElemsPerBlock);
+}
+
+int fp8mlp_quantize_x(int M, int d, const uint16_t* x, const fp8mlp_scale_state* st_x, uint8_t* x_fp8,
+                      float* partial_amax_x, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, d, 16));
+  if (M == 0) return FP8MLP_OK;
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(st_x);
+  REQUIRE_PTR(x_fp8);
+  if (partial_amax_x == nullptr || (reinterpret_cast<uintptr_t>(partial_amax_x) & 3u))
+    return fail(FP8MLP_ERR_INVALID_ARG, "partial_amax_x is NULL or misaligned");
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  const cudaError_t e = launch_quantize_x(static_cast<long long>(M) * d, x, st_x, x_fp8, partial_amax_x, stream);
+  return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "quantize_x launch");
+}
+
+int fp8mlp_w1_fp8_cache_refresh(int h, int d, const uint16_t* W1, uint8_t* W1q, float* w1_scale_inv,
+                                void* workspace, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(0, d, h));
+  REQUIRE_PTR(W1);
+  REQUIRE_PTR(W1q);
+  REQUIRE_PTR(workspace);
+  if (w1_scale_inv == nullptr) return fail(FP8MLP_ERR_INVALID_ARG, "w1_scale_inv is NULL");
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  const cudaError_t e = launch_w1_cache(h, d, W1, W1q, w1_scale_inv, static_cast<unsigned int*>(workspace),
+                                        di->status, stream);
+  return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "w1_fp8_cache_refresh launch");
+}
+
+int fp8mlp_up_proj_fused_fp8(int M, int d, int h, const uint8_t* x_fp8, const uint8_t* W1q,
+                             const float* w1_scale_inv, const fp8mlp_scale_state* st_x, const fp8mlp_scale_state* st,
+                             uint16_t* post, uint8_t* post_fp8, float* partial_amax, float* pre_debug, int flags,
+                             fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, d, h));
+  if (flags & ~(FP8MLP_FWD_EVAL_BF16 | FP8MLP_FWD_CALIBRATE)) return fail(FP8MLP_ERR_INVALID_ARG, "unknown flags");
+  const bool write_q = (flags & (FP8MLP_FWD_EVAL_BF16 | FP8MLP_FWD_CALIBRATE)) == 0;
+  if (M == 0) return FP8MLP_OK;
+  REQUIRE_PTR(x_fp8);
+  REQUIRE_PTR(W1q);
+  REQUIRE_PTR(st_x);
+  REQUIRE_PTR(post);
+  if (w1_scale_inv == nullptr) return fail(FP8MLP_ERR_INVALID_ARG, "w1_scale_inv is NULL");
+  if (partial_amax == nullptr) return fail(FP8MLP_ERR_INVALID_ARG, "partial_amax is NULL");
+  if (reinterpret_cast<uintptr_t>(partial_amax) & 3u) return fail(FP8MLP_ERR_INVALID_ARG, "partial_amax misaligned");
+  if (write_q) {
+    REQUIRE_PTR(post_fp8);
+    REQUIRE_PTR(st);
+  }
+  if (pre_debug != nullptr && (reinterpret_cast<uintptr_t>(pre_debug) & 3u))
+    return fail(FP8MLP_ERR_INVALID_ARG, "pre_debug misaligned");
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  GemmParams p{};
+  TRY(map_kmajor(&p.tmA[0], x_fp8, U8, 1, M, d, kGemmBM, "x_fp8"));
+  TRY(map_kmajor(&p.tmB[0], W1q, U8, 1, h, d, kGemmBN * kGemmBM / gemm_tile_m(GemmKind::UpQ), "W1q"));
+  TRY(map_tile32(&p.tmOut[0], post, BF16, 2, M, h, "post"));
+  if (write_q) TRY(map_tile32(&p.tmOut2, post_fp8, U8, 1, M, h, "post_fp8"));
+  fill_common(p, GemmKind::UpQ, di, M, h, d, 1);
+  p.write_q = write_q ? 1 : 0;
+  p.partial_amax = partial_amax;
+  p.pre_debug = pre_debug;
+  p.st = st;
+  p.st_in = st_x;
+  p.w_in_scale_inv = w1_scale_inv;
+  return launch(GemmKind::UpQ, p, di, stream, "up_proj_fused_fp8 launch");
+}
+
 int fp8mlp_bwd_dpre(int M, int d, int h, const uint16_t* dOut, const uint16_t* W2, const uint16_t* post,
                     uint16_t* dPre, fp8mlp_stream_t stream) {
   g_detail.clear();

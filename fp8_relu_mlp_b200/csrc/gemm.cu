@@ -8,6 +8,7 @@ namespace fp8mlp {
 using CfgUp = GemmCfg<2, kGemmBN, 5, false, false, false, Epi::UpFused>;
 using CfgDown8 = GemmCfg<2, kGemmBN, 6, true, false, false, Epi::DownScaled>;
 using CfgBf16MnB = GemmCfg<2, kGemmBN, 6, false, false, true, Epi::StoreBf16>;
+using CfgUpQ = GemmCfg<2, kGemmBN, 5, true, false, false, Epi::UpFused>;
 using CfgDPre = GemmCfg<2, kGemmBN, 3, false, false, false, Epi::DPre>;
 // dW: one long tile per CTA pair, so a light epilogue (4 warps) and more stages
 using CfgDW = GemmCfg<2, kGemmBN, 6, false, true, true, Epi::StoreF32, 4>;
@@ -67,6 +68,8 @@ int gemm_tile_m(GemmKind kind) {
       return CfgDPre::TILE_M;
     case GemmKind::DW:
       return CfgDW::TILE_M;
+    case GemmKind::UpQ:
+      return CfgUpQ::TILE_M;
   }
   return 128;
 }
@@ -83,6 +86,8 @@ cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int num_tiles, int n
       return launch_one<CfgDPre>(p, num_tiles, num_sms, s);
     case GemmKind::DW:
       return launch_one<CfgDW>(p, num_tiles, num_sms, s);
+    case GemmKind::UpQ:
+      return launch_one<CfgUpQ>(p, num_tiles, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }

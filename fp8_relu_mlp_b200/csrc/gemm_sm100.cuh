@@ -24,7 +24,8 @@
 namespace fp8mlp {
 
 enum class Epi : int {
-  UpFused = 0,     // post = bf16(relu(acc)^2), q = e4m3(post*s), partial amax
+  UpFused = 0,     // post = bf16(relu(pre)^2), q = e4m3(post*s), partial amax;
+                   // pre = acc (BF16 inputs) or acc * s_x^-1 * s_w1^-1 (e4m3 inputs)
   DownScaled = 1,  // out = bf16(acc * s^-1 * s_w^-1)
   StoreBf16 = 2,   // out = bf16(acc)
   DPre = 3,        // dPre = bf16(2 sqrt(post) * acc), post read by TMA (hardware sqrt.approx)
@@ -46,6 +47,8 @@ struct alignas(64) GemmParams {
   float* pre_debug;
   const fp8mlp_scale_state* st;
   const float* w2_scale_inv;
+  const fp8mlp_scale_state* st_in;  // UpFused on e4m3 inputs: x's delayed scale
+  const float* w_in_scale_inv;      // UpFused on e4m3 inputs: 1 / s_w1
   unsigned int* status;
   unsigned long long timeout_ns;
   int debug_flags;
@@ -325,6 +328,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
       if (p.write_q) s_up = p.st->scale;
     }
     if constexpr (C::EPI == Epi::DownScaled) comb = __fmul_rn(p.st->scale_inv, *p.w2_scale_inv);
+    // e4m3 up-projection: dequantise the accumulator before relu and the square
+    float dq = 1.f;
+    if constexpr (C::EPI == Epi::UpFused && C::FP8) dq = __fmul_rn(p.st_in->scale_inv, *p.w_in_scale_inv);
     // DPre: rounds of post prefetch started (one round = a tile's NAUX chunks,
     // ring slot c = chunk c) and how many slots the latest round has reached
     uint32_t aux_rounds = 0, aux_last = 0;
@@ -385,6 +391,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
 
         if constexpr (C::EPI == Epi::UpFused) {
           uint32_t pk[16], qk[8];
+          if constexpr (C::FP8) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__fmul_rn(__uint_as_float(v[i]), dq));
+          }
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float a = fmaxf(__uint_as_float(v[2 * i]), 0.f);

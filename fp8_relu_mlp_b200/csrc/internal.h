@@ -16,6 +16,7 @@ enum class GemmKind : int {
   Bf16MnB = 2,  // post . W2 (eval) and dPre . W1 (dX): BF16, K-major A, MN-major B
   DPre = 3,     // K5: dOut . W2^T -> dPre with the 2 sqrt(post) epilogue
   DW = 4,       // K7/K8: dPre^T . x and post^T . dOut (BF16, MN-major A/B), fp32 out
+  UpQ = 5,      // K1 on e4m3 x and W1 (dequantised in the epilogue)
 };
 constexpr int kGemmBM = 128;  // accumulator rows per CTA
 constexpr int kGemmBN = 256;  // output tile columns
@@ -77,6 +78,13 @@ cudaError_t launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, 
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, k, static_cast<KArgs>(args)...);
 }
+
+// e4m3 copies of x (delayed scale) and W1 (exact scale) for the FP8 up-projection
+constexpr int kXElemsPerBlock = 8192;  // elements of x per partial max |x|
+cudaError_t launch_quantize_x(long long n, const uint16_t* x, const fp8mlp_scale_state* st, uint8_t* xq,
+                              float* partial, cudaStream_t s);
+cudaError_t launch_w1_cache(int h, int d, const uint16_t* W1, uint8_t* W1q, float* w1_scale_inv,
+                            unsigned int* partial, unsigned int* status, cudaStream_t s);
 
 // status word symbol address on the current device
 cudaError_t status_word_address(unsigned int** ptr);

@@ -285,6 +285,89 @@ __global__ void residual_add_kernel(size_t n_vec, const uint4* __restrict__ r, c
   }
 }
 
+// x_q = e4m3(fp32(x * s_x)) with s_x = st->scale; block b also writes the
+// max |x| over its kXElemsPerBlock elements (BF16 magnitude bits: integer
+// order = value order) as the partial amax of x's delayed scale.
+__global__ void __launch_bounds__(256) quantize_x_kernel(const uint4* __restrict__ x, long long n_vec,
+                                                         const fp8mlp_scale_state* st, uint2* __restrict__ xq,
+                                                         float* __restrict__ partial) {
+  pdl_wait();
+  pdl_launch_dependents();
+  __shared__ unsigned int wmax[8];
+  const float s = st->scale;
+  const long long base = static_cast<long long>(blockIdx.x) * (kXElemsPerBlock / 8);
+  unsigned int m = 0;
+#pragma unroll
+  for (int k = 0; k < kXElemsPerBlock / 8 / 256; ++k) {
+    const long long i = base + k * 256 + threadIdx.x;
+    if (i < n_vec) {
+      const uint4 v = x[i];
+      const unsigned int w4[4] = {v.x, v.y, v.z, v.w};
+      uint32_t q[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const uint32_t a = pack_e4m3x2(__fmul_rn(bf16lo_to_f32(w4[2 * j]), s), __fmul_rn(bf16hi_to_f32(w4[2 * j]), s));
+        const uint32_t b = pack_e4m3x2(__fmul_rn(bf16lo_to_f32(w4[2 * j + 1]), s),
+                                       __fmul_rn(bf16hi_to_f32(w4[2 * j + 1]), s));
+        q[j] = a | (b << 16);
+      }
+      xq[i] = make_uint2(q[0], q[1]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        m = max(m, w4[j] & 0x7FFFu);
+        m = max(m, (w4[j] >> 16) & 0x7FFFu);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned int r = 0;
+    for (int w = 0; w < 8; ++w) r = max(r, wmax[w]);
+    partial[blockIdx.x] = __uint_as_float(r << 16);
+  }
+}
+
+// W1q = e4m3(fp32(W1 * s_w1)), s_w1 = 448 / max|W1| from the partial maxima;
+// flat (W1 [h,d] is already K-major for the up-projection).
+__global__ void __launch_bounds__(256) w1_quant_kernel(long long n_vec, const uint4* __restrict__ W1,
+                                                       uint2* __restrict__ W1q, float* w1_scale_inv,
+                                                       const unsigned int* __restrict__ partial, int nparts,
+                                                       unsigned int* status) {
+  pdl_wait();
+  pdl_launch_dependents();
+  __shared__ unsigned int wmax[8];
+  unsigned int am = 0;
+  for (int i = threadIdx.x; i < nparts; i += 256) am = max(am, partial[i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, o));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = am;
+  __syncthreads();
+  am = 0;
+  for (int w = 0; w < 8; ++w) am = max(am, wmax[w]);
+  bool degenerate;
+  const float s = w2_scale_from(am, &degenerate);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    w1_scale_inv[0] = __fdiv_rn(1.f, s);
+    if (degenerate) atomicOr(status, STATUS_W2_DEGENERATE);
+  }
+  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n_vec; i += static_cast<long long>(gridDim.x) * 256) {
+    const uint4 v = W1[i];
+    const unsigned int w4[4] = {v.x, v.y, v.z, v.w};
+    uint32_t q[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t a = pack_e4m3x2(__fmul_rn(bf16lo_to_f32(w4[2 * j]), s), __fmul_rn(bf16hi_to_f32(w4[2 * j]), s));
+      const uint32_t b = pack_e4m3x2(__fmul_rn(bf16lo_to_f32(w4[2 * j + 1]), s),
+                                     __fmul_rn(bf16hi_to_f32(w4[2 * j + 1]), s));
+      q[j] = a | (b << 16);
+    }
+    W1q[i] = make_uint2(q[0], q[1]);
+  }
+}
+
 int grid_for(size_t work, int per_block, int num_sms, int blocks_per_sm) {
   size_t g = (work + per_block - 1) / per_block;
   const size_t cap = static_cast<size_t>(num_sms) * blocks_per_sm;
@@ -319,6 +402,29 @@ cudaError_t launch_w2_cache(int h, int d, const uint16_t* W2, uint8_t* W2q_t, fl
   dim3 grid((d + 63) / 64, (h + 63) / 64);
   e = launch_pdl(w2_quant_t_kernel, grid, dim3(256), 0, s, h, d, W2, W2q_t, w2_scale_inv,
                  static_cast<const unsigned int*>(partial), nparts, status);
+  count_launches(1);
+  return e;
+}
+
+cudaError_t launch_quantize_x(long long n, const uint16_t* x, const fp8mlp_scale_state* st, uint8_t* xq,
+                              float* partial, cudaStream_t s) {
+  const int nparts = static_cast<int>((n + kXElemsPerBlock - 1) / kXElemsPerBlock);
+  const cudaError_t e = launch_pdl(quantize_x_kernel, dim3(nparts), dim3(256), 0, s,
+                                   reinterpret_cast<const uint4*>(x), n / 8, st, reinterpret_cast<uint2*>(xq), partial);
+  count_launches(1);
+  return e;
+}
+
+cudaError_t launch_w1_cache(int h, int d, const uint16_t* W1, uint8_t* W1q, float* w1_scale_inv,
+                            unsigned int* partial, unsigned int* status, cudaStream_t s) {
+  const long long n = static_cast<long long>(h) * d;
+  const int nparts = static_cast<int>((n + kW2ElemsPerBlock - 1) / kW2ElemsPerBlock);
+  cudaError_t e = launch_pdl(w2_amax_kernel, dim3(nparts), dim3(256), 0, s, reinterpret_cast<const uint4*>(W1), n / 8,
+                             partial);
+  count_launches(1);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(w1_quant_kernel, dim3(nparts), dim3(256), 0, s, n / 8, reinterpret_cast<const uint4*>(W1),
+                 reinterpret_cast<uint2*>(W1q), w1_scale_inv, static_cast<const unsigned int*>(partial), nparts, status);
   count_launches(1);
   return e;
 }

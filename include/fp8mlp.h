@@ -158,6 +158,38 @@ int fp8mlp_mlp_fwd(int M, int d, int h, const uint16_t* x, const uint16_t* W1, c
                    uint8_t* post_fp8, float* partial_amax, uint16_t* out, float* pre_debug, int flags,
                    fp8mlp_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * FP8 up-projection ("NanoGPT Speedrun (Track 1)", From Unoptimized, item 5:
+ * the MLP GEMMs in e4m3 in the training forward, BF16 backward).  x and W1
+ * enter the up-projection as e4m3 copies: x under its own delayed scale s_x
+ * (the same recurrence as post's, from max |x| of the previous step), W1
+ * under an exact cache scale.  The backward keeps the BF16 x and W1.
+ * ------------------------------------------------------------------------ */
+
+/* x_fp8 = e4m3_satfinite(fp32(x * st_x->scale)), x [M,d] bf16 -> x_fp8 [M,d];
+ * partial_amax_x[b] = max |x| over elements [8192 b, 8192 b + 8192) of the
+ * flat x (fp8mlp_x_partial_amax_count entries; reduce them with
+ * fp8mlp_amax_reduce_update_scale into st_x for the next step). */
+int fp8mlp_quantize_x(int M, int d, const uint16_t* x, const fp8mlp_scale_state* st_x, uint8_t* x_fp8,
+                      float* partial_amax_x, fp8mlp_stream_t stream);
+int fp8mlp_x_partial_amax_count(int M, int d);
+
+/* Exact FP8 copy of W1 (not transposed; W1 [h,d] is K-major for the
+ * up-projection): s_w1 = fp32(448 / max|W1|) (1 if 0 or not finite),
+ * W1q[i,k] = e4m3_satfinite(fp32(W1[i,k] * s_w1)), w1_scale_inv[0] = 1/s_w1.
+ * workspace: fp8mlp_workspace_size(0,d,h) bytes, as for the W2 cache. */
+int fp8mlp_w1_fp8_cache_refresh(int h, int d, const uint16_t* W1, uint8_t* W1q, float* w1_scale_inv,
+                                void* workspace, fp8mlp_stream_t stream);
+
+/* fp8mlp_up_proj_fused on e4m3 inputs: the accumulator is dequantised in the
+ * epilogue, pre = fp32(acc * fp32(st_x->scale_inv * w1_scale_inv[0])), then
+ * post, the FP8 copy of post and the partial amax exactly as in
+ * fp8mlp_up_proj_fused.  x_fp8 [M,d], W1q [h,d] e4m3. */
+int fp8mlp_up_proj_fused_fp8(int M, int d, int h, const uint8_t* x_fp8, const uint8_t* W1q,
+                             const float* w1_scale_inv, const fp8mlp_scale_state* st_x, const fp8mlp_scale_state* st,
+                             uint16_t* post, uint8_t* post_fp8, float* partial_amax, float* pre_debug, int flags,
+                             fp8mlp_stream_t stream);
+
 /* Number of row blocks and column blocks of the partial-amax tensor for an
  * [M,h] post, and the block size in rows / columns.  Returns FP8MLP_OK. */
 int fp8mlp_partial_amax_shape(int M, int h, int* row_blocks, int* col_blocks, int* block_rows,

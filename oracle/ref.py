@@ -424,3 +424,41 @@ def stack_backward(saved, layers, dr_top):
         drn = rmsnorm_bwd(S["r"], g["dX"])
         dr = bf16_bits_from_f32(f32(bf16_to_f64(dr) + drn))
     return dr, grads
+
+
+# ----------------------------------------------------------------------------
+# FP8 up-projection ("NanoGPT Speedrun (Track 1)", From Unoptimized, item 5:
+# the MLP GEMMs in e4m3 in the training forward, BF16 backward).  Both inputs
+# of the up-projection are e4m3 copies: x under its own delayed scale s_x (the
+# same recurrence as post's, over max |x|), W1 under an exact cache scale.
+# ----------------------------------------------------------------------------
+
+
+def quantise_x(x, s_x):
+    """x_q = e4m3(fp32(x * s_x)) of the BF16 x, and max |x| (the amax that
+    drives the next step's s_x)."""
+    X = bf16_to_f64(x).astype(np.float32)
+    q = e4m3_bits_from_f32((X * np.float32(s_x)).astype(np.float32))
+    a = np.float32(np.abs(X).max()) if X.size else np.float32(0.0)
+    return q, a
+
+
+def w1_cache(W1):
+    """Exact FP8 copy of W1 (not transposed: W1 [h,d] is already K-major for
+    the up-projection): s_w1 = fp32(448 / max|W1|), W1q = e4m3(fp32(W1 s_w1)).
+    Returns (W1q [h,d] uint8, s_w1, s_w1_inv)."""
+    W = bf16_to_f64(W1)
+    a = np.float32(np.abs(W).max()) if W.size else np.float32(0.0)
+    s = np.float32(np.float32(E4M3_MAX) / a) if (np.isfinite(a) and a > 0) else np.float32(1.0)
+    q = e4m3_bits_from_f32((W.astype(np.float32) * s).astype(np.float32))
+    return q, s, np.float32(np.float32(1.0) / s)
+
+
+def up_proj_fp8(x_q, W1q, s_x_inv, s_w1_inv):
+    """pre = fp32( fp32(sum_k dec(x_q[m,k]) dec(W1q[i,k])) * fp32(s_x^-1 s_w1^-1) ).
+
+    The accumulator is fp32 in the kernel; the dequantising factor is applied
+    to it in the epilogue, before relu and the square."""
+    comb = np.float32(np.float32(s_x_inv) * np.float32(s_w1_inv))
+    acc = f32(e4m3_to_f64(x_q) @ e4m3_to_f64(W1q).T)
+    return (acc * comb).astype(np.float32).astype(np.float64)

@@ -614,3 +614,110 @@ def test_data_parallel_step_single_rank():
         dist.destroy_process_group()
     for k in ("post", "post_fp8", "out", "dPre", "dX", "dW1", "dW2", "state", "W2q_t"):
         assert torch.equal(getattr(plain, k), getattr(b, k)), k
+
+
+# ---------------------------------------------------------------------------
+# FP8 up-projection: x quantiser, W1 cache, e4m3 up-projection
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,d", [(1, 64), (300, 80), (16384, 768)])
+def test_quantize_x_bit_exact(M, d):
+    x = synth.make_problem(M, d, 16, seed=M, x_dist="student_t3" if M > 1000 else "normal")["x"]
+    s = np.float32(448.0 / 29.0)
+    st = _state(2.0, float(s))
+    n = A.fp8mlp_x_partial_amax_count(M, d)
+    xq = Guarded((M, d), torch.uint8)
+    pa = Guarded((n,), torch.float32)
+    A.fp8mlp_quantize_x(M, d, dev_bf16(x), st, xq.t, pa.t)
+    torch.cuda.synchronize()
+    q_o, a_o = ref.quantise_x(x, s)
+    assert np.array_equal(host_bits(xq.t), q_o)
+    flat = np.abs(ref.bf16_to_f64(x)).reshape(-1)
+    want = [np.float32(flat[i * 8192:(i + 1) * 8192].max()) for i in range(n)]
+    assert np.array_equal(host_bits(pa.t), np.array(want, np.float32))
+    assert host_bits(pa.t).max() == a_o
+    assert xq.intact() and pa.intact()
+
+
+@pytest.mark.parametrize("h,d", [(256, 64), (272, 80), (3072, 768)])
+def test_w1_cache_bit_exact(h, d):
+    W1 = synth.make_problem(1, d, h, seed=h + 1)["W1"]
+    Wq = Guarded((h, d), torch.uint8)
+    inv = Guarded((4,), torch.float32)
+    ws = torch.empty(A.fp8mlp_workspace_size(0, d, h), dtype=torch.uint8, device="cuda")
+    A.fp8mlp_w1_fp8_cache_refresh(h, d, dev_bf16(W1), Wq.t, inv.t, ws)
+    torch.cuda.synchronize()
+    q_o, s_o, si_o = ref.w1_cache(W1)
+    assert np.array_equal(host_bits(Wq.t), q_o)
+    assert host_bits(inv.t)[0] == si_o
+    assert Wq.intact() and inv.intact()
+
+
+@pytest.mark.parametrize("M,d,h", SHAPES)
+def test_up_proj_fp8_bit_exact_grid(M, d, h):
+    # grid inputs with power-of-two scales: both quantisations and the fp32
+    # accumulation are exact, so pre, post, the FP8 copy and the partial amax
+    # are unique
+    P = synth.make_problem(M, d, h, seed=M + 3, x_dist="grid", w_dist="grid")
+    st_x = _state(2.0, 16.0)
+    st = _state(2.0, float(np.float32(448.0 / 37.0)))
+    xq_o, _ = ref.quantise_x(P["x"], 16.0)
+    W1q_o = ref.e4m3_bits_from_f32((ref.bf16_to_f64(P["W1"]) * 1024.0).astype(np.float32))
+    n = A.fp8mlp_x_partial_amax_count(M, d)
+    xq = torch.empty(M, d, dtype=torch.uint8, device="cuda")
+    pax = torch.empty(n, device="cuda")
+    A.fp8mlp_quantize_x(M, d, dev_bf16(P["x"]), st_x, xq, pax)
+    post = Guarded((M, h), torch.bfloat16)
+    q = Guarded((M, h), torch.uint8)
+    rb, cb, _, _ = A.fp8mlp_partial_amax_shape(M, h)
+    pa = Guarded((rb, cb), torch.float32)
+    pre = Guarded((M, h), torch.float32)
+    A.fp8mlp_up_proj_fused_fp8(M, d, h, xq, dev_u8(W1q_o), dev_f32(np.array([1 / 1024.0, 0, 0, 0], np.float32)),
+                               st_x, st, post.t, q.t, pa.t, pre.t, 0)
+    torch.cuda.synchronize()
+    assert np.array_equal(host_bits(xq), xq_o)
+    pre_o = ref.up_proj_fp8(xq_o, W1q_o, np.float32(1 / 16.0), np.float32(1 / 1024.0))
+    assert np.array_equal(host_bits(pre.t), pre_o.astype(np.float32))
+    assert np.array_equal(pre_o, ref.up_proj(P["x"], P["W1"]))   # exact: equals the BF16 up-projection
+    post_o = ref.relu2_post(pre_o)
+    assert np.array_equal(host_bits(post.t), post_o)
+    assert np.array_equal(host_bits(q.t), ref.quantise_post(post_o, np.float32(448.0 / 37.0)))
+    assert np.array_equal(host_bits(pa.t), _pa_oracle(post_o, M, h))
+    assert post.intact() and q.intact() and pa.intact() and pre.intact()
+
+
+@pytest.mark.parametrize("M,d,h", [(256, 64, 256), (1000, 768, 3072)])
+def test_fp8_up_forward_normal_inputs(M, d, h):
+    from fp8_relu_mlp_b200.block import MLPBlock
+    P = synth.make_problem(M, d, h, seed=123)
+    b = MLPBlock(M, d, h, fp8_up=True)
+    for k in ("x", "W1", "W2"):
+        getattr(b, k).copy_(MLPBlock.bits_to_bf16(P[k], b.device))
+    b.refresh_w2_cache()
+    b.refresh_w1_cache()
+    b.calibrate()
+    b.forward()
+    torch.cuda.synchronize()
+    sx = b.read_state(b.state_x)
+    sp = b.read_state()
+    # the oracle runs the same FP8 pipeline with the GPU's calibrated scales
+    # taken from the oracle's own calibration on the same inputs
+    xq_cal, ax = ref.quantise_x(P["x"], 1.0)
+    st_x = ref.scale_update(ref.scale_state_init(2.0, 1.0), ax)
+    assert np.float32(sx["scale"]) == st_x["scale"]          # amax of x is exact, so the x-scale is bit-exact
+    W1q_o, _, s_w1i = ref.w1_cache(P["W1"])
+    xq_o, _ = ref.quantise_x(P["x"], st_x["scale"])
+    pre_o = ref.up_proj_fp8(xq_o, W1q_o, st_x["scale_inv"], s_w1i)
+    st_p = ref.scale_update(ref.scale_state_init(2.0, 1.0), ref.amax(ref.relu2_post(pre_o)))
+    assert abs(sp["scale"] / float(st_p["scale"]) - 1) <= 2.0 ** -7
+    W2q_o, _, s_w2i = ref.w2_cache(P["W2"])
+    A.fp8mlp_scale_state_init(b.state, 2.0, float(st_p["scale"]))
+    b.forward()
+    torch.cuda.synchronize()
+    post_o = ref.relu2_post(pre_o)
+    out_o = ref.down_proj_fp8(ref.quantise_post(post_o, st_p["scale"]), W2q_o, st_p["scale_inv"], s_w2i)
+    assert rel_fro(ref.bf16_to_f64(host_bits(b.post)), ref.bf16_to_f64(post_o)) < 1e-2
+    assert rel_fro(ref.bf16_to_f64(host_bits(b.out)), ref.bf16_to_f64(out_o)) < TOL_OUT
+    # against the exact BF16 network: the FP8 up- and down-projection error
+    exact = ref.bf16_to_f64(ref.down_proj_bf16(ref.relu2_post(ref.up_proj(P["x"], P["W1"])), P["W2"]))
+    assert rel_fro(ref.bf16_to_f64(host_bits(b.out)), exact) < 8e-2

@@ -486,3 +486,50 @@ def test_synth_is_deterministic():
     gx = synth.make_problem(64, 32, 128, seed=5, x_dist="grid", w_dist="grid")
     X = ref.bf16_to_f64(gx["x"])
     assert np.array_equal(X * 4, np.round(X * 4)) and np.abs(X).max() <= 2
+
+
+# ---------------------------------------------------------------------------
+# FP8 up-projection
+# ---------------------------------------------------------------------------
+
+def test_quantise_x_matches_library_and_amax():
+    g = np.random.default_rng(21)
+    x = _bf16(g.standard_normal((64, 48)) * 3)
+    for s in [1.0, 37.25, 448.0 / 11.0]:
+        q, a = ref.quantise_x(x, s)
+        v = (ref.bf16_to_f64(x).astype(np.float32) * np.float32(s)).astype(np.float32)
+        assert np.array_equal(q, _e4m3_lib(v))
+        assert a == np.float32(np.abs(ref.bf16_to_f64(x)).max())
+    # negative values keep their sign bit
+    q, _ = ref.quantise_x(_bf16(np.array([[-1.0, 1.0]], np.float32)), 1.0)
+    assert list(q[0]) == [0xB8, 0x38]
+
+
+def test_w1_cache_matches_library():
+    g = np.random.default_rng(22)
+    W1 = _bf16(g.standard_normal((96, 64)) / 8)
+    q, s, si = ref.w1_cache(W1)
+    W = ref.bf16_to_f64(W1)
+    assert q.shape == W1.shape
+    assert s == _nearest_f32(Fraction(448) / Fraction(float(np.abs(W).max())))
+    assert np.array_equal(q, _e4m3_lib((W.astype(np.float32) * s).astype(np.float32)))
+    assert si == _nearest_f32(Fraction(1) / Fraction(float(s)))
+
+
+def test_up_proj_fp8_bruteforce_and_exact_grid():
+    g = np.random.default_rng(23)
+    xq = g.integers(0, 256, (5, 8)).astype(np.uint8)
+    Wq = g.integers(0, 256, (7, 8)).astype(np.uint8)
+    xq[(xq & 0x7F) == 0x7F] = 0x21
+    Wq[(Wq & 0x7F) == 0x7F] = 0x22
+    sxi, swi = np.float32(1 / 5), np.float32(1 / 9)
+    got = ref.up_proj_fp8(xq, Wq, sxi, swi)
+    want = _brute(ref.e4m3_to_f64(xq), ref.e4m3_to_f64(Wq)) * float(np.float32(sxi * swi))
+    np.testing.assert_allclose(got, want, rtol=2e-7)
+    # power-of-two scales on grid values: quantisation and dequantisation are
+    # exact, so the FP8 up-projection equals the BF16 one
+    x = _bf16(g.integers(-8, 9, (6, 16)) / 4.0)
+    W1 = _bf16(g.integers(-16, 17, (10, 16)) / 256.0)
+    xq2, _ = ref.quantise_x(x, 16.0)
+    W1q = ref.e4m3_bits_from_f32((ref.bf16_to_f64(W1) * 1024.0).astype(np.float32))
+    assert np.array_equal(ref.up_proj_fp8(xq2, W1q, 1 / 16.0, 1 / 1024.0), ref.up_proj(x, W1))
