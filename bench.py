@@ -47,7 +47,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="step16k", choices=["step16k", "train49k", "heavytail", "stack9"])
+    ap.add_argument("--workload", default="step16k", choices=["step16k", "train49k", "heavytail", "stack9", "qkv16k"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -565,6 +565,107 @@ def run_dp(a, W, world, rank, local_rank, blk, flush, dist, peaks, fp8_peak, fp8
     return None
 
 
+def run_linear(a, W, world, rank, local_rank):
+    """The FP8 linear layer on the same kernels (attention QKV projection
+    shape): per step the x quantiser, the e4m3 GEMM with its dequantising
+    epilogue, the x-scale update, the weight-cache refresh and the BF16
+    backward (dX, dW); one CUDA graph per step."""
+    import numpy as np
+    import torch
+    from fp8_relu_mlp_b200 import _abi as A
+    from fp8_relu_mlp_b200 import synth
+    from fp8_relu_mlp_b200.block import MLPBlock
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    A.fp8mlp_set_programmatic_launch(not a.no_pdl)
+    M, K, N = W.M, W.d, W.h
+    peaks = load_peaks()
+    fp8_peak, fp8_src = measure_fp8_peak(torch, peaks["bf16_tflops"])
+    P = synth.make_problem(M, K, N, seed=rank)
+    bf, u8 = torch.bfloat16, torch.uint8
+    x = MLPBlock.bits_to_bf16(P["x"], dev)
+    Wt = MLPBlock.bits_to_bf16(P["W1"], dev)
+    g = synth.rng(5)
+    dY = MLPBlock.bits_to_bf16(synth.to_bf16_bits(g.standard_normal((M, N), dtype=np.float32)), dev)
+    st = torch.zeros(8, device=dev)
+    A.fp8mlp_scale_state_init(st, W.margin, 1.0)
+    xq = torch.empty(M, K, dtype=u8, device=dev)
+    npx = A.fp8mlp_x_partial_amax_count(M, K)
+    pax = torch.empty(npx, device=dev)
+    Wq = torch.empty(N, K, dtype=u8, device=dev)
+    winv = torch.ones(4, device=dev)
+    ws = torch.empty(A.fp8mlp_workspace_size(0, K, N), dtype=u8, device=dev)
+    y = torch.empty(M, N, dtype=bf, device=dev)
+    dX = torch.empty(M, K, dtype=bf, device=dev)
+    dW = torch.empty(N, K, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=u8, device=dev)
+    A.fp8mlp_weight_fp8_cache_refresh(N, K, Wt, Wq, winv, ws)
+    A.fp8mlp_quantize_x(M, K, x, st, xq, pax)
+    A.fp8mlp_amax_reduce_update_scale(pax, npx, st)
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record()
+        mark(0)
+        A.fp8mlp_quantize_x(M, K, x, st, xq, pax)
+        mark(1)
+        A.fp8mlp_linear_fwd_fp8(M, K, N, xq, Wq, winv, st, y)
+        mark(2)
+        A.fp8mlp_amax_reduce_update_scale(pax, npx, st)
+        A.fp8mlp_linear_bwd(M, K, N, x, Wt, dY, dX, dW)
+        A.fp8mlp_weight_fp8_cache_refresh(N, K, Wt, Wq, winv, ws)
+        mark(3)
+
+    step()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True, external=not a.eager) for _ in range(4)]
+    n_cap0 = A.fp8mlp_kernel_launch_count()
+    graph = None
+    if not a.eager:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step(ev)
+    kps = A.fp8mlp_kernel_launch_count() - n_cap0
+
+    def run():
+        graph.replay() if graph is not None else step(ev)
+
+    for _ in range(max(a.warmup, 3)):
+        flush.zero_()
+        run()
+    torch.cuda.synchronize()
+    step_ms, fwd_ms = [], []
+    with ClockSampler(local_rank) as clk:
+        for _ in range(a.steps):
+            flush.zero_()
+            run()
+            ev[3].synchronize()
+            step_ms.append(ev[0].elapsed_time(ev[3]))
+            fwd_ms.append(ev[1].elapsed_time(ev[2]))
+    total_s = sum(step_ms) * 1e-3
+    F = 2 * M * K * N
+    fwd_s = statistics.mean(fwd_ms) * 1e-3
+    achieved = F / fwd_s / 1e12
+    roof = (F / (fp8_peak * 1e12) + 2 * F / (peaks["bf16_tflops"] * 1e12)
+            + (2 * M * K + M * K) / (peaks["hbm_gbs"] * 1e9))
+    if rank == 0:
+        line = {
+            "metric": "FP8 linear (attention QKV projection) fwd+bwd tokens/s and % of FP8/BF16 roofline",
+            "value": M * a.steps / total_s, "unit": "tokens/s", "n_gpus": 1, "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": total_s / a.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 forward, bf16 backward (fp32 accumulate)", "data": "synthetic",
+            "config": dict(config_of(W), K=K, N=N),
+            "roofline": {"bound": "tensor", "kernel": "linear_fwd_fp8", "achieved": achieved, "peak": fp8_peak,
+                         "unit": "TFLOP/s", "frac": achieved / fp8_peak, "traffic": None, "peak_source": fp8_src},
+            "step_roofline": {"roofline_ms": roof * 1e3, "measured_ms": total_s / a.steps * 1e3,
+                              "frac": roof / (total_s / a.steps)},
+            "clocks": clk.summary(), "gpu_launches": int(kps * a.steps),
+            "launch_mode": "eager" if graph is None else "cuda_graph",
+        }
+        print(json.dumps(line), flush=True)
+
+
 def run_stack(a, W, world, rank, local_rank):
     """The 9-layer stack workload: per step, forward through every layer
     (RMSNorm, block, residual), backward through every layer, the scale
@@ -800,7 +901,9 @@ def main():
     if a.impl == "reference":
         run_reference(a, W, world, rank)
         return 0
-    if W.layers > 1:
+    if W.name.startswith("qkv"):
+        run_linear(a, W, world, rank, local_rank)
+    elif W.layers > 1:
         run_stack(a, W, world, rank, local_rank)
     else:
         run_ours(a, W, world, rank, local_rank)

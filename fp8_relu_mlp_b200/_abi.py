@@ -62,6 +62,9 @@ _SIGS = {
     "fp8mlp_x_partial_amax_count": [_i, _i],
     "fp8mlp_w1_fp8_cache_refresh": [_i, _i, _p, _p, _p, _p, _p],
     "fp8mlp_up_proj_fused_fp8": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _p],
+    "fp8mlp_linear_fwd_fp8": [_i, _i, _i, _p, _p, _p, _p, _p, _p],
+    "fp8mlp_weight_fp8_cache_refresh": [_i, _i, _p, _p, _p, _p, _p],
+    "fp8mlp_linear_bwd": [_i, _i, _i, _p, _p, _p, _p, _p, _p],
     "fp8mlp_bwd_dx": [_i, _i, _i, _p, _p, _p, _p],
     "fp8mlp_bwd_dw": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p],
     "fp8mlp_mlp_bwd": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p],
@@ -206,6 +209,20 @@ def fp8mlp_up_proj_fused_fp8(M, d, h, x_fp8, W1q, w1_scale_inv, st_x, st, post, 
                              pre_debug=None, flags=0, stream=None):
     return _call("fp8mlp_up_proj_fused_fp8", M, d, h, _ptr(x_fp8), _ptr(W1q), _ptr(w1_scale_inv), _ptr(st_x),
                  _ptr(st), _ptr(post), _ptr(post_fp8), _ptr(partial_amax), _ptr(pre_debug), flags, _stream(stream))
+
+
+def fp8mlp_linear_fwd_fp8(M, K, N, x_fp8, Wq, w_scale_inv, st_x, y, stream=None):
+    return _call("fp8mlp_linear_fwd_fp8", M, K, N, _ptr(x_fp8), _ptr(Wq), _ptr(w_scale_inv), _ptr(st_x), _ptr(y),
+                 _stream(stream))
+
+
+def fp8mlp_weight_fp8_cache_refresh(N, K, W, Wq, w_scale_inv, workspace, stream=None):
+    return _call("fp8mlp_weight_fp8_cache_refresh", N, K, _ptr(W), _ptr(Wq), _ptr(w_scale_inv), _ptr(workspace),
+                 _stream(stream))
+
+
+def fp8mlp_linear_bwd(M, K, N, x, W, dY, dX, dW, stream=None):
+    return _call("fp8mlp_linear_bwd", M, K, N, _ptr(x), _ptr(W), _ptr(dY), _ptr(dX), _ptr(dW), _stream(stream))
 
 
 def fp8mlp_bwd_dpre(M, d, h, dOut, W2, post, dPre, stream=None):

@@ -362,6 +362,11 @@ int fp8mlp_quantize_x(int M, int d, const uint16_t* x, const fp8mlp_scale_state*
   return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "quantize_x launch");
 }
 
+int fp8mlp_weight_fp8_cache_refresh(int N, int K, const uint16_t* W, uint8_t* Wq, float* w_scale_inv,
+                                    void* workspace, fp8mlp_stream_t stream) {
+  return fp8mlp_w1_fp8_cache_refresh(N, K, W, Wq, w_scale_inv, workspace, stream);
+}
+
 int fp8mlp_w1_fp8_cache_refresh(int h, int d, const uint16_t* W1, uint8_t* W1q, float* w1_scale_inv,
                                 void* workspace, fp8mlp_stream_t stream) {
   g_detail.clear();
@@ -414,6 +419,63 @@ int fp8mlp_up_proj_fused_fp8(int M, int d, int h, const uint8_t* x_fp8, const ui
   p.st_in = st_x;
   p.w_in_scale_inv = w1_scale_inv;
   return launch(GemmKind::UpQ, p, di, stream, "up_proj_fused_fp8 launch");
+}
+
+int fp8mlp_linear_fwd_fp8(int M, int K, int N, const uint8_t* x_fp8, const uint8_t* Wq, const float* w_scale_inv,
+                          const fp8mlp_scale_state* st_x, uint16_t* y, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, N, K));
+  if (M == 0) return FP8MLP_OK;
+  REQUIRE_PTR(x_fp8);
+  REQUIRE_PTR(Wq);
+  REQUIRE_PTR(st_x);
+  REQUIRE_PTR(y);
+  if (w_scale_inv == nullptr) return fail(FP8MLP_ERR_INVALID_ARG, "w_scale_inv is NULL");
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  GemmParams p{};
+  TRY(map_kmajor(&p.tmA[0], x_fp8, U8, 1, M, K, kGemmBM, "x_fp8"));
+  TRY(map_kmajor(&p.tmB[0], Wq, U8, 1, N, K, kGemmBN * kGemmBM / gemm_tile_m(GemmKind::Down8), "Wq"));
+  TRY(map_tile32(&p.tmOut[0], y, BF16, 2, M, N, "y"));
+  fill_common(p, GemmKind::Down8, di, M, N, K, 1);
+  p.st = st_x;
+  p.w2_scale_inv = w_scale_inv;
+  return launch(GemmKind::Down8, p, di, stream, "linear_fwd_fp8 launch");
+}
+
+int fp8mlp_linear_bwd(int M, int K, int N, const uint16_t* x, const uint16_t* W, const uint16_t* dY, uint16_t* dX,
+                      float* dW, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, N, K));
+  REQUIRE_PTR(dW);
+  if (M == 0) {
+    DeviceInfo* di = nullptr;
+    TRY(current_device(&di));
+    const cudaError_t e = cudaMemsetAsync(dW, 0, sizeof(float) * static_cast<size_t>(N) * K, stream);
+    return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "linear_bwd memset");
+  }
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(W);
+  REQUIRE_PTR(dY);
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  if (dX != nullptr) {
+    REQUIRE_PTR(dX);
+    // dX[M,K] = dY[M,N] . W[N,K]: contraction over N, W as an MN-major B operand
+    GemmParams p{};
+    TRY(map_kmajor(&p.tmA[0], dY, BF16, 2, M, N, kGemmBM, "dY"));
+    TRY(map_mnmajor(&p.tmB[0], W, N, K, "W"));
+    TRY(map_tile32(&p.tmOut[0], dX, BF16, 2, M, K, "dX"));
+    fill_common(p, GemmKind::Bf16MnB, di, M, K, N, 1);
+    TRY(launch(GemmKind::Bf16MnB, p, di, stream, "linear_bwd dX launch"));
+  }
+  // dW[N,K] = dY^T . x: contraction over the M tokens, both operands MN-major
+  GemmParams p{};
+  TRY(map_mnmajor(&p.tmA[0], dY, M, N, "dY"));
+  TRY(map_mnmajor(&p.tmB[0], x, M, K, "x"));
+  TRY(map_tile32(&p.tmOut[0], dW, F32, 4, N, K, "dW"));
+  fill_common(p, GemmKind::DW, di, N, K, M, 1);
+  return launch(GemmKind::DW, p, di, stream, "linear_bwd dW launch");
 }
 
 int fp8mlp_bwd_dpre(int M, int d, int h, const uint16_t* dOut, const uint16_t* W2, const uint16_t* post,

@@ -67,6 +67,10 @@ WORKLOADS = {
         "stack9", M=131072, d=768, h=3072, layers=9,
         description="9-layer stack of 768-dim ReLU^2 MLP blocks, M=131072 "
                     "(64x2048), BF16 residual r0~N(0,1), per-layer RMSNorm"),
+    "qkv16k": Workload(
+        "qkv16k", M=16384, d=768, h=2304,
+        description="FP8 linear layer y = x W^T as the attention QKV projection: M=16384 tokens, "
+                    "K=768, N=2304 (3x768), e4m3 forward, BF16 backward"),
     "heavytail": Workload(
         "heavytail", M=65536, d=1024, h=4096, steps=30, x_dist="student_t3",
         spike_steps=(9, 19, 29), spike_factor=2.0,

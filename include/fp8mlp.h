@@ -190,6 +190,29 @@ int fp8mlp_up_proj_fused_fp8(int M, int d, int h, const uint8_t* x_fp8, const ui
                              uint16_t* post, uint8_t* post_fp8, float* partial_amax, float* pre_debug, int flags,
                              fp8mlp_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Generic FP8 linear layer y = x . W^T (nn.Linear(K, N).weight = W [N,K]) on
+ * the same kernels: the attention QKV / output projections that "NanoGPT
+ * Speedrun (Track 1)", Changes vs Record #83, item 1 runs in e4m3 in the
+ * forward (BF16 backward, BF16 at eval).  x_fp8 from fp8mlp_quantize_x (its
+ * own delayed scale st_x), Wq from fp8mlp_weight_fp8_cache_refresh.
+ * ------------------------------------------------------------------------ */
+
+/* y[m,n] = bf16( fp32( sum_k x_fp8[m,k] Wq[n,k] ) * fp32(st_x->scale_inv * w_scale_inv[0]) ),
+ * x_fp8 [M,K] e4m3, Wq [N,K] e4m3, y [M,N] bf16.  K and N multiples of 16. */
+int fp8mlp_linear_fwd_fp8(int M, int K, int N, const uint8_t* x_fp8, const uint8_t* Wq, const float* w_scale_inv,
+                          const fp8mlp_scale_state* st_x, uint16_t* y, fp8mlp_stream_t stream);
+
+/* Exact FP8 copy of a weight W [N,K] (= fp8mlp_w1_fp8_cache_refresh with
+ * N, K for h, d). */
+int fp8mlp_weight_fp8_cache_refresh(int N, int K, const uint16_t* W, uint8_t* Wq, float* w_scale_inv,
+                                    void* workspace, fp8mlp_stream_t stream);
+
+/* BF16 backward of the linear layer: dX = bf16(dY . W) [M,K] (skipped when
+ * dX is NULL) and dW = fp32(dY^T . x) [N,K].  x [M,K], W [N,K], dY [M,N]. */
+int fp8mlp_linear_bwd(int M, int K, int N, const uint16_t* x, const uint16_t* W, const uint16_t* dY, uint16_t* dX,
+                      float* dW, fp8mlp_stream_t stream);
+
 /* Number of row blocks and column blocks of the partial-amax tensor for an
  * [M,h] post, and the block size in rows / columns.  Returns FP8MLP_OK. */
 int fp8mlp_partial_amax_shape(int M, int h, int* row_blocks, int* col_blocks, int* block_rows,

@@ -462,3 +462,23 @@ def up_proj_fp8(x_q, W1q, s_x_inv, s_w1_inv):
     comb = np.float32(np.float32(s_x_inv) * np.float32(s_w1_inv))
     acc = f32(e4m3_to_f64(x_q) @ e4m3_to_f64(W1q).T)
     return (acc * comb).astype(np.float32).astype(np.float64)
+
+
+# ----------------------------------------------------------------------------
+# Generic FP8 linear layer (attention QKV / output projections in e4m3 in the
+# forward, BF16 backward: "NanoGPT Speedrun (Track 1)", Changes vs Record #83,
+# item 1).  y = x . W^T with W [N,K] (nn.Linear weight layout).
+# ----------------------------------------------------------------------------
+
+
+def linear_fp8(x_q, Wq, s_x_inv, s_w_inv):
+    """y = bf16( fp32( fp32(sum_k dec(x_q[m,k]) dec(Wq[n,k])) * fp32(s_x^-1 s_w^-1) ) )."""
+    comb = np.float32(np.float32(s_x_inv) * np.float32(s_w_inv))
+    acc = f32(e4m3_to_f64(x_q) @ e4m3_to_f64(Wq).T)
+    return bf16_bits_from_f32((acc * comb).astype(np.float32))
+
+
+def linear_bwd(x, W, dY):
+    """BF16 backward of y = x . W^T: dX = bf16(dY . W), dW = fp32(dY^T . x)."""
+    G = bf16_to_f64(dY)
+    return (bf16_bits_from_f32(f32(G @ bf16_to_f64(W))), f32(G.T @ bf16_to_f64(x)))

@@ -721,3 +721,69 @@ def test_fp8_up_forward_normal_inputs(M, d, h):
     # against the exact BF16 network: the FP8 up- and down-projection error
     exact = ref.bf16_to_f64(ref.down_proj_bf16(ref.relu2_post(ref.up_proj(P["x"], P["W1"])), P["W2"]))
     assert rel_fro(ref.bf16_to_f64(host_bits(b.out)), exact) < 8e-2
+
+
+# ---------------------------------------------------------------------------
+# generic FP8 linear layer (attention projections)
+# ---------------------------------------------------------------------------
+
+LINEAR_SHAPES = [(300, 768, 2304), (1000, 768, 768), (129, 512, 768), (16384, 768, 2304)]
+
+
+@pytest.mark.parametrize("M,K,N", LINEAR_SHAPES[:3])
+def test_linear_fwd_fp8_bit_exact_grid(M, K, N):
+    P = synth.make_problem(M, K, N, seed=M + N, x_dist="grid", w_dist="grid")   # W1 is [N,K]
+    st_x = _state(2.0, 16.0)
+    xq_o, _ = ref.quantise_x(P["x"], 16.0)
+    Wq_o = ref.e4m3_bits_from_f32((ref.bf16_to_f64(P["W1"]) * 1024.0).astype(np.float32))
+    xq = torch.empty(M, K, dtype=torch.uint8, device="cuda")
+    pax = torch.empty(A.fp8mlp_x_partial_amax_count(M, K), device="cuda")
+    A.fp8mlp_quantize_x(M, K, dev_bf16(P["x"]), st_x, xq, pax)
+    y = Guarded((M, N), torch.bfloat16)
+    A.fp8mlp_linear_fwd_fp8(M, K, N, xq, dev_u8(Wq_o), dev_f32(np.array([1 / 1024.0, 0, 0, 0], np.float32)), st_x, y.t)
+    torch.cuda.synchronize()
+    want = ref.linear_fp8(xq_o, Wq_o, np.float32(1 / 16.0), np.float32(1 / 1024.0))
+    assert np.array_equal(host_bits(y.t), want)
+    assert y.intact()
+
+
+@pytest.mark.parametrize("M,K,N", LINEAR_SHAPES)
+def test_linear_fp8_fwd_bwd_normal(M, K, N):
+    P = synth.make_problem(M, K, N, seed=7 * M + N)
+    s_x = np.float32(448.0 / 9.0)
+    st_x = _state(2.0, float(s_x))
+    xq = torch.empty(M, K, dtype=torch.uint8, device="cuda")
+    pax = torch.empty(A.fp8mlp_x_partial_amax_count(M, K), device="cuda")
+    A.fp8mlp_quantize_x(M, K, dev_bf16(P["x"]), st_x, xq, pax)
+    Wq = torch.empty(N, K, dtype=torch.uint8, device="cuda")
+    inv = torch.empty(4, device="cuda")
+    ws = torch.empty(A.fp8mlp_workspace_size(0, K, N), dtype=torch.uint8, device="cuda")
+    A.fp8mlp_weight_fp8_cache_refresh(N, K, dev_bf16(P["W1"]), Wq, inv, ws)
+    y = Guarded((M, N), torch.bfloat16)
+    A.fp8mlp_linear_fwd_fp8(M, K, N, xq, Wq, inv, st_x, y.t)
+    g = np.random.default_rng(M)
+    dY = synth.to_bf16_bits(g.standard_normal((M, N)).astype(np.float32))
+    dX = Guarded((M, K), torch.bfloat16)
+    dW = Guarded((N, K), torch.float32)
+    A.fp8mlp_linear_bwd(M, K, N, dev_bf16(P["x"]), dev_bf16(P["W1"]), dev_bf16(dY), dX.t, dW.t)
+    torch.cuda.synchronize()
+    rows = np.arange(M) if M <= 1000 else np.unique(np.r_[0, M - 1, np.random.default_rng(1).integers(0, M, 64)])
+    xq_o, _ = ref.quantise_x(P["x"][rows], s_x)
+    Wq_o, _, swi = ref.w1_cache(P["W1"])
+    assert np.array_equal(host_bits(Wq), Wq_o)
+    y_o = ref.linear_fp8(xq_o, Wq_o, np.float32(np.float32(1) / s_x), swi)
+    assert rel_fro(ref.bf16_to_f64(host_bits(y.t)[rows]), ref.bf16_to_f64(y_o)) < 4e-3
+    exact = ref.bf16_to_f64(P["x"][rows]) @ ref.bf16_to_f64(P["W1"]).T
+    assert rel_fro(ref.bf16_to_f64(host_bits(y.t)[rows]), exact) < 6e-2
+    dX_o = ref.bf16_bits_from_f32(ref.f32(ref.bf16_to_f64(dY[rows]) @ ref.bf16_to_f64(P["W1"])))
+    assert rel_fro(ref.bf16_to_f64(host_bits(dX.t)[rows]), ref.bf16_to_f64(dX_o)) < TOL_GRAD
+    if M <= 1000:
+        _, dW_o = ref.linear_bwd(P["x"], P["W1"], dY)
+        assert rel_fro(host_bits(dW.t), dW_o) < TOL_GRAD
+    else:
+        G, X = ref.bf16_to_f64(dY), ref.bf16_to_f64(P["x"])
+        pairs = [(0, 0), (N - 1, K - 1), (N // 2, 17), (5, K // 3)]
+        got = np.array([host_bits(dW.t)[i, j] for i, j in pairs])
+        want = np.array([G[:, i] @ X[:, j] for i, j in pairs])
+        assert rel_fro(got, want) < TOL_GRAD
+    assert y.intact() and dX.intact() and dW.intact()

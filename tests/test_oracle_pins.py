@@ -533,3 +533,26 @@ def test_up_proj_fp8_bruteforce_and_exact_grid():
     xq2, _ = ref.quantise_x(x, 16.0)
     W1q = ref.e4m3_bits_from_f32((ref.bf16_to_f64(W1) * 1024.0).astype(np.float32))
     assert np.array_equal(ref.up_proj_fp8(xq2, W1q, 1 / 16.0, 1 / 1024.0), ref.up_proj(x, W1))
+
+
+def test_linear_fp8_and_bwd_bruteforce():
+    g = np.random.default_rng(31)
+    xq = g.integers(0, 256, (5, 8)).astype(np.uint8)
+    Wq = g.integers(0, 256, (6, 8)).astype(np.uint8)
+    xq[(xq & 0x7F) == 0x7F] = 0x30
+    Wq[(Wq & 0x7F) == 0x7F] = 0x31
+    y = ref.bf16_to_f64(ref.linear_fp8(xq, Wq, np.float32(1 / 3), np.float32(1 / 5)))
+    want = _brute(ref.e4m3_to_f64(xq), ref.e4m3_to_f64(Wq)) * float(np.float32(np.float32(1 / 3) * np.float32(1 / 5)))
+    np.testing.assert_allclose(y, want, rtol=2 ** -8)
+    x = _bf16(g.standard_normal((7, 8)))
+    W = _bf16(g.standard_normal((6, 8)))
+    dY = _bf16(g.standard_normal((7, 6)))
+    dX, dW = ref.linear_bwd(x, W, dY)
+    X, Wm, G = ref.bf16_to_f64(x), ref.bf16_to_f64(W), ref.bf16_to_f64(dY)
+    np.testing.assert_allclose(ref.bf16_to_f64(dX), _brute(G, Wm.T), rtol=2 ** -8)
+    np.testing.assert_allclose(dW, _brute(G.T, X.T), rtol=1e-6)
+    # torch autograd of the unquantised layer
+    Xt = torch.tensor(X, requires_grad=True)
+    Wt = torch.tensor(Wm, requires_grad=True)
+    (Xt @ Wt.T).backward(torch.tensor(G))
+    assert _rel(ref.bf16_to_f64(dX), Xt.grad.numpy()) < 1e-2 and _rel(dW, Wt.grad.numpy()) < 1e-6
