@@ -71,6 +71,11 @@ WORKLOADS = {
         "qkv16k", M=16384, d=768, h=2304,
         description="FP8 linear layer y = x W^T as the attention QKV projection: M=16384 tokens, "
                     "K=768, N=2304 (3x768), e4m3 forward, BF16 backward"),
+    "ce16k": Workload(
+        "ce16k", M=16384, d=768, h=50304,
+        description="softcapped cross-entropy over a GPT-2 LM head: M=16384 tokens, d=768, "
+                    "V=50304 (GPT-2 vocabulary padded to a multiple of 128), logits std 4, "
+                    "cap 15, one uniform target per token, fwd + bwd (dlogits, dX, dW)"),
     "heavytail": Workload(
         "heavytail", M=65536, d=1024, h=4096, steps=30, x_dist="student_t3",
         spike_steps=(9, 19, 29), spike_factor=2.0,
@@ -114,6 +119,25 @@ def make_problem(M, d, h, seed=0, x_dist="normal", w_dist="normal"):
     dOut = make_x(g, M, d, "grid" if x_dist == "grid" else "normal")
     return dict(x=to_bf16_bits(x), W1=to_bf16_bits(W1), W2=to_bf16_bits(W2),
                 dOut=to_bf16_bits(dOut))
+
+
+def make_head_problem(M, d, V, T=1, seed=0, x_dist="normal", logit_std=4.0, ignore_frac=0.0):
+    """One LM-head problem: x [M,d] and W [V,d] as BF16 bits, targets [M,T]
+    int32 uniform in [0, V), a fraction ``ignore_frac`` of them set to -1.
+
+    W ~ N(0, logit_std^2 / d) gives logits of standard deviation about
+    logit_std for x ~ N(0, 1); ``grid`` draws x = k/4, W = k/256."""
+    g = rng(seed)
+    if x_dist == "grid":
+        x = _grid(g, (M, d), 8, 4)
+        W = _grid(g, (V, d), 16, 256)
+    else:
+        x = make_x(g, M, d, x_dist)
+        W = _normal(g, (V, d), logit_std ** 2 / d)
+    tg = g.integers(0, V, size=(M, T)).astype(np.int32)
+    if ignore_frac > 0:
+        tg[g.random((M, T)) < ignore_frac] = -1
+    return dict(x=to_bf16_bits(x), W=to_bf16_bits(W), targets=tg)
 
 
 def perturb(W_bits, seed, step, var, which):

@@ -482,3 +482,99 @@ def linear_bwd(x, W, dY):
     """BF16 backward of y = x . W^T: dX = bf16(dY . W), dW = fp32(dY^T . x)."""
     G = bf16_to_f64(dY)
     return (bf16_bits_from_f32(f32(G @ bf16_to_f64(W))), f32(G.T @ bf16_to_f64(x)))
+
+
+# ----------------------------------------------------------------------------
+# Softcapped cross-entropy over a language-model head.
+#   [RUO] item 5: a fused softcapped cross-entropy that never materialises
+#         the [M,V] logits in fp32.
+#   [SLOW] "A Retrospective on Our World Records", SlowRun section: one LM
+#         head scored against several successive targets at each position,
+#         through an FP8 soft-capped cross-entropy kernel.
+#   [R83-1] "NanoGPT Speedrun (Track 1)", Changes vs Record #83, item 1: the
+#         earlier record ran FP8 only in the LM head.
+# Readings where the pages are silent (each also listed in DESIGN.md):
+#   * softcap z = c * tanh(y / c), c > 0 (a cap of the form 2c * sigmoid(y/c')
+#     differs from it by a per-row constant, which cross-entropy ignores);
+#   * T targets per position, weights w_t; a target outside [0, V) is ignored;
+#     loss_m = sum over valid t of w_t * (logsumexp_v z[m,v] - z[m, tgt[m,t]]);
+#   * reductions: the sum over rows, and the mean = sum / (sum of the valid
+#     weights), 0 when no target is valid;
+#   * FP8 head: y = fp32( fp32(sum_k dec(x_q) dec(Wq)) * fp32(s_x^-1 s_w^-1) ),
+#     BF16 backward (straight-through over the quantisation, like the MLP);
+#   * dlogits = dL/dy rounded to BF16; dX = bf16(dlogits . W),
+#     dW = fp32(dlogits^T . x).
+# ----------------------------------------------------------------------------
+
+
+def head_logits(x, W):
+    """y = x . W^T in fp64 from BF16 x [M,d] and W [V,d]."""
+    return bf16_to_f64(x) @ bf16_to_f64(W).T
+
+
+def head_logits_fp8(x_q, Wq, s_x_inv, s_w_inv):
+    """y = fp32( fp32(sum_k dec(x_q[m,k]) dec(Wq[v,k])) * fp32(s_x^-1 s_w^-1) ), as fp64."""
+    comb = np.float32(np.float32(s_x_inv) * np.float32(s_w_inv))
+    acc = f32(e4m3_to_f64(x_q) @ e4m3_to_f64(Wq).T)
+    return (acc * comb).astype(np.float32).astype(np.float64)
+
+
+def softcap(y, c):
+    """z = c tanh(y / c)."""
+    return c * np.tanh(np.asarray(y, dtype=np.float64) / c)
+
+
+def _ce_targets(targets, weights, V):
+    """(clipped target indices [M,T], effective weights [M,T]: w_t where the
+    target is in [0, V), else 0)."""
+    tg = np.asarray(targets, dtype=np.int64)
+    w = np.broadcast_to(np.asarray(weights, dtype=np.float64), tg.shape)
+    valid = (tg >= 0) & (tg < V)
+    return np.where(valid, tg, 0), np.where(valid, w, 0.0)
+
+
+def ce_forward(y, targets, weights, c):
+    """Loss of the softcapped logits y [M,V] (fp64) against targets [M,T].
+
+    Returns dict(lse [M], row_loss [M], loss_sum, weight_sum, mean)."""
+    y = np.asarray(y, dtype=np.float64)
+    M, V = y.shape
+    z = softcap(y, c)
+    zmax = z.max(axis=1) if V else np.zeros(M)
+    lse = zmax + np.log(np.exp(z - zmax[:, None]).sum(axis=1))
+    tg, w = _ce_targets(targets, weights, V)
+    zt = np.take_along_axis(z, tg, axis=1)
+    row = (w * (lse[:, None] - zt)).sum(axis=1)
+    ws = float(w.sum())
+    s = float(row.sum())
+    return dict(lse=lse, row_loss=row, loss_sum=s, weight_sum=ws, mean=s / ws if ws > 0 else 0.0)
+
+
+def ce_grad_scale(dloss, weight_sum, mean):
+    """g: the factor that multiplies every row's gradient -- dloss for the
+    summed loss, dloss / weight_sum for the mean (0 when no weight)."""
+    if not mean:
+        return float(dloss)
+    return float(dloss) / weight_sum if weight_sum > 0 else 0.0
+
+
+def ce_backward_dlogits(y, targets, weights, c, lse, g):
+    """dL/dy [M,V] in fp64 for the loss sum_m loss_m scaled by g:
+    g * (W_m softmax(z_m) - sum_t w_t onehot(tgt_t)) * (1 - tanh(y/c)^2),
+    W_m = sum of row m's valid weights."""
+    y = np.asarray(y, dtype=np.float64)
+    M, V = y.shape
+    th = np.tanh(y / c)
+    p = np.exp(c * th - np.asarray(lse, dtype=np.float64)[:, None])
+    tg, w = _ce_targets(targets, weights, V)
+    dz = w.sum(axis=1)[:, None] * p
+    for t in range(tg.shape[1]):
+        np.subtract.at(dz, (np.arange(M), tg[:, t]), w[:, t])
+    return g * dz * (1.0 - th * th)
+
+
+def ce_backward(x, W, dlogits_f64):
+    """BF16 backward through the head: dlogits = bf16(dL/dy), dX, dW."""
+    dl = bf16_bits_from_f32(f32(dlogits_f64))
+    dX, dW = linear_bwd(x, W, dl)
+    return dl, dX, dW

@@ -64,7 +64,43 @@ MUTATIONS = {
                          ["test_rmsnorm_constant_rows_and_autograd"]),
     "amax_drops_last_block": ("partial_amax", lambda orig: (lambda post, rows, cols: orig(post, rows, cols)[:-1]),
                               ["test_amax_partials_equal_brute_max"]),
+    "ce_softcap_derivative_dropped": ("ce_backward_dlogits",
+                                      lambda orig: (lambda y, tg, w, c, lse, g: orig(y, tg, w, c, lse, g) / (1.0 - np.tanh(np.asarray(y) / c) ** 2)),
+                                      ["test_ce_bruteforce_with_ignored_targets", "test_ce_softcapped_vs_torch_autograd"]),
+    "ce_onehot_dropped": ("ce_backward_dlogits", lambda orig: _ce_grad_no_onehot,
+                          ["test_ce_zero_logits_closed_form", "test_ce_softcapped_vs_torch_autograd"]),
+    "ce_target_reads_raw_logit": ("ce_forward", lambda orig: _ce_fwd_raw_target,
+                                  ["test_ce_bruteforce_with_ignored_targets", "test_ce_softcapped_vs_torch_autograd"]),
+    "ce_weights_ignored": ("ce_forward", lambda orig: (lambda y, tg, w, c: orig(y, tg, np.ones(np.shape(tg)[1]), c)),
+                           ["test_ce_bruteforce_with_ignored_targets", "test_ce_multi_target_is_sum_of_single_targets"]),
+    "ce_out_of_range_target_clipped": ("_ce_targets", lambda orig: _ce_targets_clipped,
+                                       ["test_ce_bruteforce_with_ignored_targets", "test_ce_zero_logits_closed_form"]),
+    "ce_fp8_scale_dropped": ("head_logits_fp8", lambda orig: (lambda xq, Wq, a, b: orig(xq, Wq, 1.0, 1.0)),
+                             ["test_ce_head_logits_fp8_bruteforce_and_exact_grid"]),
 }
+
+
+def _ce_grad_no_onehot(y, tg, w, c, lse, g):
+    th = np.tanh(np.asarray(y) / c)
+    _, we = ref._ce_targets(tg, w, np.shape(y)[1])
+    return g * we.sum(axis=1)[:, None] * np.exp(c * th - np.asarray(lse)[:, None]) * (1.0 - th * th)
+
+
+def _ce_fwd_raw_target(y, tg, w, c):
+    y = np.asarray(y, np.float64)
+    z = ref.softcap(y, c)
+    zmax = z.max(axis=1)
+    lse = zmax + np.log(np.exp(z - zmax[:, None]).sum(axis=1))
+    t, we = ref._ce_targets(tg, w, y.shape[1])
+    row = (we * (lse[:, None] - np.take_along_axis(y, t, axis=1))).sum(axis=1)
+    ws = float(we.sum())
+    return dict(lse=lse, row_loss=row, loss_sum=float(row.sum()), weight_sum=ws, mean=float(row.sum()) / ws)
+
+
+def _ce_targets_clipped(targets, weights, V):
+    tg = np.clip(np.asarray(targets, np.int64), 0, V - 1)
+    return tg, np.broadcast_to(np.asarray(weights, np.float64), tg.shape).copy()
+
 
 PARAMS = {"test_e4m3_exhaustive_over_bf16": dict(s=3.7),
           "test_scale_update_closed_form": dict(A=3.0, margin=2.0),

@@ -556,3 +556,151 @@ def test_linear_fp8_and_bwd_bruteforce():
     Wt = torch.tensor(Wm, requires_grad=True)
     (Xt @ Wt.T).backward(torch.tensor(G))
     assert _rel(ref.bf16_to_f64(dX), Xt.grad.numpy()) < 1e-2 and _rel(dW, Wt.grad.numpy()) < 1e-6
+
+
+# ---------------------------------------------------------------------------
+# Softcapped cross-entropy over the LM head
+# ---------------------------------------------------------------------------
+
+def _ce_brute(y, targets, weights, c):
+    """Pure-Python loops over the math module: per-row loss and dL/dy of the
+    summed loss."""
+    import math
+    loss, grad = [], []
+    for m in range(len(y)):
+        V = len(y[m])
+        z = [c * math.tanh(y[m][v] / c) for v in range(V)]
+        mx = max(z)
+        s = 0.0
+        for v in range(V):
+            s += math.exp(z[v] - mx)
+        lse = mx + math.log(s)
+        row, wsum = 0.0, 0.0
+        for t, tg in enumerate(targets[m]):
+            if 0 <= tg < V:
+                row += weights[t] * (lse - z[tg])
+                wsum += weights[t]
+        gr = []
+        for v in range(V):
+            dz = wsum * math.exp(z[v] - lse)
+            for t, tg in enumerate(targets[m]):
+                if tg == v:
+                    dz -= weights[t]
+            th = math.tanh(y[m][v] / c)
+            gr.append(dz * (1.0 - th * th))
+        loss.append(row)
+        grad.append(gr)
+    return loss, grad
+
+
+def test_ce_bruteforce_with_ignored_targets():
+    g = np.random.default_rng(41)
+    y = g.standard_normal((3, 6)) * 8.0
+    tg = np.array([[2, 5, -1], [0, 0, 3], [6, 1, 4]])  # -1 and 6 (= V) are ignored
+    w = [1.0, 0.5, 0.25]
+    c = 5.0
+    f = ref.ce_forward(y, tg, w, c)
+    loss, grad = _ce_brute(y.tolist(), tg.tolist(), w, c)
+    np.testing.assert_allclose(f["row_loss"], loss, rtol=1e-12)
+    assert f["weight_sum"] == 1.5 + 1.75 + 0.75
+    np.testing.assert_allclose(f["mean"], sum(loss) / 4.0, rtol=1e-12)
+    np.testing.assert_allclose(ref.ce_backward_dlogits(y, tg, w, c, f["lse"], 1.0), grad, rtol=1e-10, atol=1e-14)
+
+
+def test_ce_uncapped_limit_matches_torch():
+    # c -> infinity: z = y, and the loss is the library's cross-entropy
+    g = np.random.default_rng(43)
+    y = g.standard_normal((16, 50)) * 3.0
+    tg = g.integers(0, 50, (16, 1))
+    f = ref.ce_forward(y, tg, [1.0], 1e9)
+    Y = torch.tensor(y)
+    want = torch.nn.functional.cross_entropy(Y, torch.tensor(tg[:, 0]), reduction="none")
+    np.testing.assert_allclose(f["row_loss"], want.numpy(), rtol=1e-12)
+    np.testing.assert_allclose(f["lse"], torch.logsumexp(Y, 1).numpy(), rtol=1e-12)
+
+
+def test_ce_softcapped_vs_torch_autograd():
+    g = np.random.default_rng(47)
+    M, V, c = 8, 40, 15.0
+    y = g.standard_normal((M, V)) * 10.0
+    tg = g.integers(0, V, (M, 3))
+    tg[1, 2] = -1
+    tg[5, 0] = -1
+    w = [1.0, 0.5, 0.25]
+    Y = torch.tensor(y, requires_grad=True)
+    Z = c * torch.tanh(Y / c)
+    Tg = torch.tensor(tg)
+    loss_sum = sum(w[t] * torch.nn.functional.cross_entropy(Z, Tg[:, t], ignore_index=-1, reduction="sum")
+                   for t in range(3))
+    wsum = sum(w[t] * float((tg[:, t] >= 0).sum()) for t in range(3))
+    (loss_sum / wsum).backward()
+    f = ref.ce_forward(y, tg, w, c)
+    np.testing.assert_allclose(f["loss_sum"], float(loss_sum.detach()), rtol=1e-12)
+    np.testing.assert_allclose(f["mean"], float(loss_sum.detach()) / wsum, rtol=1e-12)
+    gs = ref.ce_grad_scale(1.0, f["weight_sum"], mean=True)
+    np.testing.assert_allclose(ref.ce_backward_dlogits(y, tg, w, c, f["lse"], gs), Y.grad.numpy(),
+                               rtol=1e-9, atol=1e-15)
+
+
+def test_ce_zero_logits_closed_form():
+    # z = 0 everywhere: every valid target costs ln V; softmax is uniform and
+    # tanh'(0) = 1, so dL/dy = 1/V - onehot
+    M, V = 4, 37
+    tg = np.array([[0], [36], [5], [-3]])
+    f = ref.ce_forward(np.zeros((M, V)), tg, [1.0], 15.0)
+    np.testing.assert_allclose(f["row_loss"], [np.log(V)] * 3 + [0.0], rtol=1e-15)
+    dy = ref.ce_backward_dlogits(np.zeros((M, V)), tg, [1.0], 15.0, f["lse"], 1.0)
+    want = np.full((M, V), 1.0 / V)
+    want[3] = 0.0
+    for m in range(3):
+        want[m, tg[m, 0]] -= 1.0
+    np.testing.assert_allclose(dy, want, rtol=1e-13, atol=1e-16)
+
+
+def test_ce_multi_target_is_sum_of_single_targets():
+    g = np.random.default_rng(53)
+    y = g.standard_normal((6, 20)) * 20.0
+    tg = g.integers(-2, 22, (6, 3))
+    w = [1.0, 0.75, 0.5]
+    f = ref.ce_forward(y, tg, w, 15.0)
+    singles = [ref.ce_forward(y, tg[:, t:t + 1], [w[t]], 15.0) for t in range(3)]
+    np.testing.assert_allclose(f["row_loss"], sum(s["row_loss"] for s in singles), rtol=1e-12)
+    assert f["weight_sum"] == sum(s["weight_sum"] for s in singles)
+    dy = ref.ce_backward_dlogits(y, tg, w, 15.0, f["lse"], 1.0)
+    dys = sum(ref.ce_backward_dlogits(y, tg[:, t:t + 1], [w[t]], 15.0, f["lse"], 1.0) for t in range(3))
+    np.testing.assert_allclose(dy, dys, rtol=1e-12, atol=1e-15)
+
+
+def test_ce_head_logits_fp8_bruteforce_and_exact_grid():
+    g = np.random.default_rng(59)
+    xq = g.integers(0, 256, (5, 16)).astype(np.uint8)
+    Wq = g.integers(0, 256, (9, 16)).astype(np.uint8)
+    xq[(xq & 0x7F) == 0x7F] = 0x25
+    Wq[(Wq & 0x7F) == 0x7F] = 0x26
+    sxi, swi = np.float32(1 / 7), np.float32(1 / 3)
+    want = _brute(ref.e4m3_to_f64(xq), ref.e4m3_to_f64(Wq)) * float(np.float32(sxi * swi))
+    np.testing.assert_allclose(ref.head_logits_fp8(xq, Wq, sxi, swi), want, rtol=2e-7)
+    x = _bf16(g.integers(-8, 9, (6, 32)) / 4.0)
+    W = _bf16(g.integers(-16, 17, (11, 32)) / 256.0)
+    np.testing.assert_array_equal(ref.head_logits(x, W), _brute(ref.bf16_to_f64(x), ref.bf16_to_f64(W)))
+    xq2, _ = ref.quantise_x(x, 16.0)
+    Wq2 = ref.e4m3_bits_from_f32((ref.bf16_to_f64(W) * 1024.0).astype(np.float32))
+    assert np.array_equal(ref.head_logits_fp8(xq2, Wq2, 1 / 16.0, 1 / 1024.0), ref.head_logits(x, W))
+
+
+def test_ce_backward_through_head_vs_torch_autograd():
+    g = np.random.default_rng(61)
+    M, d, V, c = 12, 16, 48, 15.0
+    x = _bf16(g.standard_normal((M, d)))
+    W = _bf16(g.standard_normal((V, d)) * 2.0)
+    tg = g.integers(0, V, (M, 1))
+    y = ref.head_logits(x, W)
+    f = ref.ce_forward(y, tg, [1.0], c)
+    dl, dX, dW = ref.ce_backward(x, W, ref.ce_backward_dlogits(y, tg, [1.0], c, f["lse"], 1.0))
+    Xt = torch.tensor(ref.bf16_to_f64(x), requires_grad=True)
+    Wt = torch.tensor(ref.bf16_to_f64(W), requires_grad=True)
+    torch.nn.functional.cross_entropy(c * torch.tanh((Xt @ Wt.T) / c), torch.tensor(tg[:, 0]),
+                                      reduction="sum").backward()
+    # dlogits is rounded to BF16 (relative error <= 2^-9 per element)
+    assert _rel(ref.bf16_to_f64(dX), Xt.grad.numpy()) < 1e-2
+    assert _rel(dW, Wt.grad.numpy()) < 1e-2
