@@ -33,6 +33,8 @@ STATUS_W2_DEGENERATE = 4
 STATE_KEPT_SCALE = 1
 FWD_EVAL_BF16 = 1
 FWD_CALIBRATE = 2
+CE_SUM = 0
+CE_MEAN = 1
 DEBUG_STALL_PRODUCER = 1
 E4M3_MAX = 448.0
 
@@ -65,6 +67,10 @@ _SIGS = {
     "fp8mlp_linear_fwd_fp8": [_i, _i, _i, _p, _p, _p, _p, _p, _p],
     "fp8mlp_weight_fp8_cache_refresh": [_i, _i, _p, _p, _p, _p, _p],
     "fp8mlp_linear_bwd": [_i, _i, _i, _p, _p, _p, _p, _p, _p],
+    "fp8mlp_ce_fwd": [_i, _i, _i, _i, _p, _p, _p, _p, _f, _p, _p, _p, _p, _p],
+    "fp8mlp_ce_fwd_fp8": [_i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _f, _p, _p, _p, _p, _p],
+    "fp8mlp_ce_bwd_dlogits": [_i, _i, _i, _i, _p, _p, _p, _p, _f, _p, _p, _p, _i, _p, _p],
+    "fp8mlp_ce_bwd_dlogits_fp8": [_i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _f, _p, _p, _p, _i, _p, _p],
     "fp8mlp_bwd_dx": [_i, _i, _i, _p, _p, _p, _p],
     "fp8mlp_bwd_dw": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p],
     "fp8mlp_mlp_bwd": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p],
@@ -83,6 +89,8 @@ for _n, _a in _SIGS.items():
     _fn.restype = ctypes.c_int
 lib.fp8mlp_workspace_size.argtypes = [_i, _i, _i]
 lib.fp8mlp_workspace_size.restype = _sz
+lib.fp8mlp_ce_workspace_size.argtypes = [_i, _i, _i]
+lib.fp8mlp_ce_workspace_size.restype = _sz
 lib.fp8mlp_kernel_launch_count.argtypes = []
 lib.fp8mlp_kernel_launch_count.restype = ctypes.c_ulonglong
 for _n in ("fp8mlp_error_string",):
@@ -223,6 +231,49 @@ def fp8mlp_weight_fp8_cache_refresh(N, K, W, Wq, w_scale_inv, workspace, stream=
 
 def fp8mlp_linear_bwd(M, K, N, x, W, dY, dX, dW, stream=None):
     return _call("fp8mlp_linear_bwd", M, K, N, _ptr(x), _ptr(W), _ptr(dY), _ptr(dX), _ptr(dW), _stream(stream))
+
+
+def _host_floats(seq):
+    """A host float array for a C `const float*` (None stays NULL); the
+    returned object must stay alive for the call."""
+    if seq is None:
+        return None
+    vals = [float(v) for v in seq]
+    return (ctypes.c_float * len(vals))(*vals)
+
+
+def fp8mlp_ce_workspace_size(M, V, T):
+    return int(lib.fp8mlp_ce_workspace_size(M, V, T))
+
+
+def fp8mlp_ce_fwd(M, d, V, T, x, W, targets, target_weights, softcap, lse, row_loss, loss, workspace, stream=None):
+    w = _host_floats(target_weights)
+    return _call("fp8mlp_ce_fwd", M, d, V, T, _ptr(x), _ptr(W), _ptr(targets), ctypes.cast(w, _p) if w else None,
+                 softcap, _ptr(lse), _ptr(row_loss), _ptr(loss), _ptr(workspace), _stream(stream))
+
+
+def fp8mlp_ce_fwd_fp8(M, d, V, T, x_fp8, st_x, Wq, w_scale_inv, targets, target_weights, softcap, lse, row_loss,
+                      loss, workspace, stream=None):
+    w = _host_floats(target_weights)
+    return _call("fp8mlp_ce_fwd_fp8", M, d, V, T, _ptr(x_fp8), _ptr(st_x), _ptr(Wq), _ptr(w_scale_inv),
+                 _ptr(targets), ctypes.cast(w, _p) if w else None, softcap, _ptr(lse), _ptr(row_loss), _ptr(loss),
+                 _ptr(workspace), _stream(stream))
+
+
+def fp8mlp_ce_bwd_dlogits(M, d, V, T, x, W, targets, target_weights, softcap, lse, loss, dloss, reduction, dlogits,
+                          stream=None):
+    w = _host_floats(target_weights)
+    return _call("fp8mlp_ce_bwd_dlogits", M, d, V, T, _ptr(x), _ptr(W), _ptr(targets),
+                 ctypes.cast(w, _p) if w else None, softcap, _ptr(lse), _ptr(loss), _ptr(dloss), reduction,
+                 _ptr(dlogits), _stream(stream))
+
+
+def fp8mlp_ce_bwd_dlogits_fp8(M, d, V, T, x_fp8, st_x, Wq, w_scale_inv, targets, target_weights, softcap, lse, loss,
+                              dloss, reduction, dlogits, stream=None):
+    w = _host_floats(target_weights)
+    return _call("fp8mlp_ce_bwd_dlogits_fp8", M, d, V, T, _ptr(x_fp8), _ptr(st_x), _ptr(Wq), _ptr(w_scale_inv),
+                 _ptr(targets), ctypes.cast(w, _p) if w else None, softcap, _ptr(lse), _ptr(loss), _ptr(dloss),
+                 reduction, _ptr(dlogits), _stream(stream))
 
 
 def fp8mlp_bwd_dpre(M, d, h, dOut, W2, post, dPre, stream=None):

@@ -180,6 +180,134 @@ int current_device(DeviceInfo** info) {
 
 using namespace fp8mlp;
 
+namespace {
+
+// ---- softcapped cross-entropy: workspace layout and shared checks ----------
+struct CeLayout {
+  int nblk = 0;    // row blocks of the row pass
+  int nparts = 0;  // partial sums per row (128-column groups, whole tiles)
+  size_t off_partial = 0, off_ztgt = 0, total = 0;
+};
+
+CeLayout ce_layout(int M, int V, int T) {
+  auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  CeLayout L;
+  L.nblk = cdiv(M, kCeRowsPerBlock);
+  L.nparts = cdiv(V, kGemmBN) * (kGemmBN / ce_partial_cols());
+  // [block sums: 2 doubles per row block][partials: nparts x M][z - c at targets: M x T]
+  L.off_partial = al(sizeof(double) * 2 * static_cast<size_t>(L.nblk));
+  L.off_ztgt = L.off_partial + al(sizeof(float) * static_cast<size_t>(L.nparts) * M);
+  L.total = L.off_ztgt + al(sizeof(float) * static_cast<size_t>(M) * T);
+  return L;
+}
+
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+#define REQUIRE_PTR4(p)                                                                   \
+  do {                                                                                    \
+    if ((p) == nullptr) return fail(FP8MLP_ERR_INVALID_ARG, #p " is NULL");               \
+    if (!aligned4(p)) return fail(FP8MLP_ERR_INVALID_ARG, #p " is not 4-byte aligned");  \
+  } while (0)
+
+// shape, cap and weight checks; fills p's cross-entropy fields
+int ce_setup(int M, int d, int V, int T, const int32_t* targets, const float* target_weights, float softcap,
+             GemmParams* p) {
+  TRY(check_dims(M, d, V));
+  if (T < 1 || T > 4) return fail(FP8MLP_ERR_INVALID_ARG, "T (targets per row) must be 1..4");
+  if (!(softcap > 0.f && softcap <= 40.f)) return fail(FP8MLP_ERR_INVALID_ARG, "softcap must be in (0, 40]");
+  for (int t = 0; t < 4; ++t) {
+    const float w = t >= T ? 0.f : (target_weights != nullptr ? target_weights[t] : 1.f);
+    if (!std::isfinite(w)) return fail(FP8MLP_ERR_INVALID_ARG, "target weights must be finite");
+    p->ce_w[t] = w;
+  }
+  if (M > 0) REQUIRE_PTR4(targets);
+  p->ce_T = T;
+  p->ce_targets = targets;
+  p->ce_cap = softcap;
+  const double log2e = 1.4426950408889634;
+  p->ce_k = static_cast<float>(-2.0 * log2e / softcap);
+  p->ce_cl2 = static_cast<float>(softcap * log2e);
+  return FP8MLP_OK;
+}
+
+int ce_fwd_impl(bool fp8, int M, int d, int V, int T, const void* x, const void* W, const fp8mlp_scale_state* st_x,
+                const float* w_scale_inv, const int32_t* targets, const float* target_weights, float softcap,
+                float* lse, float* row_loss, float* loss, void* workspace, cudaStream_t stream) {
+  GemmParams p{};
+  TRY(ce_setup(M, d, V, T, targets, target_weights, softcap, &p));
+  REQUIRE_PTR4(loss);
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  if (M == 0) {
+    const cudaError_t e = cudaMemsetAsync(loss, 0, 3 * sizeof(float), stream);
+    return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "ce_fwd memset");
+  }
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(W);
+  REQUIRE_PTR(workspace);
+  REQUIRE_PTR4(lse);
+  if (row_loss != nullptr) REQUIRE_PTR4(row_loss);
+  const GemmKind kind = fp8 ? GemmKind::CeFwd8 : GemmKind::CeFwd;
+  const CUtensorMapDataType dt = fp8 ? U8 : BF16;
+  const int es = fp8 ? 1 : 2;
+  if (fp8) {
+    REQUIRE_PTR(st_x);
+    if (w_scale_inv == nullptr) return fail(FP8MLP_ERR_INVALID_ARG, "w_scale_inv is NULL");
+    p.st_in = st_x;
+    p.w_in_scale_inv = w_scale_inv;
+  }
+  TRY(map_kmajor(&p.tmA[0], x, dt, es, M, d, kGemmBM, "x"));
+  TRY(map_kmajor(&p.tmB[0], W, dt, es, V, d, kGemmBN * kGemmBM / gemm_tile_m(kind), "W"));
+  fill_common(p, kind, di, M, V, d, 1);
+  const CeLayout L = ce_layout(M, V, T);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.ce_partial = reinterpret_cast<float*>(ws + L.off_partial);
+  p.ce_ztgt = reinterpret_cast<float*>(ws + L.off_ztgt);
+  TRY(launch(kind, p, di, stream, "ce_fwd launch"));
+  const cudaError_t e = launch_ce_finalize(M, L.nparts, T, V, targets, p.ce_w, softcap, p.ce_partial, p.ce_ztgt,
+                                           lse, row_loss, reinterpret_cast<double*>(ws), loss, stream);
+  return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "ce_fwd finalize launch");
+}
+
+int ce_bwd_impl(bool fp8, int M, int d, int V, int T, const void* x, const void* W, const fp8mlp_scale_state* st_x,
+                const float* w_scale_inv, const int32_t* targets, const float* target_weights, float softcap,
+                const float* lse, const float* loss, const float* dloss, int reduction, uint16_t* dlogits,
+                cudaStream_t stream) {
+  GemmParams p{};
+  TRY(ce_setup(M, d, V, T, targets, target_weights, softcap, &p));
+  if (reduction != FP8MLP_CE_SUM && reduction != FP8MLP_CE_MEAN)
+    return fail(FP8MLP_ERR_INVALID_ARG, "reduction must be FP8MLP_CE_SUM or FP8MLP_CE_MEAN");
+  if (M == 0) return FP8MLP_OK;
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(W);
+  REQUIRE_PTR(dlogits);
+  REQUIRE_PTR4(lse);
+  REQUIRE_PTR4(loss);
+  if (dloss != nullptr) REQUIRE_PTR4(dloss);
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  const GemmKind kind = fp8 ? GemmKind::CeBwd8 : GemmKind::CeBwd;
+  const CUtensorMapDataType dt = fp8 ? U8 : BF16;
+  const int es = fp8 ? 1 : 2;
+  if (fp8) {
+    REQUIRE_PTR(st_x);
+    if (w_scale_inv == nullptr) return fail(FP8MLP_ERR_INVALID_ARG, "w_scale_inv is NULL");
+    p.st_in = st_x;
+    p.w_in_scale_inv = w_scale_inv;
+  }
+  TRY(map_kmajor(&p.tmA[0], x, dt, es, M, d, kGemmBM, "x"));
+  TRY(map_kmajor(&p.tmB[0], W, dt, es, V, d, kGemmBN * kGemmBM / gemm_tile_m(kind), "W"));
+  TRY(map_tile32(&p.tmOut[0], dlogits, BF16, 2, M, V, "dlogits"));
+  fill_common(p, kind, di, M, V, d, 1);
+  p.ce_lse = lse;
+  p.ce_loss = loss;
+  p.ce_dloss = dloss;
+  p.ce_mean = reduction == FP8MLP_CE_MEAN ? 1 : 0;
+  return launch(kind, p, di, stream, "ce_bwd_dlogits launch");
+}
+
+}  // namespace
+
 extern "C" {
 
 int fp8mlp_partial_amax_shape(int M, int h, int* row_blocks, int* col_blocks, int* block_rows, int* block_cols) {
@@ -476,6 +604,45 @@ int fp8mlp_linear_bwd(int M, int K, int N, const uint16_t* x, const uint16_t* W,
   TRY(map_tile32(&p.tmOut[0], dW, F32, 4, N, K, "dW"));
   fill_common(p, GemmKind::DW, di, N, K, M, 1);
   return launch(GemmKind::DW, p, di, stream, "linear_bwd dW launch");
+}
+
+size_t fp8mlp_ce_workspace_size(int M, int V, int T) {
+  if (M <= 0 || V <= 0 || T <= 0) return 0;
+  return ce_layout(M, V, T).total;
+}
+
+int fp8mlp_ce_fwd(int M, int d, int V, int T, const uint16_t* x, const uint16_t* W, const int32_t* targets,
+                  const float* target_weights, float softcap, float* lse, float* row_loss, float* loss,
+                  void* workspace, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  return ce_fwd_impl(false, M, d, V, T, x, W, nullptr, nullptr, targets, target_weights, softcap, lse, row_loss, loss,
+                     workspace, stream);
+}
+
+int fp8mlp_ce_fwd_fp8(int M, int d, int V, int T, const uint8_t* x_fp8, const fp8mlp_scale_state* st_x,
+                      const uint8_t* Wq, const float* w_scale_inv, const int32_t* targets,
+                      const float* target_weights, float softcap, float* lse, float* row_loss, float* loss,
+                      void* workspace, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  return ce_fwd_impl(true, M, d, V, T, x_fp8, Wq, st_x, w_scale_inv, targets, target_weights, softcap, lse, row_loss,
+                     loss, workspace, stream);
+}
+
+int fp8mlp_ce_bwd_dlogits(int M, int d, int V, int T, const uint16_t* x, const uint16_t* W, const int32_t* targets,
+                          const float* target_weights, float softcap, const float* lse, const float* loss,
+                          const float* dloss, int reduction, uint16_t* dlogits, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  return ce_bwd_impl(false, M, d, V, T, x, W, nullptr, nullptr, targets, target_weights, softcap, lse, loss, dloss,
+                     reduction, dlogits, stream);
+}
+
+int fp8mlp_ce_bwd_dlogits_fp8(int M, int d, int V, int T, const uint8_t* x_fp8, const fp8mlp_scale_state* st_x,
+                              const uint8_t* Wq, const float* w_scale_inv, const int32_t* targets,
+                              const float* target_weights, float softcap, const float* lse, const float* loss,
+                              const float* dloss, int reduction, uint16_t* dlogits, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  return ce_bwd_impl(true, M, d, V, T, x_fp8, Wq, st_x, w_scale_inv, targets, target_weights, softcap, lse, loss,
+                     dloss, reduction, dlogits, stream);
 }
 
 int fp8mlp_bwd_dpre(int M, int d, int h, const uint16_t* dOut, const uint16_t* W2, const uint16_t* post,

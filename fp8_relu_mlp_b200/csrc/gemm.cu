@@ -1,4 +1,5 @@
-// Instantiations of the tcgen05 GEMM for the five roles of the MLP block.
+// Instantiations of the tcgen05 GEMM for the roles of the MLP block, the FP8
+// linear layer and the softcapped cross-entropy head.
 #include "internal.h"
 
 namespace fp8mlp {
@@ -12,6 +13,12 @@ using CfgUpQ = GemmCfg<2, kGemmBN, 5, true, false, false, Epi::UpFused>;
 using CfgDPre = GemmCfg<2, kGemmBN, 3, false, false, false, Epi::DPre>;
 // dW: one long tile per CTA pair, so a light epilogue (4 warps) and more stages
 using CfgDW = GemmCfg<2, kGemmBN, 6, false, true, true, Epi::StoreF32, 4>;
+// LM head with the softcapped cross-entropy in the epilogue; the forward
+// stores no tile, so its shared memory all goes to the operand ring
+using CfgCeF = GemmCfg<2, kGemmBN, 6, false, false, false, Epi::CeFwd>;
+using CfgCeF8 = GemmCfg<2, kGemmBN, 6, true, false, false, Epi::CeFwd>;
+using CfgCeB = GemmCfg<2, kGemmBN, 6, false, false, false, Epi::CeBwd>;
+using CfgCeB8 = GemmCfg<2, kGemmBN, 6, true, false, false, Epi::CeBwd>;
 
 namespace {
 
@@ -56,6 +63,11 @@ cudaError_t launch_one(const GemmParams& p, int num_tiles, int num_sms, cudaStre
 
 int up_partial_cols() { return CfgUp::BN / CfgUp::EPI_SPLIT; }
 
+int ce_partial_cols() {
+  static_assert(CfgCeF::BN / CfgCeF::EPI_SPLIT == CfgCeF8::BN / CfgCeF8::EPI_SPLIT, "same partial layout");
+  return CfgCeF::BN / CfgCeF::EPI_SPLIT;
+}
+
 int gemm_tile_m(GemmKind kind) {
   switch (kind) {
     case GemmKind::Up:
@@ -70,6 +82,14 @@ int gemm_tile_m(GemmKind kind) {
       return CfgDW::TILE_M;
     case GemmKind::UpQ:
       return CfgUpQ::TILE_M;
+    case GemmKind::CeFwd:
+      return CfgCeF::TILE_M;
+    case GemmKind::CeFwd8:
+      return CfgCeF8::TILE_M;
+    case GemmKind::CeBwd:
+      return CfgCeB::TILE_M;
+    case GemmKind::CeBwd8:
+      return CfgCeB8::TILE_M;
   }
   return 128;
 }
@@ -88,6 +108,14 @@ cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int num_tiles, int n
       return launch_one<CfgDW>(p, num_tiles, num_sms, s);
     case GemmKind::UpQ:
       return launch_one<CfgUpQ>(p, num_tiles, num_sms, s);
+    case GemmKind::CeFwd:
+      return launch_one<CfgCeF>(p, num_tiles, num_sms, s);
+    case GemmKind::CeFwd8:
+      return launch_one<CfgCeF8>(p, num_tiles, num_sms, s);
+    case GemmKind::CeBwd:
+      return launch_one<CfgCeB>(p, num_tiles, num_sms, s);
+    case GemmKind::CeBwd8:
+      return launch_one<CfgCeB8>(p, num_tiles, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }

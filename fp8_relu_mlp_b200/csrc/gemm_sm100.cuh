@@ -30,6 +30,10 @@ enum class Epi : int {
   StoreBf16 = 2,   // out = bf16(acc)
   DPre = 3,        // dPre = bf16(2 sqrt(post) * acc), post read by TMA (hardware sqrt.approx)
   StoreF32 = 4,    // out = acc (fp32)
+  CeFwd = 5,       // softcapped cross-entropy, forward: per row and column group the
+                   // sum of exp(z - c), z = c tanh(y/c), and z at the row's targets;
+                   // nothing [M,V] is written
+  CeBwd = 6,       // softcapped cross-entropy, backward: dlogits = bf16(dL/dy)
 };
 
 struct alignas(64) GemmParams {
@@ -52,6 +56,20 @@ struct alignas(64) GemmParams {
   unsigned int* status;
   unsigned long long timeout_ns;
   int debug_flags;
+  // softcapped cross-entropy (CeFwd / CeBwd); the logits are y = acc (BF16
+  // inputs) or acc * s_x^-1 * s_w^-1 (e4m3 inputs, scales in st_in / w_in_scale_inv)
+  int ce_T;                  // targets per row (1..4)
+  int ce_mean;               // CeBwd: the reduced loss is the mean over the valid weights
+  const int* ce_targets;     // [M, ce_T]; outside [0, N) = ignored
+  float ce_w[4];             // target weights
+  float ce_cap;              // c
+  float ce_k;                // -2 log2(e) / c
+  float ce_cl2;              // c log2(e)
+  float* ce_partial;         // CeFwd: [tiles_n * EPI_SPLIT][M] sums of exp(z - c)
+  float* ce_ztgt;            // CeFwd: [M, ce_T] z - c at each valid target
+  const float* ce_lse;       // CeBwd: [M]
+  const float* ce_loss;      // CeBwd: {sum, weight, mean} of the forward
+  const float* ce_dloss;     // CeBwd: gradient of the reduced loss (NULL = 1)
 };
 
 template <int CG_, int BN_, int STAGES_, bool FP8_, bool A_MN_, bool B_MN_, Epi EPI_, int NEPI_ = 8>
@@ -91,7 +109,8 @@ struct GemmCfg {
   static constexpr int NCH_W = NCHUNK / EPI_SPLIT;  // chunks per epilogue warp per tile
   static constexpr int THREADS = 64 + 32 * NEPI;
   static_assert(NEPI % 4 == 0 && NCHUNK % EPI_SPLIT == 0, "chunks per warp");
-  static constexpr int OUT_BUF = 32 * ECOLS * (EPI == Epi::StoreF32 ? 4 : 2);
+  static constexpr bool STORES = EPI != Epi::CeFwd;  // the epilogue writes a tile with TMA
+  static constexpr int OUT_BUF = !STORES ? 0 : 32 * ECOLS * (EPI == Epi::StoreF32 ? 4 : 2);
   static constexpr int OUT2_BUF = EPI == Epi::UpFused ? 32 * ECOLS : 0;
   static constexpr int SLOT = OUT_BUF + OUT2_BUF;  // one output staging slot (two per epilogue warp)
   static_assert(SLOT % 1024 == 0, "slot alignment");
@@ -125,6 +144,19 @@ __device__ __forceinline__ void store_row_bf16(uint32_t base, int lane, const ui
   for (int j = 0; j < 4; ++j)
     st_shared_v4(base + swz<3>(lane * 64 + j * 16), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
 }
+
+// Softcap z = c tanh(y/c) from e = exp(-2|y|/c) and r = 1/(1+e):
+//   |tanh(y/c)| = (1-e) r,   t - 1 = -2r (y < 0) or -2er (y >= 0),
+//   1 - t^2 = 4 e r^2
+// so neither z - c = c (t-1) nor the derivative loses digits to cancellation.
+// k = -2 log2(e) / c.  Returns t - 1.
+__device__ __forceinline__ float softcap_tm1(float y, float k, float& e, float& r) {
+  e = ex2_approx(k * fabsf(y));
+  r = rcp_approx(1.f + e);
+  return -2.f * r * (y >= 0.f ? e : 1.f);
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
 
 }  // namespace dev
 
@@ -330,7 +362,17 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
     if constexpr (C::EPI == Epi::DownScaled) comb = __fmul_rn(p.st->scale_inv, *p.w2_scale_inv);
     // e4m3 up-projection: dequantise the accumulator before relu and the square
     float dq = 1.f;
-    if constexpr (C::EPI == Epi::UpFused && C::FP8) dq = __fmul_rn(p.st_in->scale_inv, *p.w_in_scale_inv);
+    constexpr bool kCe = C::EPI == Epi::CeFwd || C::EPI == Epi::CeBwd;
+    if constexpr ((C::EPI == Epi::UpFused || kCe) && C::FP8) dq = __fmul_rn(p.st_in->scale_inv, *p.w_in_scale_inv);
+    // cross-entropy backward: g, the factor of every row's gradient
+    float ce_g = 0.f;
+    if constexpr (C::EPI == Epi::CeBwd) {
+      ce_g = p.ce_dloss != nullptr ? *p.ce_dloss : 1.f;
+      if (p.ce_mean) {
+        const float ws = p.ce_loss[1];
+        ce_g = ws > 0.f ? __fdiv_rn(ce_g, ws) : 0.f;
+      }
+    }
     // DPre: rounds of post prefetch started (one round = a tile's NAUX chunks,
     // ring slot c = chunk c) and how many slots the latest round has reached
     uint32_t aux_rounds = 0, aux_last = 0;
@@ -366,6 +408,30 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
       const int row0 = tile_rows(t);
       const int n0 = nb * C::BN;
       const int next_tile = t + npairs;
+      // cross-entropy: this thread's row, its valid targets, and (backward)
+      // (lse - c) log2(e) and g times the row's weight
+      const int ce_m = row0 + lane;
+      int ce_tg[4] = {-1, -1, -1, -1};
+      float ce_sum = 0.f, ce_L = 0.f, ce_gw = 0.f;
+      if constexpr (kCe) {
+        if (ce_m < p.M) {
+          float wsum = 0.f;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            if (t < p.ce_T) {
+              const int tv = p.ce_targets[static_cast<size_t>(ce_m) * p.ce_T + t];
+              if (tv >= 0 && tv < p.N) {
+                ce_tg[t] = tv;
+                wsum += p.ce_w[t];
+              }
+            }
+          }
+          if constexpr (C::EPI == Epi::CeBwd) {
+            ce_L = __fmul_rn(__fsub_rn(p.ce_lse[ce_m], p.ce_cap), kLog2e);
+            ce_gw = __fmul_rn(ce_g, wsum);
+          }
+        }
+      }
       if (!mbar_wait(&tfull[acc], acc_phase, w)) break;
       tc_fence_after();
       float tmax = 0.f;
@@ -382,11 +448,12 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
           else
             mbar_arrive_cluster(tempty_addr0 + acc * 8u);
         }
-        const uint32_t b = ctr & 1u;
-        uint8_t* slot = sEpi + (e * 2 + b) * C::SLOT;
+        uint8_t* slot = sEpi + (e * 2 + (ctr & 1u)) * C::SLOT;
         const uint32_t sbase = smem_u32(slot);
-        if (lane == 0) bulk_wait_read<1>();  // the store issued from this slot two chunks ago has read it
-        __syncwarp();
+        if constexpr (C::STORES) {
+          if (lane == 0) bulk_wait_read<1>();  // the store issued from this slot two chunks ago has read it
+          __syncwarp();
+        }
         const int col0 = n0 + c * C::ECOLS;
 
         if constexpr (C::EPI == Epi::UpFused) {
@@ -468,24 +535,90 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
             }
             store_row_bf16<64>(sbase, lane, pk);
           }
+        } else if constexpr (C::EPI == Epi::CeFwd) {
+          // sum over the chunk's columns inside the vocabulary of exp(z - c) =
+          // 2^(c log2(e) (t - 1)); |z| <= c keeps every term in [e^-2c, 1]
+          const int nvalid = p.N - col0;
+          float csum = 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float y = __uint_as_float(v[i]);
+            if constexpr (C::FP8) y = __fmul_rn(y, dq);
+            float ee, rr;
+            const float term = ex2_approx(p.ce_cl2 * softcap_tm1(y, p.ce_k, ee, rr));
+            csum += i < nvalid ? term : 0.f;
+          }
+          ce_sum += csum;
+          // z - c at the row's targets that fall in this chunk (one thread in
+          // the grid owns each (row, target))
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int off = ce_tg[t] - col0;
+            if (off >= 0 && off < 32) {
+              float yv = 0.f;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) yv = i == off ? __uint_as_float(v[i]) : yv;
+              if constexpr (C::FP8) yv = __fmul_rn(yv, dq);
+              float ee, rr;
+              const float tm1 = softcap_tm1(yv, p.ce_k, ee, rr);
+              p.ce_ztgt[static_cast<size_t>(ce_m) * p.ce_T + t] = __fmul_rn(p.ce_cap, tm1);
+            }
+          }
+        } else if constexpr (C::EPI == Epi::CeBwd) {
+          // dL/dy = g (W_m softmax(z) - sum_t w_t onehot(tgt_t)) (1 - t^2)
+          float dy[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float y = __uint_as_float(v[i]);
+            if constexpr (C::FP8) y = __fmul_rn(y, dq);
+            float ee, rr;
+            const float tm1 = softcap_tm1(y, p.ce_k, ee, rr);
+            const float prob = ex2_approx(fmaf(p.ce_cl2, tm1, -ce_L));  // exp(z - lse)
+            const float der = 4.f * ee * rr * rr;
+            dy[i] = ce_gw * prob * der;
+          }
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int off = ce_tg[t] - col0;
+            if (off >= 0 && off < 32) {
+              float yv = 0.f;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) yv = i == off ? __uint_as_float(v[i]) : yv;
+              if constexpr (C::FP8) yv = __fmul_rn(yv, dq);
+              float ee, rr;
+              softcap_tm1(yv, p.ce_k, ee, rr);
+              const float sub = ce_g * p.ce_w[t] * (4.f * ee * rr * rr);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) dy[i] = i == off ? dy[i] - sub : dy[i];
+            }
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(dy[2 * i], dy[2 * i + 1]);
+          store_row_bf16<64>(sbase, lane, pk);
         } else {  // StoreF32
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             st_shared_v4(sbase + swz<7>(lane * 128 + j * 16), v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
         }
         if (!ok) break;
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&p.tmOut[g], slot, col0, row0);
-          if constexpr (C::EPI == Epi::UpFused) {
-            if (p.write_q) tma_store_2d(&p.tmOut2, slot + C::OUT_BUF, col0, row0);
+        if constexpr (C::STORES) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&p.tmOut[g], slot, col0, row0);
+            if constexpr (C::EPI == Epi::UpFused) {
+              if (p.write_q) tma_store_2d(&p.tmOut2, slot + C::OUT_BUF, col0, row0);
+            }
+            bulk_commit();
           }
-          bulk_commit();
         }
         ++ctr;
       }
       if (!ok) break;
+      if constexpr (C::EPI == Epi::CeFwd) {
+        if (ce_m < p.M) p.ce_partial[static_cast<size_t>(nb * C::EPI_SPLIT + half) * p.M + ce_m] = ce_sum;
+      }
       if constexpr (C::EPI == Epi::UpFused) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));

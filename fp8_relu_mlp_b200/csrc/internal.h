@@ -17,6 +17,10 @@ enum class GemmKind : int {
   DPre = 3,     // K5: dOut . W2^T -> dPre with the 2 sqrt(post) epilogue
   DW = 4,       // K7/K8: dPre^T . x and post^T . dOut (BF16, MN-major A/B), fp32 out
   UpQ = 5,      // K1 on e4m3 x and W1 (dequantised in the epilogue)
+  CeFwd = 6,    // LM head x . W^T -> softcapped cross-entropy partial sums (BF16)
+  CeFwd8 = 7,   // the same on e4m3 x and W
+  CeBwd = 8,    // LM head x . W^T recomputed -> BF16 dlogits (BF16)
+  CeBwd8 = 9,   // the same on e4m3 x and W
 };
 constexpr int kGemmBM = 128;  // accumulator rows per CTA
 constexpr int kGemmBN = 256;  // output tile columns
@@ -85,6 +89,15 @@ cudaError_t launch_quantize_x(long long n, const uint16_t* x, const fp8mlp_scale
                               float* partial, cudaStream_t s);
 cudaError_t launch_w1_cache(int h, int d, const uint16_t* W1, uint8_t* W1q, float* w1_scale_inv,
                             unsigned int* partial, unsigned int* status, cudaStream_t s);
+
+// softcapped cross-entropy: rows -> lse, row loss and per-block sums; then
+// the block sums -> {sum, weight, mean}, both in a fixed order
+constexpr int kCeRowsPerBlock = 32;
+constexpr int kCeSlices = 8;  // threads per row in the row pass
+int ce_partial_cols();        // vocabulary columns covered by one partial sum
+cudaError_t launch_ce_finalize(int M, int nparts, int T, int V, const int* targets, const float* w, float cap,
+                               const float* partial, const float* ztgt, float* lse, float* row_loss,
+                               double* block_sums, float* loss, cudaStream_t s);
 
 // status word symbol address on the current device
 cudaError_t status_word_address(unsigned int** ptr);

@@ -213,6 +213,70 @@ int fp8mlp_weight_fp8_cache_refresh(int N, int K, const uint16_t* W, uint8_t* Wq
 int fp8mlp_linear_bwd(int M, int K, int N, const uint16_t* x, const uint16_t* W, const uint16_t* dY, uint16_t* dX,
                       float* dW, fp8mlp_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Softcapped cross-entropy over a language-model head, without [M,V] logits.
+ * "NanoGPT Speedrun (Track 1)", From Unoptimized / Approach, item 5: a fused
+ * softcapped cross-entropy that never materialises the [M,V] logits in fp32;
+ * "A Retrospective on Our World Records", SlowRun section: one LM head scored
+ * against several successive targets at each position through an FP8
+ * soft-capped cross-entropy kernel; Changes vs Record #83, item 1: FP8 in the
+ * LM head.
+ *
+ *   y = x . W^T          x [M,d] bf16, W [V,d] bf16  (or their e4m3 copies:
+ *                        y = fp32(acc) * fp32(st_x->scale_inv * w_scale_inv[0]))
+ *   z = c tanh(y / c)    the softcap, 0 < c <= 40
+ *   lse[m] = logsumexp_v z[m,v]
+ *   loss_m = sum over t < T with 0 <= targets[m,t] < V of w_t (lse[m] - z[m, targets[m,t]])
+ *   loss[0] = sum_m loss_m, loss[1] = sum of the valid weights,
+ *   loss[2] = loss[0] / loss[1] (0 when no target is valid)
+ *
+ * targets [M,T] int32 row-major, 1 <= T <= 4; a target outside [0,V) is
+ * ignored.  target_weights: HOST array of T floats, or NULL for all 1.
+ * V and d multiples of 16 (pad the vocabulary; padded columns take part in
+ * the softmax).  The cap bounds |z| by c, so exp(z - c) never overflows and
+ * never falls below e^-80: no running maximum is kept.  lse [M] and loss[3]
+ * fp32 (caller-owned, 4-byte aligned); row_loss [M] fp32 or NULL.  The
+ * reductions run in double in a fixed order (deterministic).
+ * ------------------------------------------------------------------------ */
+#define FP8MLP_CE_SUM 0  /* the backward differentiates loss[0] */
+#define FP8MLP_CE_MEAN 1 /* the backward differentiates loss[2]  */
+
+/* Bytes of workspace (16-byte aligned, caller-owned, no initial contents)
+ * that fp8mlp_ce_fwd / fp8mlp_ce_fwd_fp8 need for M rows, V columns and T
+ * targets: per-row partial sums over 128-column groups, z at the targets and
+ * per-block sums.  0 for M = 0. */
+size_t fp8mlp_ce_workspace_size(int M, int V, int T);
+
+/* Forward on BF16 x and W: one GEMM whose epilogue softcaps and sums the
+ * logits tile by tile (nothing [M,V] is written), then two small passes. */
+int fp8mlp_ce_fwd(int M, int d, int V, int T, const uint16_t* x, const uint16_t* W, const int32_t* targets,
+                  const float* target_weights, float softcap, float* lse, float* row_loss, float* loss,
+                  void* workspace, fp8mlp_stream_t stream);
+
+/* Forward on the e4m3 copies: x_fp8 [M,d] from fp8mlp_quantize_x under st_x,
+ * Wq [V,d] from fp8mlp_weight_fp8_cache_refresh (scale 1 / w_scale_inv[0]). */
+int fp8mlp_ce_fwd_fp8(int M, int d, int V, int T, const uint8_t* x_fp8, const fp8mlp_scale_state* st_x,
+                      const uint8_t* Wq, const float* w_scale_inv, const int32_t* targets,
+                      const float* target_weights, float softcap, float* lse, float* row_loss, float* loss,
+                      void* workspace, fp8mlp_stream_t stream);
+
+/* Gradient of the loss with respect to the logits, recomputing y exactly as
+ * the forward did (same kernel, same precision):
+ *   dlogits[m,v] = bf16( g (W_m softmax(z_m)_v - sum_t w_t [v == targets[m,t]]) (1 - (z/c)^2) )
+ * W_m = sum of row m's valid weights; g = dloss[0] (NULL: 1), divided by
+ * loss[1] when reduction is FP8MLP_CE_MEAN (0 when loss[1] is 0).  lse and
+ * loss from the forward; dlogits [M,V] bf16.  The BF16 backward through the
+ * head is then fp8mlp_linear_bwd(M, d, V, x, W, dlogits, dX, dW). */
+int fp8mlp_ce_bwd_dlogits(int M, int d, int V, int T, const uint16_t* x, const uint16_t* W, const int32_t* targets,
+                          const float* target_weights, float softcap, const float* lse, const float* loss,
+                          const float* dloss, int reduction, uint16_t* dlogits, fp8mlp_stream_t stream);
+
+/* fp8mlp_ce_bwd_dlogits for a forward run on the e4m3 copies. */
+int fp8mlp_ce_bwd_dlogits_fp8(int M, int d, int V, int T, const uint8_t* x_fp8, const fp8mlp_scale_state* st_x,
+                              const uint8_t* Wq, const float* w_scale_inv, const int32_t* targets,
+                              const float* target_weights, float softcap, const float* lse, const float* loss,
+                              const float* dloss, int reduction, uint16_t* dlogits, fp8mlp_stream_t stream);
+
 /* Number of row blocks and column blocks of the partial-amax tensor for an
  * [M,h] post, and the block size in rows / columns.  Returns FP8MLP_OK. */
 int fp8mlp_partial_amax_shape(int M, int h, int* row_blocks, int* col_blocks, int* block_rows,

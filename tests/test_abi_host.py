@@ -118,3 +118,46 @@ def test_python_binding_rejects_non_contiguous():
     t = torch.zeros(4, 4)[:, ::2]
     with pytest.raises(ValueError):
         A.fp8mlp_bwd_dx(4, 16, 16, t, t, t, stream=0)
+
+
+def _ce_rc(**kw):
+    a = dict(M=256, d=64, V=512, T=1, x=FAKE, W=FAKE, targets=FAKE, w=None, cap=15.0, lse=FAKE, row=None,
+             loss=FAKE, ws=FAKE)
+    a.update(kw)
+    return _rc("fp8mlp_ce_fwd", a["M"], a["d"], a["V"], a["T"], a["x"], a["W"], a["targets"], a["w"],
+               ctypes.c_float(a["cap"]), a["lse"], a["row"], a["loss"], a["ws"], None)
+
+
+def test_ce_argument_checks():
+    assert _ce_rc(T=0) == A.ERR_INVALID_ARG
+    assert _ce_rc(T=5) == A.ERR_INVALID_ARG
+    assert _ce_rc(cap=0.0) == A.ERR_INVALID_ARG
+    assert _ce_rc(cap=41.0) == A.ERR_INVALID_ARG            # exp(-2c) would leave fp32's normal range
+    assert _ce_rc(cap=float("nan")) == A.ERR_INVALID_ARG
+    assert _ce_rc(V=500) == A.ERR_UNSUPPORTED_SHAPE         # vocabulary not a multiple of 16
+    assert _ce_rc(targets=None) == A.ERR_INVALID_ARG
+    assert _ce_rc(targets=FAKE + 2) == A.ERR_INVALID_ARG     # int32 targets need 4-byte alignment
+    assert _ce_rc(loss=None) == A.ERR_INVALID_ARG
+    bad_w = (ctypes.c_float * 1)(float("inf"))
+    assert _ce_rc(w=ctypes.cast(bad_w, ctypes.c_void_p)) == A.ERR_INVALID_ARG
+    # the backward's reduction selector
+    rc = _rc("fp8mlp_ce_bwd_dlogits", 256, 64, 512, 1, FAKE, FAKE, FAKE, None, ctypes.c_float(15.0), FAKE, FAKE,
+             None, 2, FAKE, None)
+    assert rc == A.ERR_INVALID_ARG
+
+
+def test_ce_workspace_layout():
+    # [block sums][partials: 2 per 256-column tile x M][z at targets: M x T], 256-byte aligned pieces
+    M, V, T = 16384, 50304, 1
+    nparts = 2 * -(-V // 256)
+    want = (2 * 8 * (M // 32)) + 4 * nparts * M + 4 * M * T
+    got = A.fp8mlp_ce_workspace_size(M, V, T)
+    assert want <= got < want + 3 * 256
+    assert A.fp8mlp_ce_workspace_size(0, V, T) == 0
+
+
+def test_ce_valid_call_without_gpu_reports_no_device():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _ce_rc() == A.ERR_NO_DEVICE
