@@ -39,6 +39,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "ReLU² MLP fwd+bwd tokens/s and % of FP8/BF16 roofline at d=768,h=3072"
+LINEAR_METRIC = "FP8 linear (attention QKV projection) fwd+bwd tokens/s and % of FP8/BF16 roofline"
+CE_METRIC = "softcapped cross-entropy LM head fwd+bwd tokens/s and % of FP8/BF16 roofline at d=768,V=50304"
+CE_CAP = 15.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
@@ -47,7 +50,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="step16k", choices=["step16k", "train49k", "heavytail", "stack9", "qkv16k"])
+    ap.add_argument("--workload", default="step16k", choices=["step16k", "train49k", "heavytail", "stack9", "qkv16k", "ce16k"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -56,6 +59,8 @@ def parse():
     ap.add_argument("--no-pdl", action="store_true", help="launch without programmatic dependent launch")
     ap.add_argument("--fp8-up", action="store_true",
                     help="run the up-projection on e4m3 copies of x and W1 as well (x quantiser + W1 cache per step)")
+    ap.add_argument("--bf16-head", action="store_true",
+                    help="ce16k: BF16 logits instead of the e4m3 LM head")
     ap.add_argument("--replicas", action="store_true",
                     help="with N>1, run independent replicas (no partial-amax / dW all-reduce)")
     return ap.parse_args()
@@ -203,6 +208,39 @@ def oracle_step_timer(W, tokens, seed=0):
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:  # pragma: no cover
         threads = 1
+    if W.name.startswith("ce"):
+        # the LM head: logits, softcapped cross-entropy, its gradient and the
+        # BF16 backward through the head (e4m3 logits from the oracle's copies)
+        # The step refreshes the weight cache once per W.M tokens; a sampled
+        # step of `tokens` tokens re-quantises the same share of W's rows.
+        # The full e4m3 copy the logits need is built once, before timing.
+        H = synth.make_head_problem(tokens, W.d, W.h, T=1, seed=seed)
+        Wq, _, swi = ref.w1_cache(H["W"])
+        share = max(1, (W.h * tokens) // W.M)
+
+        def step():
+            ref.w1_cache(H["W"][:share])
+            xq, _ = ref.quantise_x(H["x"], np.float32(448.0 / 10.0))
+            y = ref.head_logits_fp8(xq, Wq, np.float32(10.0 / 448.0), swi)
+            f = ref.ce_forward(y, H["targets"], [1.0], CE_CAP)
+            g = ref.ce_grad_scale(1.0, f["weight_sum"], True)
+            ref.ce_backward(H["x"], H["W"], ref.ce_backward_dlogits(y, H["targets"], [1.0], CE_CAP, f["lse"], g))
+            return np
+        return step, threads
+    if W.name.startswith("qkv"):
+        P = synth.make_problem(tokens, W.d, W.h, seed=seed)
+        g = synth.rng(5)
+        dY = synth.to_bf16_bits(g.standard_normal((tokens, W.h), dtype=np.float32))
+        st = {"s": ref.scale_state_init(W.margin, 1.0)}
+
+        def step():
+            xq, a = ref.quantise_x(P["x"], st["s"]["scale"])
+            Wq, _, swi = ref.w1_cache(P["W1"])
+            ref.linear_fp8(xq, Wq, st["s"]["scale_inv"], swi)
+            st["s"] = ref.scale_update(st["s"], a)
+            ref.linear_bwd(P["x"], P["W1"], dY)
+            return np
+        return step, threads
     if W.layers > 1:
         g = synth.rng(seed)
         r0 = synth.to_bf16_bits(synth.make_x(g, tokens, W.d, "normal"))
@@ -233,9 +271,25 @@ def oracle_step_timer(W, tokens, seed=0):
     return step, threads
 
 
-def cpu_baseline(W, seconds, tokens=512):
+def oracle_tokens(W, kind):
+    """Tokens per oracle step: about a second of host work per step."""
+    if W.name.startswith("ce"):
+        return 64
     if W.layers > 1:
-        tokens = 128
+        return 128 if kind == "baseline" else 32
+    return 512 if kind == "baseline" else 256
+
+
+def metric_of(W):
+    if W.name.startswith("ce"):
+        return CE_METRIC
+    if W.name.startswith("qkv"):
+        return LINEAR_METRIC
+    return METRIC
+
+
+def cpu_baseline(W, seconds, tokens=None):
+    tokens = tokens or oracle_tokens(W, "baseline")
     step, threads = oracle_step_timer(W, tokens)
     t0 = time.perf_counter()
     reps = 0
@@ -246,14 +300,17 @@ def cpu_baseline(W, seconds, tokens=512):
         if el >= seconds or reps >= 50:
             break
     return {"value": tokens * reps / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{reps} oracle steps of {tokens} tokens of the {W.name} workload "
-                      f"(d={W.d}, h={W.h}, {W.layers} layer(s); fwd+bwd+scale+W2 cache), {el:.1f} s"}
+            "sample": ("each step also re-quantises its token share of the head's rows (weight cache); "
+                       if W.name.startswith("ce") else "") +
+                      f"{reps} oracle steps of {tokens} tokens of the {W.name} workload "
+                      f"(d={W.d}, {'V' if W.name.startswith('ce') else 'h'}={W.h}, {W.layers} layer(s); "
+                      f"the whole fwd+bwd step), {el:.1f} s"}
 
 
 def run_reference(a, W, world, rank):
     if rank != 0:
         return
-    tokens = 256 if W.layers == 1 else 32
+    tokens = oracle_tokens(W, "reference")
     step, threads = oracle_step_timer(W, tokens)
     for _ in range(a.warmup):
         step()
@@ -263,7 +320,10 @@ def run_reference(a, W, world, rank):
     el = time.perf_counter() - t0
     v = tokens * a.steps / el
     sample = f"{a.steps} oracle steps of {tokens} tokens each (bounded sample of {W.name}: M={W.M}, d={W.d}, h={W.h})"
-    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": a.gpus, "steps": a.steps,
+    if W.name.startswith("ce"):
+        sample += (f"; each step also re-quantises {tokens}/{W.M} of the head's rows, its share of the "
+                   f"once-per-step weight-cache refresh")
+    line = {"metric": metric_of(W), "value": v, "unit": "tokens/s", "n_gpus": a.gpus, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": el / a.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64 (bf16/e4m3 rounding emulated)", "data": "synthetic",
             "config": config_of(W), "impl": "reference",
@@ -651,7 +711,7 @@ def run_linear(a, W, world, rank, local_rank):
             + (2 * M * K + M * K) / (peaks["hbm_gbs"] * 1e9))
     if rank == 0:
         line = {
-            "metric": "FP8 linear (attention QKV projection) fwd+bwd tokens/s and % of FP8/BF16 roofline",
+            "metric": LINEAR_METRIC,
             "value": M * a.steps / total_s, "unit": "tokens/s", "n_gpus": 1, "steps": a.steps, "warmup": a.warmup,
             "ms_per_step": total_s / a.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3 forward, bf16 backward (fp32 accumulate)", "data": "synthetic",
@@ -664,6 +724,254 @@ def run_linear(a, W, world, rank, local_rank):
             "launch_mode": "eager" if graph is None else "cuda_graph",
         }
         print(json.dumps(line), flush=True)
+
+
+def ce_work(M, d, V, fp8):
+    """FLOPs (by precision) and minimum HBM bytes of each call of a head step."""
+    F = 2 * M * d * V
+    e = 1 if fp8 else 2
+    nparts = 2 * -(-V // 256)
+    w = {
+        "ce_fwd": dict(bf16=0 if fp8 else F, fp8=F if fp8 else 0,
+                       bytes=e * M * d + e * V * d + 4 * M + 8 * nparts * M + 12 * M),
+        "ce_bwd_dlogits": dict(bf16=0 if fp8 else F, fp8=F if fp8 else 0,
+                               bytes=e * M * d + e * V * d + 8 * M + 2 * M * V),
+        "dx": dict(bf16=F, fp8=0, bytes=2 * M * V + 2 * V * d + 2 * M * d),
+        "dw": dict(bf16=F, fp8=0, bytes=2 * M * V + 2 * M * d + 4 * V * d),
+    }
+    if fp8:
+        w["quantize_x"] = dict(bf16=0, fp8=0, bytes=3 * M * d)
+        w["w_cache"] = dict(bf16=0, fp8=0, bytes=2 * (2 * V * d) + V * d)
+    return w
+
+
+def run_ce(a, W, world, rank, local_rank):
+    """The softcapped cross-entropy LM head: per step (e4m3 head) the x
+    quantiser, the fused head GEMM + cross-entropy, the x-scale update, the
+    dlogits GEMM, dX and dW through the BF16 head, the weight-cache refresh;
+    (BF16 head) the fused GEMM, dlogits, dX, dW.  Every rank runs its own
+    tokens (weak scaling, no collective).  One CUDA graph per step."""
+    import numpy as np
+    import torch
+    from fp8_relu_mlp_b200 import _abi as A
+    from fp8_relu_mlp_b200 import synth
+    from fp8_relu_mlp_b200.block import MLPBlock
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    A.fp8mlp_set_programmatic_launch(not a.no_pdl)
+    fp8 = not a.bf16_head
+    M, d, V = W.M, W.d, W.h
+    peaks = load_peaks()
+    fp8_peak, fp8_src = measure_fp8_peak(torch, peaks["bf16_tflops"])
+    H = synth.make_head_problem(M, d, V, T=1, seed=rank)
+    bf, u8, f32 = torch.bfloat16, torch.uint8, torch.float32
+    x = MLPBlock.bits_to_bf16(H["x"], dev)
+    Wt = MLPBlock.bits_to_bf16(H["W"], dev)
+    tg = torch.from_numpy(H["targets"]).to(dev)
+    lse = torch.empty(M, device=dev)
+    loss = torch.zeros(3, device=dev)
+    ws = torch.empty(A.fp8mlp_ce_workspace_size(M, V, 1), dtype=u8, device=dev)
+    dl = torch.empty(M, V, dtype=bf, device=dev)
+    dX = torch.empty(M, d, dtype=bf, device=dev)
+    dW = torch.empty(V, d, dtype=f32, device=dev)
+    st = torch.zeros(8, device=dev)
+    A.fp8mlp_scale_state_init(st, W.margin, 1.0)
+    xq = torch.empty(M, d, dtype=u8, device=dev)
+    npx = A.fp8mlp_x_partial_amax_count(M, d)
+    pax = torch.empty(npx, device=dev)
+    Wq = torch.empty(V, d, dtype=u8, device=dev)
+    winv = torch.ones(4, device=dev)
+    wsw = torch.empty(A.fp8mlp_workspace_size(0, d, V), dtype=u8, device=dev)
+    flush = torch.empty(256 << 20, dtype=u8, device=dev)
+    if fp8:
+        # the delayed x-scale needs one step of history
+        A.fp8mlp_weight_fp8_cache_refresh(V, d, Wt, Wq, winv, wsw)
+        A.fp8mlp_quantize_x(M, d, x, st, xq, pax)
+        A.fp8mlp_amax_reduce_update_scale(pax, npx, st)
+
+    calls = []
+    if fp8:
+        calls.append(("quantize_x", lambda: A.fp8mlp_quantize_x(M, d, x, st, xq, pax)))
+        calls.append(("ce_fwd", lambda: A.fp8mlp_ce_fwd_fp8(M, d, V, 1, xq, st, Wq, winv, tg, None, CE_CAP, lse,
+                                                            None, loss, ws)))
+        calls.append(("ce_bwd_dlogits", lambda: A.fp8mlp_ce_bwd_dlogits_fp8(M, d, V, 1, xq, st, Wq, winv, tg, None,
+                                                                            CE_CAP, lse, loss, None, A.CE_MEAN,
+                                                                            dl)))
+        calls.append(("x_scale", lambda: A.fp8mlp_amax_reduce_update_scale(pax, npx, st)))
+    else:
+        calls.append(("ce_fwd", lambda: A.fp8mlp_ce_fwd(M, d, V, 1, x, Wt, tg, None, CE_CAP, lse, None, loss, ws)))
+        calls.append(("ce_bwd_dlogits", lambda: A.fp8mlp_ce_bwd_dlogits(M, d, V, 1, x, Wt, tg, None, CE_CAP, lse,
+                                                                        loss, None, A.CE_MEAN, dl)))
+    # dX = dlogits . W is the same contraction as the MLP's dX = dPre . W1
+    calls.append(("dx", lambda: A.fp8mlp_bwd_dx(M, d, V, dl, Wt, dX)))
+    calls.append(("dw", lambda: A.fp8mlp_linear_bwd(M, d, V, x, Wt, dl, None, dW)))
+    if fp8:
+        calls.append(("w_cache", lambda: A.fp8mlp_weight_fp8_cache_refresh(V, d, Wt, Wq, winv, wsw)))
+    names = [n for n, _ in calls]
+    n_ev = len(calls) + 1
+
+    def step(ev=None, marks=None):
+        for i, (_, f) in enumerate(calls):
+            if ev is not None and (marks is None or i in marks):
+                ev[i].record()
+            f()
+        if ev is not None:
+            ev[n_ev - 1].record()
+
+    def graph_of(marks):
+        ev = [torch.cuda.Event(enable_timing=True, external=not a.eager) for _ in range(n_ev)]
+        if a.eager:
+            return None, ev
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(ev, marks)
+        return g, ev
+
+    def replay(g, ev, marks):
+        if g is not None:
+            g.replay()
+        else:
+            step(ev, marks)
+
+    step()
+    torch.cuda.synchronize()
+    # untimed breakdown: an event between every call
+    g_b, ev_b = graph_of(None)
+    per = {n: [] for n in names}
+    for _ in range(5):
+        flush.zero_()
+        replay(g_b, ev_b, None)
+        ev_b[-1].synchronize()
+        for i, n in enumerate(names):
+            per[n].append(ev_b[i].elapsed_time(ev_b[i + 1]))
+    breakdown = {n: statistics.median(v) for n, v in per.items()}
+    dom_i = max(range(len(names)), key=lambda k: breakdown[names[k]])
+    marks = {0, dom_i, dom_i + 1}
+    n_cap0 = A.fp8mlp_kernel_launch_count()
+    g_t, ev_t = graph_of(marks)
+    kernels_per_step = A.fp8mlp_kernel_launch_count() - n_cap0
+    for _ in range(max(a.warmup, 3)):
+        flush.zero_()
+        replay(g_t, ev_t, marks)
+    torch.cuda.synchronize()
+    A.fp8mlp_clear_device_status()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = A.fp8mlp_kernel_launch_count()
+    step_ms, dom_ms = [], []
+    with ClockSampler(local_rank) as clk:
+        for _ in range(a.steps):
+            flush.zero_()
+            replay(g_t, ev_t, marks)
+            ev_t[-1].synchronize()
+            step_ms.append(ev_t[0].elapsed_time(ev_t[-1]))
+            dom_ms.append(ev_t[dom_i].elapsed_time(ev_t[dom_i + 1]))
+        torch.cuda.synchronize()
+    launches = (A.fp8mlp_kernel_launch_count() - n0) if g_t is None else kernels_per_step * a.steps
+    status = A.fp8mlp_get_device_status()
+    total_s = sum(step_ms) * 1e-3
+    if dist:
+        t = torch.tensor([total_s], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_s = float(t.item())
+    work = ce_work(M, d, V, fp8)
+    dom = names[dom_i]
+    wd = work.get(dom, dict(bf16=0, fp8=0, bytes=0))
+    dom_s = statistics.mean(dom_ms) * 1e-3
+    if wd["bf16"] or wd["fp8"]:
+        peak_dom = fp8_peak if wd["fp8"] else peaks["bf16_tflops"]
+        roofline = {"bound": "tensor", "kernel": dom, "achieved": (wd["bf16"] + wd["fp8"]) / dom_s / 1e12,
+                    "peak": peak_dom, "unit": "TFLOP/s", "traffic": load_traffic(W.name).get(dom),
+                    "peak_source": fp8_src if wd["fp8"] else f"bf16_tflops burst of {peaks['source']} peaks"}
+    else:
+        roofline = {"bound": "hbm", "kernel": dom, "achieved": wd["bytes"] / dom_s / 1e9, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "traffic": load_traffic(W.name).get(dom),
+                    "peak_source": f"hbm_gbs of {peaks['source']} peaks"}
+    roofline["frac"] = roofline["achieved"] / roofline["peak"]
+    roof_t = sum(max(w["bf16"] / (peaks["bf16_tflops"] * 1e12) + w["fp8"] / (fp8_peak * 1e12),
+                     w["bytes"] / (peaks["hbm_gbs"] * 1e9)) for w in work.values())
+    fwd_s = breakdown["ce_fwd"] * 1e-3
+    wf = work["ce_fwd"]
+    fwd_roof = wf["bf16"] / (peaks["bf16_tflops"] * 1e12) + wf["fp8"] / (fp8_peak * 1e12)
+
+    e2e = None
+    if not a.no_e2e:
+        # the same step through the public API with host buffers: x and the
+        # targets come in from pinned host memory, the loss and dX go back
+        xh = torch.from_numpy(H["x"].view(np.int16)).view(bf).pin_memory()
+        th = torch.from_numpy(H["targets"]).pin_memory()
+        lh = torch.empty(3, dtype=f32).pin_memory()
+        dxh = torch.empty(M, d, dtype=bf).pin_memory()
+
+        def body():
+            x.copy_(xh, non_blocking=True)
+            tg.copy_(th, non_blocking=True)
+            step()
+            lh.copy_(loss, non_blocking=True)
+            dxh.copy_(dX, non_blocking=True)
+
+        body()
+        torch.cuda.synchronize()
+        ge = None
+        if not a.eager:
+            ge = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(ge):
+                body()
+        for _ in range(max(a.warmup, 3)):
+            ge.replay() if ge is not None else body()
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+        e0.record()
+        for _ in range(a.steps):
+            ge.replay() if ge is not None else body()
+        e1.record()
+        e1.synchronize()
+        te = e0.elapsed_time(e1) * 1e-3
+        if dist:
+            tt = torch.tensor([te], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            te = float(tt.item())
+        e2e = {"value": M * world * a.steps / te, "unit": "tokens/s",
+               "h2d_bytes_per_step": int(xh.numel() * 2 + th.numel() * 4),
+               "d2h_bytes_per_step": int(lh.numel() * 4 + dxh.numel() * 2)}
+    if rank == 0:
+        line = {
+            "metric": CE_METRIC, "value": M * world * a.steps / total_s, "unit": "tokens/s", "n_gpus": world,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": total_s / a.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": ("e4m3 head forward" if fp8 else "bf16 head forward") + ", bf16 backward (fp32 accumulate)",
+            "data": "synthetic (seeded; GPT-2 vocabulary padded to 50304, d=768)",
+            "config": dict(config_of(W), V=V, softcap=CE_CAP, targets_per_token=1, reduction="mean",
+                           head="e4m3 (x quantiser + weight cache in the step)" if fp8 else "bf16",
+                           parallelism=f"dp{world} replicas" if world > 1 else "single GPU"),
+            "roofline": roofline,
+            "step_roofline": {"roofline_ms": roof_t * 1e3, "measured_ms": total_s / a.steps * 1e3,
+                              "frac": roof_t / (total_s / a.steps), "fwd_ms": fwd_s * 1e3,
+                              "fwd_roofline_ms": fwd_roof * 1e3, "fwd_frac": fwd_roof / fwd_s,
+                              "peaks": {"bf16_tflops": peaks["bf16_tflops"], "fp8_tflops": fp8_peak,
+                                        "hbm_gbs": peaks["hbm_gbs"]}},
+            "kernels_ms": breakdown,
+            "kernels_ms_note": "median of 5 untimed steps with an event between every call; ce_fwd includes "
+                               "its two small reduction kernels",
+            "clocks": clk.summary(), "gpu_launches": int(launches), "device_status": status,
+            "launch_mode": ("eager" if g_t is None else "cuda_graph") + ("" if a.no_pdl else " + programmatic dependent launch"),
+        }
+        if e2e:
+            line["e2e"] = e2e
+        if not a.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(W, a.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 def run_stack(a, W, world, rank, local_rank):
@@ -903,6 +1211,8 @@ def main():
         return 0
     if W.name.startswith("qkv"):
         run_linear(a, W, world, rank, local_rank)
+    elif W.name.startswith("ce"):
+        run_ce(a, W, world, rank, local_rank)
     elif W.layers > 1:
         run_stack(a, W, world, rank, local_rank)
     else:

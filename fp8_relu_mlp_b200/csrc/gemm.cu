@@ -15,10 +15,10 @@ using CfgDPre = GemmCfg<2, kGemmBN, 3, false, false, false, Epi::DPre>;
 using CfgDW = GemmCfg<2, kGemmBN, 6, false, true, true, Epi::StoreF32, 4>;
 // LM head with the softcapped cross-entropy in the epilogue; the forward
 // stores no tile, so its shared memory all goes to the operand ring
-using CfgCeF = GemmCfg<2, kGemmBN, 6, false, false, false, Epi::CeFwd>;
-using CfgCeF8 = GemmCfg<2, kGemmBN, 6, true, false, false, Epi::CeFwd>;
-using CfgCeB = GemmCfg<2, kGemmBN, 6, false, false, false, Epi::CeBwd>;
-using CfgCeB8 = GemmCfg<2, kGemmBN, 6, true, false, false, Epi::CeBwd>;
+using CfgCeF = GemmCfg<2, kGemmBN, 6, false, false, false, Epi::CeFwd, 16>;
+using CfgCeF8 = GemmCfg<2, kGemmBN, 6, true, false, false, Epi::CeFwd, 16>;
+using CfgCeB = GemmCfg<2, kGemmBN, 5, false, false, false, Epi::CeBwd, 16>;
+using CfgCeB8 = GemmCfg<2, kGemmBN, 5, true, false, false, Epi::CeBwd, 16>;
 
 namespace {
 

@@ -145,15 +145,43 @@ __device__ __forceinline__ void store_row_bf16(uint32_t base, int lane, const ui
     st_shared_v4(base + swz<3>(lane * 64 + j * 16), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
 }
 
-// Softcap z = c tanh(y/c) from e = exp(-2|y|/c) and r = 1/(1+e):
-//   |tanh(y/c)| = (1-e) r,   t - 1 = -2r (y < 0) or -2er (y >= 0),
-//   1 - t^2 = 4 e r^2
-// so neither z - c = c (t-1) nor the derivative loses digits to cancellation.
-// k = -2 log2(e) / c.  Returns t - 1.
-__device__ __forceinline__ float softcap_tm1(float y, float k, float& e, float& r) {
-  e = ex2_approx(k * fabsf(y));
-  r = rcp_approx(1.f + e);
-  return -2.f * r * (y >= 0.f ? e : 1.f);
+// Softcap z = c tanh(y/c), t = tanh(y/c), from e = exp(-2|y|/c) in (0, 1]
+// and r = 1/(1+e):
+//   t - 1 = -2 s r  with s = e (y >= 0) or 1 (y < 0),     1 - t^2 = 4 e r^2,
+// so neither z - c = c (t - 1) nor the derivative loses digits to
+// cancellation.  kd = -2 log2(e) / c times the dequantising factor of the
+// accumulator (y = acc * dq, dq > 0), so e = 2^(kd |acc|).
+// r is computed on the FMA pipe (the special-function unit, which also runs
+// both exponentials, is the epilogue's bottleneck): a quadratic start with
+// relative error < 1.02e-2 on e in [0, 1] and two Newton-Raphson steps
+// r <- r + r (1 - (1+e) r), relative error < 1.4e-7 in fp32.
+__device__ __forceinline__ void softcap_er(float acc, float kd, float& e, float& r) {
+  e = ex2_approx(kd * fabsf(acc));
+  const float x = 1.f + e;
+  r = fmaf(fmaf(0.32321758f, e, -0.80804528f), e, 0.98988505f);
+  r = fmaf(r, fmaf(-x, r, 1.f), r);
+  r = fmaf(r, fmaf(-x, r, 1.f), r);
+}
+
+// softcap_er on the two accumulators (a0, a1) at once, packed: returns
+// e = (e0, e1) and r = (r0, r1) as fp32 pairs; kd2 = (kd, kd)
+__device__ __forceinline__ void softcap_er2(float a0, float a1, uint64_t kd2, uint64_t& e, uint64_t& r) {
+  const uint64_t one = f2_pack(1.f, 1.f), m1 = f2_pack(-1.f, -1.f);
+  float t0, t1;
+  f2_unpack(f2_mul(f2_pack(fabsf(a0), fabsf(a1)), kd2), t0, t1);
+  e = f2_pack(ex2_approx(t0), ex2_approx(t1));
+  const uint64_t nx = f2_fma(e, m1, m1);  // -(1 + e)
+  r = f2_fma(f2_fma(f2_pack(0.32321758f, 0.32321758f), e, f2_pack(-0.80804528f, -0.80804528f)), e,
+             f2_pack(0.98988505f, 0.98988505f));
+  r = f2_fma(r, f2_fma(nx, r, one), r);
+  r = f2_fma(r, f2_fma(nx, r, one), r);
+}
+
+// s r of the pair, s = e (accumulator >= 0) or 1: t - 1 = -2 s r
+__device__ __forceinline__ uint64_t softcap_sr2(float a0, float a1, uint64_t e, uint64_t r) {
+  float e0, e1;
+  f2_unpack(e, e0, e1);
+  return f2_mul(f2_pack(a0 >= 0.f ? e0 : 1.f, a1 >= 0.f ? e1 : 1.f), r);
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -364,7 +392,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
     float dq = 1.f;
     constexpr bool kCe = C::EPI == Epi::CeFwd || C::EPI == Epi::CeBwd;
     if constexpr ((C::EPI == Epi::UpFused || kCe) && C::FP8) dq = __fmul_rn(p.st_in->scale_inv, *p.w_in_scale_inv);
-    // cross-entropy backward: g, the factor of every row's gradient
+    // cross-entropy: the exponent constants (the e4m3 dequantising factor
+    // folded into kd) and, backward, g, the factor of every row's gradient
+    const float ce_kd = kCe ? p.ce_k * dq : 0.f;
+    const float ce_K = -2.f * p.ce_cl2;
     float ce_g = 0.f;
     if constexpr (C::EPI == Epi::CeBwd) {
       ce_g = p.ce_dloss != nullptr ? *p.ce_dloss : 1.f;
@@ -412,7 +443,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
       // (lse - c) log2(e) and g times the row's weight
       const int ce_m = row0 + lane;
       int ce_tg[4] = {-1, -1, -1, -1};
-      float ce_sum = 0.f, ce_L = 0.f, ce_gw = 0.f;
+      float ce_sum = 0.f, ce_L = 0.f, ce_gw4 = 0.f;
       if constexpr (kCe) {
         if (ce_m < p.M) {
           float wsum = 0.f;
@@ -428,7 +459,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
           }
           if constexpr (C::EPI == Epi::CeBwd) {
             ce_L = __fmul_rn(__fsub_rn(p.ce_lse[ce_m], p.ce_cap), kLog2e);
-            ce_gw = __fmul_rn(ce_g, wsum);
+            ce_gw4 = 4.f * __fmul_rn(ce_g, wsum);
           }
         }
       }
@@ -537,57 +568,78 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
           }
         } else if constexpr (C::EPI == Epi::CeFwd) {
           // sum over the chunk's columns inside the vocabulary of exp(z - c) =
-          // 2^(c log2(e) (t - 1)); |z| <= c keeps every term in [e^-2c, 1]
-          const int nvalid = p.N - col0;
-          float csum = 0.f;
+          // 2^(c log2(e) (t - 1)) = 2^(K s r), K = -2 c log2(e); |z| <= c keeps
+          // every term in [e^-2c, 1]
+          // (pairs of columns in packed fp32)
+          const uint64_t kd2 = f2_pack(ce_kd, ce_kd), K2 = f2_pack(ce_K, ce_K);
+          uint64_t csum2 = f2_pack(0.f, 0.f);
+          if (col0 + 32 <= p.N) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float y = __uint_as_float(v[i]);
-            if constexpr (C::FP8) y = __fmul_rn(y, dq);
-            float ee, rr;
-            const float term = ex2_approx(p.ce_cl2 * softcap_tm1(y, p.ce_k, ee, rr));
-            csum += i < nvalid ? term : 0.f;
+            for (int i = 0; i < 32; i += 2) {
+              const float a0 = __uint_as_float(v[i]), a1 = __uint_as_float(v[i + 1]);
+              uint64_t e2, r2;
+              softcap_er2(a0, a1, kd2, e2, r2);
+              float g0, g1;
+              f2_unpack(f2_mul(softcap_sr2(a0, a1, e2, r2), K2), g0, g1);
+              csum2 = f2_add(csum2, f2_pack(ex2_approx(g0), ex2_approx(g1)));
+            }
+          } else {  // the vocabulary's last, partial chunk
+            const int nvalid = p.N - col0;
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const float a0 = __uint_as_float(v[i]), a1 = __uint_as_float(v[i + 1]);
+              uint64_t e2, r2;
+              softcap_er2(a0, a1, kd2, e2, r2);
+              float g0, g1;
+              f2_unpack(f2_mul(softcap_sr2(a0, a1, e2, r2), K2), g0, g1);
+              csum2 = f2_add(csum2, f2_pack(i < nvalid ? ex2_approx(g0) : 0.f, i + 1 < nvalid ? ex2_approx(g1) : 0.f));
+            }
           }
-          ce_sum += csum;
-          // z - c at the row's targets that fall in this chunk (one thread in
-          // the grid owns each (row, target))
+          float cs0, cs1;
+          f2_unpack(csum2, cs0, cs1);
+          ce_sum += cs0 + cs1;
+          // z - c = -2c s r at the row's targets that fall in this chunk (one
+          // thread in the grid owns each (row, target))
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
             const int off = ce_tg[t] - col0;
             if (off >= 0 && off < 32) {
-              float yv = 0.f;
+              float av = 0.f;
 #pragma unroll
-              for (int i = 0; i < 32; ++i) yv = i == off ? __uint_as_float(v[i]) : yv;
-              if constexpr (C::FP8) yv = __fmul_rn(yv, dq);
+              for (int i = 0; i < 32; ++i) av = i == off ? __uint_as_float(v[i]) : av;
               float ee, rr;
-              const float tm1 = softcap_tm1(yv, p.ce_k, ee, rr);
-              p.ce_ztgt[static_cast<size_t>(ce_m) * p.ce_T + t] = __fmul_rn(p.ce_cap, tm1);
+              softcap_er(av, ce_kd, ee, rr);
+              p.ce_ztgt[static_cast<size_t>(ce_m) * p.ce_T + t] = (-2.f * p.ce_cap) * ((av >= 0.f ? ee : 1.f) * rr);
             }
           }
         } else if constexpr (C::EPI == Epi::CeBwd) {
-          // dL/dy = g (W_m softmax(z) - sum_t w_t onehot(tgt_t)) (1 - t^2)
+          // dL/dy = g (W_m softmax(z) - sum_t w_t onehot(tgt_t)) (1 - t^2),
+          // softmax(z) = 2^(K s r - (lse - c) log2(e)),  1 - t^2 = 4 e r^2
+          // (pairs of columns in packed fp32)
           float dy[32];
+          const uint64_t kd2 = f2_pack(ce_kd, ce_kd), K2 = f2_pack(ce_K, ce_K);
+          const uint64_t nL2 = f2_pack(-ce_L, -ce_L), gw2 = f2_pack(ce_gw4, ce_gw4);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float y = __uint_as_float(v[i]);
-            if constexpr (C::FP8) y = __fmul_rn(y, dq);
-            float ee, rr;
-            const float tm1 = softcap_tm1(y, p.ce_k, ee, rr);
-            const float prob = ex2_approx(fmaf(p.ce_cl2, tm1, -ce_L));  // exp(z - lse)
-            const float der = 4.f * ee * rr * rr;
-            dy[i] = ce_gw * prob * der;
+          for (int i = 0; i < 32; i += 2) {
+            const float a0 = __uint_as_float(v[i]), a1 = __uint_as_float(v[i + 1]);
+            uint64_t e2, r2;
+            softcap_er2(a0, a1, kd2, e2, r2);
+            float g0, g1;
+            f2_unpack(f2_fma(K2, softcap_sr2(a0, a1, e2, r2), nL2), g0, g1);
+            const uint64_t prob = f2_pack(ex2_approx(g0), ex2_approx(g1));  // exp(z - lse)
+            const uint64_t der = f2_mul(f2_mul(e2, r2), r2);                // (1 - t^2) / 4
+            f2_unpack(f2_mul(f2_mul(gw2, prob), der), dy[i], dy[i + 1]);
           }
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
             const int off = ce_tg[t] - col0;
             if (off >= 0 && off < 32) {
-              float yv = 0.f;
+              float av = 0.f;
 #pragma unroll
-              for (int i = 0; i < 32; ++i) yv = i == off ? __uint_as_float(v[i]) : yv;
-              if constexpr (C::FP8) yv = __fmul_rn(yv, dq);
+              for (int i = 0; i < 32; ++i) av = i == off ? __uint_as_float(v[i]) : av;
               float ee, rr;
-              softcap_tm1(yv, p.ce_k, ee, rr);
-              const float sub = ce_g * p.ce_w[t] * (4.f * ee * rr * rr);
+              softcap_er(av, ce_kd, ee, rr);
+              const float sub = (4.f * ce_g * p.ce_w[t]) * ((ee * rr) * rr);
 #pragma unroll
               for (int i = 0; i < 32; ++i) dy[i] = i == off ? dy[i] - sub : dy[i];
             }

@@ -6,9 +6,9 @@ Tolerances follow from the arithmetic of the kernels:
     exact in fp32); otherwise within eps_y = d 2^-24 max_v sum_k |x_k W_vk|
     (fp32 accumulation in any order; 2^-14 per add for the e4m3 GEMM, whose
     accumulation need not round to full fp32);
-  * lse, z - c: the hardware 2^x and reciprocal (relative error ~2^-22) and
-    the fp32 sum of 128 terms per thread give |error| < 3e-5; tested at
-    5e-5 + eps_y;
+  * lse, z - c: the hardware 2^x (relative error ~2^-22), the Newton
+    reciprocal (< 1.4e-7) and the fp32 sum of 128 terms per thread give
+    |error| < 3e-5; tested at 5e-5 + eps_y;
   * dlogits: BF16 rounding (2^-9 relative) plus, where the one-hot cancels
     against the softmax, an absolute part 1e-4 g W_m p (1 - t^2).
 """
