@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 32 * C::NEPI * CG);
+      mbar_init(&tempty[a], C::NEPI * CG);  // one arrival per epilogue warp of the pair
     }
     for (int i = 0; i < C::NEPI * C::NAUX; ++i) mbar_init(&auxb[i], 1);
     mbar_init(fin, 1);
@@ -473,11 +473,17 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
         uint32_t v[32];
         tmem_ld32(tmem_base + lane_base + acc * C::BN + c * C::ECOLS, v);
         if (cw == C::NCH_W - 1) {
+          // every lane's TMEM loads of this accumulator are complete (the load
+          // waits); order them before the warp's single release to the MMA
+          // issuer (a cluster-scope release per lane stalls on a memory barrier)
           tc_fence_before();
-          if constexpr (CG == 1)
-            mbar_arrive(&tempty[acc]);
-          else
-            mbar_arrive_cluster(tempty_addr0 + acc * 8u);
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (CG == 1)
+              mbar_arrive(&tempty[acc]);
+            else
+              mbar_arrive_cluster(tempty_addr0 + acc * 8u);
+          }
         }
         uint8_t* slot = sEpi + (e * 2 + (ctr & 1u)) * C::SLOT;
         const uint32_t sbase = smem_u32(slot);
