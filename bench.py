@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--no-pdl", action="store_true", help="launch without programmatic dependent launch")
     ap.add_argument("--fp8-up", action="store_true",
                     help="run the up-projection on e4m3 copies of x and W1 as well (x quantiser + W1 cache per step)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the workload's token count (small cases for profiling; not a bench line)")
     ap.add_argument("--bf16-head", action="store_true",
                     help="ce16k: BF16 logits instead of the e4m3 LM head")
     ap.add_argument("--replicas", action="store_true",
@@ -730,10 +732,10 @@ def ce_work(M, d, V, fp8):
     """FLOPs (by precision) and minimum HBM bytes of each call of a head step."""
     F = 2 * M * d * V
     e = 1 if fp8 else 2
-    nparts = 2 * -(-V // 256)
+    nparts = 4 * -(-V // 256)  # partial sums per row: one per epilogue warp's 64 columns of a tile
     w = {
         "ce_fwd": dict(bf16=0 if fp8 else F, fp8=F if fp8 else 0,
-                       bytes=e * M * d + e * V * d + 4 * M + 8 * nparts * M + 12 * M),
+                       bytes=e * M * d + e * V * d + 2 * 4 * nparts * M + 12 * M),
         "ce_bwd_dlogits": dict(bf16=0 if fp8 else F, fp8=F if fp8 else 0,
                                bytes=e * M * d + e * V * d + 8 * M + 2 * M * V),
         "dx": dict(bf16=F, fp8=0, bytes=2 * M * V + 2 * V * d + 2 * M * d),
@@ -1203,6 +1205,11 @@ def main():
     a = parse()
     from fp8_relu_mlp_b200 import synth
     W = synth.WORKLOADS[a.workload]
+    if a.tokens:
+        # a smaller case of the same workload (ncu captures); the committed
+        # traffic figures are per full-size launch, so they are not looked up
+        import dataclasses
+        W = dataclasses.replace(W, M=a.tokens, name=f"{W.name}@{a.tokens}")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

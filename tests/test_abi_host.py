@@ -147,9 +147,10 @@ def test_ce_argument_checks():
 
 
 def test_ce_workspace_layout():
-    # [block sums][partials: 2 per 256-column tile x M][z at targets: M x T], 256-byte aligned pieces
+    # [block sums][partials: 4 per 256-column tile (one per epilogue warp's
+    # 64 columns) x M][z at targets: M x T], 256-byte aligned pieces
     M, V, T = 16384, 50304, 1
-    nparts = 2 * -(-V // 256)
+    nparts = 4 * -(-V // 256)
     want = (2 * 8 * (M // 32)) + 4 * nparts * M + 4 * M * T
     got = A.fp8mlp_ce_workspace_size(M, V, T)
     assert want <= got < want + 3 * 256
