@@ -120,6 +120,57 @@ class MLPBlock:
         self.backward()
         self.update_scale()
 
+    def train_step_overlapped(self, side, refresh_w2: bool = True, mark=None):
+        """One training step with the small launches off the critical path.
+
+        ``side`` is a second CUDA stream.  The W2 cache refresh (from the
+        current W2: call this after the optimizer's update) runs on ``side``
+        beside the up-projection, which does not read the cache, and is joined
+        before the down-projection; the delayed-scale update runs on ``side``
+        beside the backward GEMMs, which do not read the scale, and is joined
+        at the end.  The calls and their results are those of
+        ``refresh_w2_cache(); train_step()``.  With the FP8 up-projection the
+        W1 cache refresh (the same workspace) stays on the main stream, first.
+        ``mark(i)``, if given, is called on the main stream at 0 (start), after
+        the up-projection (1), the down-projection (2), dPre (3), dX (4), dW
+        (5), and at the end (7)."""
+        mark = mark or (lambda i: None)
+        M, d, h = self.M, self.d, self.h
+        main = torch.cuda.current_stream(self.device) if self.stream is None else self.stream
+        mark(0)
+        if self.fp8_up:
+            self.refresh_w1_cache()
+        if refresh_w2:
+            side.wait_stream(main)
+            with torch.cuda.stream(side):
+                A.fp8mlp_w2_fp8_cache_refresh(h, d, self.W2, self.W2q_t, self.w2_scale_inv, self.workspace, side)
+        if self.fp8_up:
+            self._quantize_x()
+            self._up_fp8(0)
+        else:
+            A.fp8mlp_up_proj_fused(M, d, h, self.x, self.W1, self.state, self.post, self.post_fp8, self.partial_amax,
+                                   None, 0, self.stream)
+        mark(1)
+        if refresh_w2:
+            main.wait_stream(side)
+        A.fp8mlp_down_proj_fp8(M, d, h, self.post_fp8, self.W2q_t, self.w2_scale_inv, self.state, self.out,
+                               self.stream)
+        mark(2)
+        side.wait_stream(main)
+        with torch.cuda.stream(side):
+            A.fp8mlp_amax_reduce_update_scale(self.partial_amax, self.partial_amax.numel(), self.state, side)
+            if self.fp8_up:
+                A.fp8mlp_amax_reduce_update_scale(self.partial_amax_x, A.fp8mlp_x_partial_amax_count(M, d),
+                                                  self.state_x, side)
+        A.fp8mlp_bwd_dpre(M, d, h, self.dOut, self.W2, self.post, self.dPre, self.stream)
+        mark(3)
+        A.fp8mlp_bwd_dx(M, d, h, self.dPre, self.W1, self.dX, self.stream)
+        mark(4)
+        A.fp8mlp_bwd_dw(M, d, h, self.x, self.dPre, self.post, self.dOut, self.dW1, self.dW2, self.stream)
+        mark(5)
+        main.wait_stream(side)
+        mark(7)
+
     # ------------------------------------------------------------ CUDA graph
     def capture(self, fn):
         """Record the library calls made by ``fn()`` into a CUDA graph and return
