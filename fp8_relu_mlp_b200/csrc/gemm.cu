@@ -10,7 +10,7 @@ using CfgUp = GemmCfg<2, kGemmBN, 5, false, false, false, Epi::UpFused>;
 using CfgDown8 = GemmCfg<2, kGemmBN, 6, true, false, false, Epi::DownScaled>;
 using CfgBf16MnB = GemmCfg<2, kGemmBN, 6, false, false, true, Epi::StoreBf16>;
 using CfgUpQ = GemmCfg<2, kGemmBN, 5, true, false, false, Epi::UpFused>;
-using CfgDPre = GemmCfg<2, kGemmBN, 3, false, false, false, Epi::DPre>;
+using CfgDPre = GemmCfg<2, kGemmBN, 4, false, false, false, Epi::DPre>;
 // dW: one long tile per CTA pair, so a light epilogue (4 warps) and more stages
 using CfgDW = GemmCfg<2, kGemmBN, 6, false, true, true, Epi::StoreF32, 4>;
 // LM head with the softcapped cross-entropy in the epilogue; the forward
