@@ -72,7 +72,8 @@ struct alignas(64) GemmParams {
   const float* ce_dloss;     // CeBwd: gradient of the reduced loss (NULL = 1)
 };
 
-template <int CG_, int BN_, int STAGES_, bool FP8_, bool A_MN_, bool B_MN_, Epi EPI_, int NEPI_ = 8>
+template <int CG_, int BN_, int STAGES_, bool FP8_, bool A_MN_, bool B_MN_, Epi EPI_, int NEPI_ = 8,
+          int AUX_RING_ = 4>
 struct GemmCfg {
   static constexpr int CG = CG_;           // CTAs per UMMA (1, or 2 = the pair of a cluster)
   static constexpr int BM = 128;           // accumulator rows per CTA (TMEM lanes)
@@ -114,11 +115,12 @@ struct GemmCfg {
   static constexpr int OUT2_BUF = EPI == Epi::UpFused ? 32 * ECOLS : 0;
   static constexpr int SLOT = OUT_BUF + OUT2_BUF;  // one output staging slot (two per epilogue warp)
   static_assert(SLOT % 1024 == 0, "slot alignment");
-  // DPre: each epilogue warp keeps the post block of a whole tile (NCHUNK
-  // chunks of 32x32) in its own ring, loaded one tile ahead
+  // DPre: each epilogue warp streams its 32x32 blocks of post through a ring
+  // of NAUX slots of its own, loaded NAUX chunks ahead of use
   static constexpr int AUX_CHUNK = EPI == Epi::DPre ? 32 * ECOLS * 2 : 0;
-  static constexpr int AUX_WARP = AUX_CHUNK * NCH_W;
-  static constexpr int NAUX = EPI == Epi::DPre ? NCH_W : 0;
+  static constexpr int NAUX = EPI == Epi::DPre ? AUX_RING_ : 0;  // ring slots per warp
+  static constexpr int AUX_WARP = AUX_CHUNK * NAUX;
+  static_assert(NAUX == 0 || (NAUX <= NCH_W && NCH_W % NAUX == 0), "post ring");
   static constexpr int TMEM_COLS = 512;
   static_assert(2 * BN <= TMEM_COLS, "two accumulators");
   static constexpr int NUM_BARS = 2 * STAGES + 4 + NEPI * NAUX + 1;
@@ -404,9 +406,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
         ce_g = ws > 0.f ? __fdiv_rn(ce_g, ws) : 0.f;
       }
     }
-    // DPre: rounds of post prefetch started (one round = a tile's NAUX chunks,
-    // ring slot c = chunk c) and how many slots the latest round has reached
-    uint32_t aux_rounds = 0, aux_last = 0;
+    // DPre: this warp's post chunks, counted over its tiles (chunk q = tile
+    // iter, column chunk cw: q = iter * NCH_W + cw), go through ring slot
+    // q % NAUX; aux_issued = chunks whose load has been issued
+    uint32_t aux_issued = 0;
     uint8_t* aux_ring = sAux + e * C::AUX_WARP;
     uint64_t* my_auxb = auxb + e * C::NAUX;
     auto tile_rows = [&](int tile) {  // first row of this warp's 32 rows in `tile`
@@ -426,8 +429,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
             tma_load_2d(aux_ring + c * C::AUX_CHUNK, &p.tmAux, &my_auxb[c], c0 + (c_begin + c) * C::ECOLS, r0);
           }
         }
-        aux_rounds = 1;
-        aux_last = C::NAUX;
+        aux_issued = C::NAUX;
       }
     }
     uint32_t iter = 0;  // tiles processed by this CTA
@@ -545,24 +547,29 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
           store_row_bf16<64>(sbase, lane, pk);
         } else if constexpr (C::EPI == Epi::DPre) {
           // post of this chunk was loaded one tile ahead into ring slot c
-          if (!mbar_wait(&my_auxb[cw], iter & 1u, w)) {
+          const uint32_t q_aux = iter * C::NCH_W + cw;
+          const int slot_aux = static_cast<int>(q_aux % C::NAUX);
+          if (!mbar_wait(&my_auxb[slot_aux], (q_aux / C::NAUX) & 1u, w)) {
             ok = false;
           } else {
-            const uint32_t ab = smem_u32(aux_ring + cw * C::AUX_CHUNK);
+            const uint32_t ab = smem_u32(aux_ring + slot_aux * C::AUX_CHUNK);
             uint32_t pp[16], pk[16];
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               ld_shared_v4(ab + swz<3>(lane * 64 + j * 16), pp[4 * j], pp[4 * j + 1], pp[4 * j + 2], pp[4 * j + 3]);
             __syncwarp();
-            // ring slot c is free again: fetch the next tile's chunk c into it
-            if (next_tile < num_tiles) {
+            // the slot is free again: fetch chunk q + NAUX into it (column
+            // chunk cw + NAUX of this tile, or of the next one)
+            const int cw_n = cw + C::NAUX;
+            const int t_n = cw_n < C::NCH_W ? t : next_tile;
+            if (t_n < num_tiles) {
+              const int cn = cw_n < C::NCH_W ? cw_n : cw_n - C::NCH_W;
               if (lane == 0) {
-                mbar_arrive_expect_tx(&my_auxb[cw], C::AUX_CHUNK);
-                tma_load_2d(aux_ring + cw * C::AUX_CHUNK, &p.tmAux, &my_auxb[cw],
-                            tile_cols(next_tile) + c * C::ECOLS, tile_rows(next_tile));
+                mbar_arrive_expect_tx(&my_auxb[slot_aux], C::AUX_CHUNK);
+                tma_load_2d(aux_ring + slot_aux * C::AUX_CHUNK, &p.tmAux, &my_auxb[slot_aux],
+                            tile_cols(t_n) + (c_begin + cn) * C::ECOLS, tile_rows(t_n));
               }
-              if (cw == 0) aux_rounds = iter + 2;
-              aux_last = cw + 1;
+              aux_issued = q_aux + C::NAUX + 1;
             }
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -693,9 +700,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
     if (lane == 0) {
       if constexpr (C::EPI == Epi::DPre) {
         // the last load issued into each ring slot must have landed before exit
-        for (int c = 0; c < C::NAUX; ++c) {
-          const uint32_t n = static_cast<uint32_t>(c) < aux_last ? aux_rounds : aux_rounds - 1u;
-          if (n > 0) mbar_wait_drain(&my_auxb[c], (n - 1u) & 1u, p.timeout_ns);
+        for (uint32_t c = 0; c < static_cast<uint32_t>(C::NAUX); ++c) {
+          if (aux_issued > c) {
+            const uint32_t q_last = c + ((aux_issued - 1u - c) / C::NAUX) * C::NAUX;  // last chunk in slot c
+            mbar_wait_drain(&my_auxb[c], (q_last / C::NAUX) & 1u, p.timeout_ns);
+          }
         }
       }
       bulk_wait<0>();

@@ -579,6 +579,40 @@ def test_overlapped_step_matches_serial(fp8_up):
         assert torch.equal(getattr(e, k), getattr(g, k)), k
 
 
+def test_host_pipeline_matches_in_place_steps():
+    # inputs from pinned host memory and results back to it, with the copies
+    # overlapped across two buffer sets: the same step sequence as stepping
+    # the block in place, so the host copies of the last step's results, the
+    # scale state and the weight gradients are bit-identical
+    from fp8_relu_mlp_b200.block import MLPBlock
+    from fp8_relu_mlp_b200.hostio import block_pipeline
+    M, d, h = 1000, 768, 3072
+    P = synth.make_problem(M, d, h, seed=79)
+
+    def make():
+        b = MLPBlock(M, d, h)
+        for k in ("x", "W1", "W2", "dOut"):
+            getattr(b, k).copy_(MLPBlock.bits_to_bf16(P[k], b.device))
+        b.refresh_w2_cache()
+        b.calibrate()
+        return b
+
+    side = torch.cuda.Stream()
+    ref_b, pipe_b = make(), make()
+    pipe = block_pipeline(pipe_b, side)          # one warm-up step per buffer set
+    host_in = [MLPBlock.bits_to_bf16(P[k], "cpu").pin_memory() for k in ("x", "dOut")]
+    host_out = [torch.empty(M, d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    pipe.run(host_in, host_out, steps=5)
+    for _ in range(2 + 5):
+        ref_b.refresh_w2_cache()
+        ref_b.train_step()
+    torch.cuda.synchronize()
+    assert torch.equal(host_out[0], ref_b.out.cpu())
+    assert torch.equal(host_out[1], ref_b.dX.cpu())
+    for k in ("state", "dW1", "dW2", "W2q_t", "partial_amax"):
+        assert torch.equal(getattr(ref_b, k), getattr(pipe_b, k)), k
+
+
 # ---------------------------------------------------------------------------
 # layer stack: RMSNorm + block + residual, forward and backward
 # ---------------------------------------------------------------------------
