@@ -689,17 +689,18 @@ def run_linear(a, W, world, rank, local_rank):
     A.fp8mlp_quantize_x(M, K, x, st, xq, pax)
     A.fp8mlp_amax_reduce_update_scale(pax, npx, st)
 
-    def step(ev=None):
+    def step(ev=None, bufs=None):
         def mark(i):
             if ev is not None:
                 ev[i].record()
+        xb, dYb, yb, dXb = bufs if bufs is not None else (x, dY, y, dX)
         mark(0)
-        A.fp8mlp_quantize_x(M, K, x, st, xq, pax)
+        A.fp8mlp_quantize_x(M, K, xb, st, xq, pax)
         mark(1)
-        A.fp8mlp_linear_fwd_fp8(M, K, N, xq, Wq, winv, st, y)
+        A.fp8mlp_linear_fwd_fp8(M, K, N, xq, Wq, winv, st, yb)
         mark(2)
         A.fp8mlp_amax_reduce_update_scale(pax, npx, st)
-        A.fp8mlp_linear_bwd(M, K, N, x, Wt, dY, dX, dW)
+        A.fp8mlp_linear_bwd(M, K, N, xb, Wt, dYb, dXb, dW)
         A.fp8mlp_weight_fp8_cache_refresh(N, K, Wt, Wq, winv, ws)
         mark(3)
 
@@ -735,6 +736,26 @@ def run_linear(a, W, world, rank, local_rank):
     achieved = F / fwd_s / 1e12
     roof = (F / (fp8_peak * 1e12) + 2 * F / (peaks["bf16_tflops"] * 1e12)
             + (2 * M * K + M * K) / (peaks["hbm_gbs"] * 1e9))
+    e2e = None
+    if not a.no_e2e:
+        # x and the upstream gradient dY in from pinned host memory, y and dX
+        # back, every step; copies overlapped with the neighbouring steps
+        from fp8_relu_mlp_b200.hostio import HostPipeline
+        xh, dyh = x.cpu().pin_memory(), dY.cpu().pin_memory()
+        yh, dxh = torch.empty_like(y, device="cpu").pin_memory(), torch.empty_like(dX, device="cpu").pin_memory()
+        sets = [(x, dY, y, dX), (x.clone(), dY.clone(), torch.empty_like(y), torch.empty_like(dX))]
+        pipe = HostPipeline(lambda k: step(bufs=sets[k]), [[sb[0], sb[1]] for sb in sets],
+                            [[sb[2], sb[3]] for sb in sets], device=dev, graph=not a.eager)
+        pipe.run([xh, dyh], [yh, dxh], max(a.warmup, 3))
+        torch.cuda.synchronize()
+        timer = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        pipe.run([xh, dyh], [yh, dxh], a.steps, timer)
+        timer[1].synchronize()
+        te = timer[0].elapsed_time(timer[1]) * 1e-3
+        e2e = {"value": M * a.steps / te, "unit": "tokens/s",
+               "h2d_bytes_per_step": int(2 * (xh.numel() + dyh.numel())),
+               "d2h_bytes_per_step": int(2 * (yh.numel() + dxh.numel())),
+               "overlap": "copies on two streams beside the compute, double-buffered device sets"}
     if rank == 0:
         line = {
             "metric": LINEAR_METRIC,
@@ -749,6 +770,8 @@ def run_linear(a, W, world, rank, local_rank):
             "clocks": clk.summary(), "gpu_launches": int(kps * a.steps),
             "launch_mode": "eager" if graph is None else "cuda_graph",
         }
+        if e2e:
+            line["e2e"] = e2e
         print(json.dumps(line), flush=True)
 
 
@@ -820,24 +843,30 @@ def run_ce(a, W, world, rank, local_rank):
         A.fp8mlp_quantize_x(M, d, x, st, xq, pax)
         A.fp8mlp_amax_reduce_update_scale(pax, npx, st)
 
-    calls = []
-    if fp8:
-        calls.append(("quantize_x", lambda: A.fp8mlp_quantize_x(M, d, x, st, xq, pax)))
-        calls.append(("ce_fwd", lambda: A.fp8mlp_ce_fwd_fp8(M, d, V, 1, xq, st, Wq, winv, tg, None, CE_CAP, lse,
-                                                            None, loss, ws)))
-        calls.append(("ce_bwd_dlogits", lambda: A.fp8mlp_ce_bwd_dlogits_fp8(M, d, V, 1, xq, st, Wq, winv, tg, None,
-                                                                            CE_CAP, lse, loss, None, A.CE_MEAN,
-                                                                            dl)))
-        calls.append(("x_scale", lambda: A.fp8mlp_amax_reduce_update_scale(pax, npx, st)))
-    else:
-        calls.append(("ce_fwd", lambda: A.fp8mlp_ce_fwd(M, d, V, 1, x, Wt, tg, None, CE_CAP, lse, None, loss, ws)))
-        calls.append(("ce_bwd_dlogits", lambda: A.fp8mlp_ce_bwd_dlogits(M, d, V, 1, x, Wt, tg, None, CE_CAP, lse,
-                                                                        loss, None, A.CE_MEAN, dl)))
-    # dX = dlogits . W is the same contraction as the MLP's dX = dPre . W1
-    calls.append(("dx", lambda: A.fp8mlp_bwd_dx(M, d, V, dl, Wt, dX)))
-    calls.append(("dw", lambda: A.fp8mlp_linear_bwd(M, d, V, x, Wt, dl, None, dW)))
-    if fp8:
-        calls.append(("w_cache", lambda: A.fp8mlp_weight_fp8_cache_refresh(V, d, Wt, Wq, winv, wsw)))
+    def make_calls(x, tg, dX, loss):
+        """The step's calls on one set of input / result buffers."""
+        calls = []
+        if fp8:
+            calls.append(("quantize_x", lambda: A.fp8mlp_quantize_x(M, d, x, st, xq, pax)))
+            calls.append(("ce_fwd", lambda: A.fp8mlp_ce_fwd_fp8(M, d, V, 1, xq, st, Wq, winv, tg, None, CE_CAP, lse,
+                                                                None, loss, ws)))
+            calls.append(("ce_bwd_dlogits", lambda: A.fp8mlp_ce_bwd_dlogits_fp8(M, d, V, 1, xq, st, Wq, winv, tg,
+                                                                                None, CE_CAP, lse, loss, None,
+                                                                                A.CE_MEAN, dl)))
+            calls.append(("x_scale", lambda: A.fp8mlp_amax_reduce_update_scale(pax, npx, st)))
+        else:
+            calls.append(("ce_fwd", lambda: A.fp8mlp_ce_fwd(M, d, V, 1, x, Wt, tg, None, CE_CAP, lse, None, loss,
+                                                            ws)))
+            calls.append(("ce_bwd_dlogits", lambda: A.fp8mlp_ce_bwd_dlogits(M, d, V, 1, x, Wt, tg, None, CE_CAP,
+                                                                            lse, loss, None, A.CE_MEAN, dl)))
+        # dX = dlogits . W is the same contraction as the MLP's dX = dPre . W1
+        calls.append(("dx", lambda: A.fp8mlp_bwd_dx(M, d, V, dl, Wt, dX)))
+        calls.append(("dw", lambda: A.fp8mlp_linear_bwd(M, d, V, x, Wt, dl, None, dW)))
+        if fp8:
+            calls.append(("w_cache", lambda: A.fp8mlp_weight_fp8_cache_refresh(V, d, Wt, Wq, winv, wsw)))
+        return calls
+
+    calls = make_calls(x, tg, dX, loss)
     names = [n for n, _ in calls]
     n_ev = len(calls) + 1
 
@@ -929,45 +958,40 @@ def run_ce(a, W, world, rank, local_rank):
     e2e = None
     if not a.no_e2e:
         # the same step through the public API with host buffers: x and the
-        # targets come in from pinned host memory, the loss and dX go back
+        # targets come in from pinned host memory, the loss and dX go back,
+        # every step; the copies overlap the neighbouring steps' compute
+        # (two buffer sets, hostio.HostPipeline)
+        from fp8_relu_mlp_b200.hostio import HostPipeline
         xh = torch.from_numpy(H["x"].view(np.int16)).view(bf).pin_memory()
         th = torch.from_numpy(H["targets"]).pin_memory()
         lh = torch.empty(3, dtype=f32).pin_memory()
         dxh = torch.empty(M, d, dtype=bf).pin_memory()
+        sets = [dict(x=x, tg=tg, dX=dX, loss=loss),
+                dict(x=x.clone(), tg=tg.clone(), dX=torch.empty_like(dX), loss=torch.zeros_like(loss))]
+        set_calls = [make_calls(**sb) for sb in sets]
 
-        def body():
-            x.copy_(xh, non_blocking=True)
-            tg.copy_(th, non_blocking=True)
-            step()
-            lh.copy_(loss, non_blocking=True)
-            dxh.copy_(dX, non_blocking=True)
+        def set_step(k):
+            for _, f in set_calls[k]:
+                f()
 
-        body()
-        torch.cuda.synchronize()
-        ge = None
-        if not a.eager:
-            ge = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(ge):
-                body()
-        for _ in range(max(a.warmup, 3)):
-            ge.replay() if ge is not None else body()
+        pipe = HostPipeline(set_step, [[sb["x"], sb["tg"]] for sb in sets], [[sb["loss"], sb["dX"]] for sb in sets],
+                            device=dev, graph=not a.eager)
+        pipe.run([xh, th], [lh, dxh], max(a.warmup, 3))
         torch.cuda.synchronize()
         if dist:
             dist.barrier()
-        e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
-        e0.record()
-        for _ in range(a.steps):
-            ge.replay() if ge is not None else body()
-        e1.record()
-        e1.synchronize()
-        te = e0.elapsed_time(e1) * 1e-3
+        timer = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        pipe.run([xh, th], [lh, dxh], a.steps, timer)
+        timer[1].synchronize()
+        te = timer[0].elapsed_time(timer[1]) * 1e-3
         if dist:
             tt = torch.tensor([te], device=dev, dtype=torch.float64)
             dist.all_reduce(tt, op=dist.ReduceOp.MAX)
             te = float(tt.item())
         e2e = {"value": M * world * a.steps / te, "unit": "tokens/s",
                "h2d_bytes_per_step": int(xh.numel() * 2 + th.numel() * 4),
-               "d2h_bytes_per_step": int(lh.numel() * 4 + dxh.numel() * 2)}
+               "d2h_bytes_per_step": int(lh.numel() * 4 + dxh.numel() * 2),
+               "overlap": "copies on two streams beside the compute, double-buffered device sets"}
     if rank == 0:
         line = {
             "metric": CE_METRIC, "value": M * world * a.steps / total_s, "unit": "tokens/s", "n_gpus": world,
