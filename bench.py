@@ -392,11 +392,11 @@ def run_ours(a, W, world, rank, local_rank):
         mark(1)
         A.fp8mlp_down_proj_fp8(M, d, h, blk.post_fp8, blk.W2q_t, blk.w2_scale_inv, blk.state, blk.out)
         mark(2)
-        A.fp8mlp_bwd_dpre(M, d, h, blk.dOut, blk.W2, blk.post, blk.dPre)
+        A.fp8mlp_bwd_dpre(M, d, h, blk.dOut, blk.W2, blk.post, blk.dPre, A.LAUNCH_OVERLAP_PREVIOUS)
         mark(3)
         A.fp8mlp_bwd_dx(M, d, h, blk.dPre, blk.W1, blk.dX)
         mark(4)
-        A.fp8mlp_bwd_dw(M, d, h, blk.x, blk.dPre, blk.post, blk.dOut, blk.dW1, blk.dW2)
+        A.fp8mlp_bwd_dw(M, d, h, blk.x, blk.dPre, blk.post, blk.dOut, blk.dW1, blk.dW2, A.LAUNCH_OVERLAP_PREVIOUS)
         mark(5)
         blk.update_scale()
         mark(6)

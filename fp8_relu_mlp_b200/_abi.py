@@ -35,6 +35,7 @@ FWD_EVAL_BF16 = 1
 FWD_CALIBRATE = 2
 CE_SUM = 0
 CE_MEAN = 1
+LAUNCH_OVERLAP_PREVIOUS = 1
 DEBUG_STALL_PRODUCER = 1
 E4M3_MAX = 448.0
 
@@ -59,7 +60,7 @@ _SIGS = {
     "fp8mlp_amax_reduce_update_scale": [_p, _i, _p, _p],
     "fp8mlp_w2_fp8_cache_refresh": [_i, _i, _p, _p, _p, _p, _p],
     "fp8mlp_w2_fp8_cache_refresh_noalloc": [_i, _i, _p, _p, _p, _p],
-    "fp8mlp_bwd_dpre": [_i, _i, _i, _p, _p, _p, _p, _p],
+    "fp8mlp_bwd_dpre": [_i, _i, _i, _p, _p, _p, _p, _i, _p],
     "fp8mlp_quantize_x": [_i, _i, _p, _p, _p, _p, _p],
     "fp8mlp_x_partial_amax_count": [_i, _i],
     "fp8mlp_w1_fp8_cache_refresh": [_i, _i, _p, _p, _p, _p, _p],
@@ -72,7 +73,7 @@ _SIGS = {
     "fp8mlp_ce_bwd_dlogits": [_i, _i, _i, _i, _p, _p, _p, _p, _f, _p, _p, _p, _i, _p, _p],
     "fp8mlp_ce_bwd_dlogits_fp8": [_i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _f, _p, _p, _p, _i, _p, _p],
     "fp8mlp_bwd_dx": [_i, _i, _i, _p, _p, _p, _p],
-    "fp8mlp_bwd_dw": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p],
+    "fp8mlp_bwd_dw": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _i, _p],
     "fp8mlp_mlp_bwd": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p],
     "fp8mlp_rmsnorm_fwd": [_i, _i, _p, _p, _p, _p],
     "fp8mlp_rmsnorm_bwd": [_i, _i, _p, _p, _p, _p, _p, _p],
@@ -276,17 +277,17 @@ def fp8mlp_ce_bwd_dlogits_fp8(M, d, V, T, x_fp8, st_x, Wq, w_scale_inv, targets,
                  reduction, _ptr(dlogits), _stream(stream))
 
 
-def fp8mlp_bwd_dpre(M, d, h, dOut, W2, post, dPre, stream=None):
-    return _call("fp8mlp_bwd_dpre", M, d, h, _ptr(dOut), _ptr(W2), _ptr(post), _ptr(dPre), _stream(stream))
+def fp8mlp_bwd_dpre(M, d, h, dOut, W2, post, dPre, flags=0, stream=None):
+    return _call("fp8mlp_bwd_dpre", M, d, h, _ptr(dOut), _ptr(W2), _ptr(post), _ptr(dPre), flags, _stream(stream))
 
 
 def fp8mlp_bwd_dx(M, d, h, dPre, W1, dX, stream=None):
     return _call("fp8mlp_bwd_dx", M, d, h, _ptr(dPre), _ptr(W1), _ptr(dX), _stream(stream))
 
 
-def fp8mlp_bwd_dw(M, d, h, x, dPre, post, dOut, dW1, dW2, stream=None):
+def fp8mlp_bwd_dw(M, d, h, x, dPre, post, dOut, dW1, dW2, flags=0, stream=None):
     return _call("fp8mlp_bwd_dw", M, d, h, _ptr(x), _ptr(dPre), _ptr(post), _ptr(dOut), _ptr(dW1), _ptr(dW2),
-                 _stream(stream))
+                 flags, _stream(stream))
 
 
 def fp8mlp_mlp_bwd(M, d, h, x, W1, W2, post, dOut, dPre, dX, dW1, dW2, stream=None):

@@ -127,8 +127,10 @@ class MLPBlock:
         current W2: call this after the optimizer's update) runs on ``side``
         beside the up-projection, which does not read the cache, and is joined
         before the down-projection; the delayed-scale update runs on ``side``
-        beside the backward GEMMs, which do not read the scale, and is joined
-        at the end.  The calls and their results are those of
+        beside the dX and dW GEMMs, which do not read the scale, and is joined
+        at the end.  dPre and dW are launched with
+        ``LAUNCH_OVERLAP_PREVIOUS`` (each reads nothing the GEMM before it
+        writes).  The calls and their results are those of
         ``refresh_w2_cache(); train_step()``.  With the FP8 up-projection the
         W1 cache refresh (the same workspace) stays on the main stream, first.
         ``mark(i)``, if given, is called on the main stream at 0 (start), after
@@ -156,17 +158,20 @@ class MLPBlock:
         A.fp8mlp_down_proj_fp8(M, d, h, self.post_fp8, self.W2q_t, self.w2_scale_inv, self.state, self.out,
                                self.stream)
         mark(2)
+        # dPre does not read the down-projection's output: it may start while
+        # that GEMM finishes its last wave (likewise dW after dX)
+        A.fp8mlp_bwd_dpre(M, d, h, self.dOut, self.W2, self.post, self.dPre, A.LAUNCH_OVERLAP_PREVIOUS, self.stream)
+        mark(3)
         side.wait_stream(main)
         with torch.cuda.stream(side):
             A.fp8mlp_amax_reduce_update_scale(self.partial_amax, self.partial_amax.numel(), self.state, side)
             if self.fp8_up:
                 A.fp8mlp_amax_reduce_update_scale(self.partial_amax_x, A.fp8mlp_x_partial_amax_count(M, d),
                                                   self.state_x, side)
-        A.fp8mlp_bwd_dpre(M, d, h, self.dOut, self.W2, self.post, self.dPre, self.stream)
-        mark(3)
         A.fp8mlp_bwd_dx(M, d, h, self.dPre, self.W1, self.dX, self.stream)
         mark(4)
-        A.fp8mlp_bwd_dw(M, d, h, self.x, self.dPre, self.post, self.dOut, self.dW1, self.dW2, self.stream)
+        A.fp8mlp_bwd_dw(M, d, h, self.x, self.dPre, self.post, self.dOut, self.dW1, self.dW2,
+                        A.LAUNCH_OVERLAP_PREVIOUS, self.stream)
         mark(5)
         main.wait_stream(side)
         mark(7)

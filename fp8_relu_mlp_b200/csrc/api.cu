@@ -37,6 +37,11 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
     if (!aligned16(p)) return fail(FP8MLP_ERR_INVALID_ARG, #p " is not 16-byte aligned"); \
   } while (0)
 
+int check_launch_flags(int flags) {
+  if (flags & ~FP8MLP_LAUNCH_OVERLAP_PREVIOUS) return fail(FP8MLP_ERR_INVALID_ARG, "unknown launch flags");
+  return FP8MLP_OK;
+}
+
 int check_dims(int M, int d, int h) {
   if (M < 0) return fail(FP8MLP_ERR_INVALID_ARG, "M < 0");
   if (d < 16 || h < 16) return fail(FP8MLP_ERR_UNSUPPORTED_SHAPE, "d and h must be >= 16");
@@ -646,9 +651,10 @@ int fp8mlp_ce_bwd_dlogits_fp8(int M, int d, int V, int T, const uint8_t* x_fp8, 
 }
 
 int fp8mlp_bwd_dpre(int M, int d, int h, const uint16_t* dOut, const uint16_t* W2, const uint16_t* post,
-                    uint16_t* dPre, fp8mlp_stream_t stream) {
+                    uint16_t* dPre, int flags, fp8mlp_stream_t stream) {
   g_detail.clear();
   TRY(check_dims(M, d, h));
+  TRY(check_launch_flags(flags));
   if (M == 0) return FP8MLP_OK;
   REQUIRE_PTR(dOut);
   REQUIRE_PTR(W2);
@@ -662,6 +668,7 @@ int fp8mlp_bwd_dpre(int M, int d, int h, const uint16_t* dOut, const uint16_t* W
   TRY(map_tile32(&p.tmOut[0], dPre, BF16, 2, M, h, "dPre"));
   TRY(map_tile32(&p.tmAux, post, BF16, 2, M, h, "post"));
   fill_common(p, GemmKind::DPre, di, M, h, d, 1);
+  p.launch_flags = flags;
   return launch(GemmKind::DPre, p, di, stream, "bwd_dpre launch");
 }
 
@@ -684,9 +691,10 @@ int fp8mlp_bwd_dx(int M, int d, int h, const uint16_t* dPre, const uint16_t* W1,
 }
 
 int fp8mlp_bwd_dw(int M, int d, int h, const uint16_t* x, const uint16_t* dPre, const uint16_t* post,
-                  const uint16_t* dOut, float* dW1, float* dW2, fp8mlp_stream_t stream) {
+                  const uint16_t* dOut, float* dW1, float* dW2, int flags, fp8mlp_stream_t stream) {
   g_detail.clear();
   TRY(check_dims(M, d, h));
+  TRY(check_launch_flags(flags));
   REQUIRE_PTR(dW1);
   REQUIRE_PTR(dW2);
   if (M == 0) {
@@ -712,6 +720,7 @@ int fp8mlp_bwd_dw(int M, int d, int h, const uint16_t* x, const uint16_t* dPre, 
   TRY(map_mnmajor(&p.tmB[1], dOut, M, d, "dOut"));
   TRY(map_tile32(&p.tmOut[1], dW2, F32, 4, h, d, "dW2"));
   fill_common(p, GemmKind::DW, di, h, d, M, 2);
+  p.launch_flags = flags;
   return launch(GemmKind::DW, p, di, stream, "bwd_dw launch");
 }
 
@@ -731,9 +740,12 @@ int fp8mlp_mlp_bwd(int M, int d, int h, const uint16_t* x, const uint16_t* W1, c
   }
   REQUIRE_PTR(dW1);
   REQUIRE_PTR(dW2);
-  TRY(fp8mlp_bwd_dpre(M, d, h, dOut, W2, post, dPre, stream));
+  TRY(fp8mlp_bwd_dpre(M, d, h, dOut, W2, post, dPre, 0, stream));
   TRY(fp8mlp_bwd_dx(M, d, h, dPre, W1, dX, stream));
-  return fp8mlp_bwd_dw(M, d, h, x, dPre, post, dOut, dW1, dW2, stream);
+  // dW reads nothing dX writes and writes nothing dX reads: it may start
+  // while the dX GEMM finishes its last wave
+  return fp8mlp_bwd_dw(M, d, h, x, dPre, post, dOut, dW1, dW2, M > 0 ? FP8MLP_LAUNCH_OVERLAP_PREVIOUS : 0,
+                       stream);
 }
 
 int fp8mlp_rmsnorm_fwd(int M, int d, const uint16_t* r, uint16_t* x, float* rstd, fp8mlp_stream_t stream) {

@@ -56,6 +56,7 @@ struct alignas(64) GemmParams {
   unsigned int* status;
   unsigned long long timeout_ns;
   int debug_flags;
+  int launch_flags;  // FP8MLP_LAUNCH_OVERLAP_PREVIOUS: wait for the previous grid only before finishing
   // softcapped cross-entropy (CeFwd / CeBwd); the logits are y = acc (BF16
   // inputs) or acc * s_x^-1 * s_w^-1 (e4m3 inputs, scales in st_in / w_in_scale_inv)
   int ce_T;                  // targets per row (1..4)
@@ -242,9 +243,20 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   // the set-up above overlaps the previous kernel's tail; from here on global
-  // memory is read and written
-  pdl_wait();
-  if (threadIdx.x == 0) pdl_launch_dependents();
+  // memory is read and written.  Every kernel of the library waits for its
+  // predecessor before it lets its dependents launch, so when this grid
+  // starts the grid two launches back has completed; a launch that reads and
+  // writes nothing the previous grid writes or reads (the caller says so
+  // with FP8MLP_LAUNCH_OVERLAP_PREVIOUS) can therefore run its tiles while
+  // that grid drains, and waits for it only before finishing (so that
+  // whatever waits for this grid also sees the previous one complete).  Such
+  // a grid lets its own dependents launch only after that wait, which keeps
+  // the two-launches-back guarantee for the next launch.
+  const bool late_wait = (p.launch_flags & FP8MLP_LAUNCH_OVERLAP_PREVIOUS) != 0;
+  if (!late_wait) {
+    pdl_wait();
+    if (threadIdx.x == 0) pdl_launch_dependents();
+  }
   const WaitCtx w{p.status, abort_flag, p.timeout_ns};
 
   const int tiles_per_group = p.tiles_m * p.tiles_n;
@@ -713,6 +725,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
   }
 
   __syncwarp();
+  if (late_wait && threadIdx.x == 0) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
   __syncthreads();
   // no CTA of a pair leaves while its peer may still read its shared memory
   // or arrive on its barriers; TMEM is freed by both CTAs together

@@ -69,7 +69,8 @@ class DataParallelStep:
         mark(0)
         A.fp8mlp_up_proj_fused(M, d, h, b.x, b.W1, b.state, b.post, b.post_fp8, b.partial_amax)
         A.fp8mlp_down_proj_fp8(M, d, h, b.post_fp8, b.W2q_t, b.w2_scale_inv, b.state, b.out)
-        A.fp8mlp_bwd_dpre(M, d, h, b.dOut, b.W2, b.post, b.dPre)
+        # dPre does not read the down-projection's output (it may overlap its tail)
+        A.fp8mlp_bwd_dpre(M, d, h, b.dOut, b.W2, b.post, b.dPre, A.LAUNCH_OVERLAP_PREVIOUS)
         mark(1)
         A.fp8mlp_bwd_dw(M, d, h, b.x, b.dPre, b.post, b.dOut, b.dW1, b.dW2)
         mark(2)

@@ -349,23 +349,40 @@ size_t fp8mlp_workspace_size(int M, int d, int h);
  * "A Retrospective on Our World Records": BF16 backward from the BF16 post)
  * ------------------------------------------------------------------------ */
 
+/* Launch flag of fp8mlp_bwd_dpre and fp8mlp_bwd_dw (no counterpart on the
+ * pages; a scheduling hint).  The caller asserts that the kernel enqueued
+ * immediately before this call on the same stream was launched by this
+ * library, and that this call reads nothing that kernel writes and writes
+ * nothing it reads or writes (e.g. dPre right after the FP8 down-projection,
+ * dW right after dX).  The GEMM then starts while that kernel finishes its
+ * last wave of tiles and waits for it only before completing, so work
+ * enqueued later still sees both complete.  (Every kernel of the library
+ * waits for its own predecessor before it lets the next kernel start -- a
+ * kernel launched with this flag lets it start only after that final wait --
+ * so the inputs produced two launches back are complete.)  With
+ * programmatic launch switched off, or when the previous kernel is not the
+ * library's, the flag changes nothing.  A false assertion is a data race. */
+#define FP8MLP_LAUNCH_OVERLAP_PREVIOUS 1
+
 /*
  * dPost = dOut . W2^T (fp32 accumulate);  relu(pre) rebuilt as sqrt(post):
  *   dPre[m,i] = bf16( fp32(2 * sqrt(post[m,i])) * dPost[m,i] )
  * sqrt is the hardware approximation (sqrt.approx.f32, about one fp32 ulp),
  * far below the BF16 rounding of dPre that follows.
  * dOut [M,d], W2 [h,d], post [M,h] -> dPre [M,h].
+ * flags: 0 or FP8MLP_LAUNCH_OVERLAP_PREVIOUS (see above).
  */
 int fp8mlp_bwd_dpre(int M, int d, int h, const uint16_t* dOut, const uint16_t* W2, const uint16_t* post,
-                    uint16_t* dPre, fp8mlp_stream_t stream);
+                    uint16_t* dPre, int flags, fp8mlp_stream_t stream);
 
 /* dX = bf16(dPre . W1):  dPre [M,h], W1 [h,d] -> dX [M,d]. */
 int fp8mlp_bwd_dx(int M, int d, int h, const uint16_t* dPre, const uint16_t* W1, uint16_t* dX,
                   fp8mlp_stream_t stream);
 
-/* dW1 = dPre^T . x and dW2 = post^T . dOut, fp32 [h,d] each, in one launch. */
+/* dW1 = dPre^T . x and dW2 = post^T . dOut, fp32 [h,d] each, in one launch.
+ * flags: 0 or FP8MLP_LAUNCH_OVERLAP_PREVIOUS (see above). */
 int fp8mlp_bwd_dw(int M, int d, int h, const uint16_t* x, const uint16_t* dPre, const uint16_t* post,
-                  const uint16_t* dOut, float* dW1, float* dW2, fp8mlp_stream_t stream);
+                  const uint16_t* dOut, float* dW1, float* dW2, int flags, fp8mlp_stream_t stream);
 
 /* Whole backward: fp8mlp_bwd_dpre, fp8mlp_bwd_dx, fp8mlp_bwd_dw. */
 int fp8mlp_mlp_bwd(int M, int d, int h, const uint16_t* x, const uint16_t* W1, const uint16_t* W2,

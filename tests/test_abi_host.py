@@ -52,7 +52,7 @@ def _rc(name, *args):
                                         (16, 64, 250, A.ERR_UNSUPPORTED_SHAPE), (16, 72, 0, A.ERR_UNSUPPORTED_SHAPE)])
 def test_shape_checks(M, d, h, code):
     assert _rc("fp8mlp_up_proj_fused", M, d, h, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, None) == code
-    assert _rc("fp8mlp_bwd_dpre", M, d, h, FAKE, FAKE, FAKE, FAKE, None) == code
+    assert _rc("fp8mlp_bwd_dpre", M, d, h, FAKE, FAKE, FAKE, FAKE, 0, None) == code
 
 
 def test_null_and_misaligned_pointers_rejected():
@@ -79,6 +79,11 @@ def test_flag_checks():
                A.FWD_EVAL_BF16 | A.FWD_CALIBRATE, None) == A.ERR_INVALID_ARG
     assert _rc("fp8mlp_set_debug_flags", 2) == A.ERR_INVALID_ARG
     assert _rc("fp8mlp_set_wait_timeout_ns", 0) == A.ERR_INVALID_ARG
+
+
+def test_launch_flag_checks():
+    assert _rc("fp8mlp_bwd_dpre", 16, 64, 256, FAKE, FAKE, FAKE, FAKE, 2, None) == A.ERR_INVALID_ARG
+    assert _rc("fp8mlp_bwd_dw", 16, 64, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, None) == A.ERR_INVALID_ARG
 
 
 def test_scale_state_init_checks():
