@@ -861,7 +861,8 @@ def run_ce(a, W, world, rank, local_rank):
                                                                             lse, loss, None, A.CE_MEAN, dl)))
         # dX = dlogits . W is the same contraction as the MLP's dX = dPre . W1
         calls.append(("dx", lambda: A.fp8mlp_bwd_dx(M, d, V, dl, Wt, dX)))
-        calls.append(("dw", lambda: A.fp8mlp_linear_bwd(M, d, V, x, Wt, dl, None, dW)))
+        # dW does not depend on dX: it may start while the dX GEMM drains
+        calls.append(("dw", lambda: A.fp8mlp_linear_bwd(M, d, V, x, Wt, dl, None, dW, A.LAUNCH_OVERLAP_PREVIOUS)))
         if fp8:
             calls.append(("w_cache", lambda: A.fp8mlp_weight_fp8_cache_refresh(V, d, Wt, Wq, winv, wsw)))
         return calls

@@ -67,7 +67,7 @@ _SIGS = {
     "fp8mlp_up_proj_fused_fp8": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _p],
     "fp8mlp_linear_fwd_fp8": [_i, _i, _i, _p, _p, _p, _p, _p, _p],
     "fp8mlp_weight_fp8_cache_refresh": [_i, _i, _p, _p, _p, _p, _p],
-    "fp8mlp_linear_bwd": [_i, _i, _i, _p, _p, _p, _p, _p, _p],
+    "fp8mlp_linear_bwd": [_i, _i, _i, _p, _p, _p, _p, _p, _i, _p],
     "fp8mlp_ce_fwd": [_i, _i, _i, _i, _p, _p, _p, _p, _f, _p, _p, _p, _p, _p],
     "fp8mlp_ce_fwd_fp8": [_i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _f, _p, _p, _p, _p, _p],
     "fp8mlp_ce_bwd_dlogits": [_i, _i, _i, _i, _p, _p, _p, _p, _f, _p, _p, _p, _i, _p, _p],
@@ -230,8 +230,9 @@ def fp8mlp_weight_fp8_cache_refresh(N, K, W, Wq, w_scale_inv, workspace, stream=
                  _stream(stream))
 
 
-def fp8mlp_linear_bwd(M, K, N, x, W, dY, dX, dW, stream=None):
-    return _call("fp8mlp_linear_bwd", M, K, N, _ptr(x), _ptr(W), _ptr(dY), _ptr(dX), _ptr(dW), _stream(stream))
+def fp8mlp_linear_bwd(M, K, N, x, W, dY, dX, dW, flags=0, stream=None):
+    return _call("fp8mlp_linear_bwd", M, K, N, _ptr(x), _ptr(W), _ptr(dY), _ptr(dX), _ptr(dW), flags,
+                 _stream(stream))
 
 
 def _host_floats(seq):

@@ -577,9 +577,10 @@ int fp8mlp_linear_fwd_fp8(int M, int K, int N, const uint8_t* x_fp8, const uint8
 }
 
 int fp8mlp_linear_bwd(int M, int K, int N, const uint16_t* x, const uint16_t* W, const uint16_t* dY, uint16_t* dX,
-                      float* dW, fp8mlp_stream_t stream) {
+                      float* dW, int flags, fp8mlp_stream_t stream) {
   g_detail.clear();
   TRY(check_dims(M, N, K));
+  TRY(check_launch_flags(flags));
   REQUIRE_PTR(dW);
   if (M == 0) {
     DeviceInfo* di = nullptr;
@@ -600,6 +601,7 @@ int fp8mlp_linear_bwd(int M, int K, int N, const uint16_t* x, const uint16_t* W,
     TRY(map_mnmajor(&p.tmB[0], W, N, K, "W"));
     TRY(map_tile32(&p.tmOut[0], dX, BF16, 2, M, K, "dX"));
     fill_common(p, GemmKind::Bf16MnB, di, M, K, N, 1);
+    p.launch_flags = flags;
     TRY(launch(GemmKind::Bf16MnB, p, di, stream, "linear_bwd dX launch"));
   }
   // dW[N,K] = dY^T . x: contraction over the M tokens, both operands MN-major
@@ -608,6 +610,8 @@ int fp8mlp_linear_bwd(int M, int K, int N, const uint16_t* x, const uint16_t* W,
   TRY(map_mnmajor(&p.tmB[0], x, M, K, "x"));
   TRY(map_tile32(&p.tmOut[0], dW, F32, 4, N, K, "dW"));
   fill_common(p, GemmKind::DW, di, N, K, M, 1);
+  // dW neither reads dX nor writes what dX reads: it may overlap its tail
+  p.launch_flags = dX != nullptr ? FP8MLP_LAUNCH_OVERLAP_PREVIOUS : flags;
   return launch(GemmKind::DW, p, di, stream, "linear_bwd dW launch");
 }
 

@@ -209,9 +209,13 @@ int fp8mlp_weight_fp8_cache_refresh(int N, int K, const uint16_t* W, uint8_t* Wq
                                     void* workspace, fp8mlp_stream_t stream);
 
 /* BF16 backward of the linear layer: dX = bf16(dY . W) [M,K] (skipped when
- * dX is NULL) and dW = fp32(dY^T . x) [N,K].  x [M,K], W [N,K], dY [M,N]. */
+ * dX is NULL) and dW = fp32(dY^T . x) [N,K].  x [M,K], W [N,K], dY [M,N].
+ * The dW GEMM, which does not depend on dX, starts while the dX GEMM
+ * finishes.  flags: 0, or FP8MLP_LAUNCH_OVERLAP_PREVIOUS for the first GEMM
+ * launched (dX, or dW when dX is NULL), with the meaning given at
+ * fp8mlp_bwd_dpre. */
 int fp8mlp_linear_bwd(int M, int K, int N, const uint16_t* x, const uint16_t* W, const uint16_t* dY, uint16_t* dX,
-                      float* dW, fp8mlp_stream_t stream);
+                      float* dW, int flags, fp8mlp_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Softcapped cross-entropy over a language-model head, without [M,V] logits.
@@ -266,7 +270,7 @@ int fp8mlp_ce_fwd_fp8(int M, int d, int V, int T, const uint8_t* x_fp8, const fp
  * W_m = sum of row m's valid weights; g = dloss[0] (NULL: 1), divided by
  * loss[1] when reduction is FP8MLP_CE_MEAN (0 when loss[1] is 0).  lse and
  * loss from the forward; dlogits [M,V] bf16.  The BF16 backward through the
- * head is then fp8mlp_linear_bwd(M, d, V, x, W, dlogits, dX, dW). */
+ * head is then fp8mlp_linear_bwd(M, d, V, x, W, dlogits, dX, dW, 0, stream). */
 int fp8mlp_ce_bwd_dlogits(int M, int d, int V, int T, const uint16_t* x, const uint16_t* W, const int32_t* targets,
                           const float* target_weights, float softcap, const float* lse, const float* loss,
                           const float* dloss, int reduction, uint16_t* dlogits, fp8mlp_stream_t stream);
