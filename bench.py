@@ -202,7 +202,7 @@ def load_traffic(workload):
 # oracle on the host cores
 # ---------------------------------------------------------------------------
 
-def oracle_step_timer(W, tokens, seed=0):
+def oracle_step_timer(W, tokens, seed=0, fp8_up=False):
     """Returns (fn running one oracle step on `tokens` tokens of the workload,
     threads used)."""
     import numpy as np
@@ -251,15 +251,23 @@ def oracle_step_timer(W, tokens, seed=0):
         r0 = synth.to_bf16_bits(synth.make_x(g, tokens, W.d, "normal"))
         dtop = synth.to_bf16_bits(synth.make_x(g, tokens, W.d, "normal"))
         Ps = [synth.make_problem(1, W.d, W.h, seed=l) for l in range(W.layers)]
-        st = {"s": [ref.scale_state_init(W.margin, 1.0) for _ in range(W.layers)]}
+        st = {"s": [ref.scale_state_init(W.margin, 1.0) for _ in range(W.layers)],
+              "x": [ref.scale_state_init(W.margin, 1.0) for _ in range(W.layers)]}
 
         def step():
             layers = []
             for P in Ps:
                 W2q_t, s_w, s_wi = ref.w2_cache(P["W2"])
                 layers.append(dict(W1=P["W1"], W2=P["W2"], W2q_t=W2q_t, w2_scale_inv=s_wi))
+                if fp8_up:
+                    layers[-1]["W1q"], _, layers[-1]["w1_scale_inv"] = ref.w1_cache(P["W1"])
             scales = [(x["scale"], x["scale_inv"]) for x in st["s"]]
-            saved, _ = ref.stack_forward(r0, layers, scales)
+            if fp8_up:
+                saved, _ = ref.stack_forward_fp8up(r0, layers, scales,
+                                                   [(x["scale"], x["scale_inv"]) for x in st["x"]])
+                st["x"] = [ref.scale_update(x, sv["x_amax"]) for x, sv in zip(st["x"], saved)]
+            else:
+                saved, _ = ref.stack_forward(r0, layers, scales)
             ref.stack_backward(saved, layers, dtop)
             st["s"] = [ref.scale_update(x, sv["amax"]) for x, sv in zip(st["s"], saved)]
             return np
@@ -293,9 +301,9 @@ def metric_of(W):
     return METRIC
 
 
-def cpu_baseline(W, seconds, tokens=None):
+def cpu_baseline(W, seconds, tokens=None, fp8_up=False):
     tokens = tokens or oracle_tokens(W, "baseline")
-    step, threads = oracle_step_timer(W, tokens)
+    step, threads = oracle_step_timer(W, tokens, fp8_up=fp8_up)
     t0 = time.perf_counter()
     reps = 0
     while True:
@@ -1046,7 +1054,7 @@ def run_stack(a, W, world, rank, local_rank):
     L, M, d, h = W.layers, W.M, W.d, W.h
     peaks = load_peaks()
     fp8_peak, fp8_src = measure_fp8_peak(torch, peaks["bf16_tflops"])
-    S = MLPStack(L, M, d, h, device=dev, margin=W.margin)
+    S = MLPStack(L, M, d, h, device=dev, margin=W.margin, fp8_up=a.fp8_up)
     g = synth.rng(1000 + rank)
     r0 = synth.to_bf16_bits(synth.make_x(g, M, d, "normal"))
     dtop = synth.to_bf16_bits(synth.make_x(g, M, d, "normal"))
@@ -1125,6 +1133,13 @@ def run_stack(a, W, world, rank, local_rank):
     # write x), residual add (read r, out; write r'), RMSNorm bwd (read r, dX,
     # dr; write dr) and the dr copy
     norm_bytes = (2 + 3 + 4) * 2 * M * d
+    if a.fp8_up:
+        # e4m3 up-projection (x and W1 copies); the RMSNorm also writes x's
+        # copy; the W1 cache is refreshed every step
+        F = 2 * M * d * h
+        work["up_fused"] = dict(bf16=0, fp8=F, bytes=M * d + h * d + 3 * M * h)
+        work["w2_cache"]["bytes"] += 2 * (2 * h * d) + h * d
+        norm_bytes += M * d
     roof_t = 0.0
     for n, w in work.items():
         roof_t += max(w["bf16"] / (peaks["bf16_tflops"] * 1e12) + w["fp8"] / (fp8_peak * 1e12),
@@ -1175,7 +1190,9 @@ def run_stack(a, W, world, rank, local_rank):
             "warmup": a.warmup, "ms_per_step": total_s / a.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16+e4m3 (fp32 accumulate)",
             "data": "synthetic (seeded; 9-layer 768-dim ReLU^2 stack of the nanochat runs)",
-            "config": dict(config_of(W), layers=L, parallelism=f"dp{world} replicas" if world > 1 else "single GPU"),
+            "config": dict(config_of(W), layers=L, parallelism=f"dp{world} replicas" if world > 1 else "single GPU",
+                           up_projection="e4m3 (x quantised in the RMSNorm kernel, W1 cache in the step)"
+                           if a.fp8_up else "bf16"),
             "roofline": {"bound": "tensor", "kernel": "bwd_dw (top layer)", "achieved": achieved,
                          "peak": peak_sus, "unit": "TFLOP/s", "frac": achieved / peak_sus,
                          "traffic": traffic,
@@ -1190,7 +1207,7 @@ def run_stack(a, W, world, rank, local_rank):
         if e2e:
             line["e2e"] = e2e
         if not a.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(W, a.cpu_seconds)
+            line["cpu_baseline"] = cpu_baseline(W, a.cpu_seconds, fp8_up=a.fp8_up)
         print(json.dumps(line), flush=True)
     if dist:
         del graph

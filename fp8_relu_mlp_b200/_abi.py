@@ -76,6 +76,7 @@ _SIGS = {
     "fp8mlp_bwd_dw": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _i, _p],
     "fp8mlp_mlp_bwd": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p],
     "fp8mlp_rmsnorm_fwd": [_i, _i, _p, _p, _p, _p],
+    "fp8mlp_rmsnorm_fwd_quant": [_i, _i, _p, _p, _p, _p, _p, _p, _p],
     "fp8mlp_rmsnorm_bwd": [_i, _i, _p, _p, _p, _p, _p, _p],
     "fp8mlp_residual_add": [_i, _i, _p, _p, _p, _p],
     "fp8mlp_get_device_status": [_p, _p],
@@ -294,6 +295,11 @@ def fp8mlp_bwd_dw(M, d, h, x, dPre, post, dOut, dW1, dW2, flags=0, stream=None):
 def fp8mlp_mlp_bwd(M, d, h, x, W1, W2, post, dOut, dPre, dX, dW1, dW2, stream=None):
     return _call("fp8mlp_mlp_bwd", M, d, h, _ptr(x), _ptr(W1), _ptr(W2), _ptr(post), _ptr(dOut), _ptr(dPre),
                  _ptr(dX), _ptr(dW1), _ptr(dW2), _stream(stream))
+
+
+def fp8mlp_rmsnorm_fwd_quant(M, d, r, x, rstd, st_x, x_fp8, row_amax, stream=None):
+    return _call("fp8mlp_rmsnorm_fwd_quant", M, d, _ptr(r), _ptr(x), _ptr(rstd), _ptr(st_x), _ptr(x_fp8),
+                 _ptr(row_amax), _stream(stream))
 
 
 def fp8mlp_rmsnorm_fwd(M, d, r, x, rstd, stream=None):

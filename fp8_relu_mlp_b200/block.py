@@ -206,33 +206,72 @@ class MLPStack:
     768-dim ReLU^2 stacks of the nanochat runs), forward and backward, all
     through the C ABI.  Each layer keeps its own block buffers (post, x, its
     delayed-scale state and W2 cache); the residual stream r_l and the RMSNorm
-    statistics are kept per layer for the backward."""
+    statistics are kept per layer for the backward.
+
+    ``fp8_up``: every up-projection runs on e4m3 copies of x and W1; the
+    RMSNorm kernel writes x's copy under the layer's delayed x-scale and the
+    per-row max |x| that drives the next one (fp8mlp_rmsnorm_fwd_quant), so
+    x is read once.  The backward keeps the BF16 x and W1."""
 
     def __init__(self, L: int, M: int, d: int, h: int, device="cuda", margin: float = 2.0,
-                 initial_scale: float = 1.0, stream=None):
+                 initial_scale: float = 1.0, stream=None, fp8_up: bool = False):
         self.L, self.M, self.d, self.h = L, M, d, h
+        self.fp8_up = fp8_up
         self.device = torch.device(device)
         self.stream = stream
-        self.blocks = [MLPBlock(M, d, h, device, margin, initial_scale, stream=stream) for _ in range(L)]
+        self.blocks = [MLPBlock(M, d, h, device, margin, initial_scale, stream=stream, fp8_up=fp8_up)
+                       for _ in range(L)]
         self.r = [torch.zeros(M, d, dtype=torch.bfloat16, device=self.device) for _ in range(L + 1)]
         self.rstd = [torch.empty(M, dtype=torch.float32, device=self.device) for _ in range(L)]
         self.dr = torch.zeros(M, d, dtype=torch.bfloat16, device=self.device)
+        if fp8_up:
+            self.row_amax = [torch.zeros(max(M, 1), dtype=torch.float32, device=self.device) for _ in range(L)]
 
     def refresh_w2_caches(self):
+        """The FP8 weight caches from the current weights (after the optimizer):
+        W2 of every layer, and W1 with ``fp8_up``."""
         for b in self.blocks:
             b.refresh_w2_cache()
+            if self.fp8_up:
+                b.refresh_w1_cache()
+
+    def _norm(self, l):
+        b = self.blocks[l]
+        if self.fp8_up:
+            A.fp8mlp_rmsnorm_fwd_quant(self.M, self.d, self.r[l], b.x, self.rstd[l], b.state_x, b.x_fp8,
+                                       self.row_amax[l], self.stream)
+        else:
+            A.fp8mlp_rmsnorm_fwd(self.M, self.d, self.r[l], b.x, self.rstd[l], self.stream)
+
+    def _update_x_scale(self, l):
+        A.fp8mlp_amax_reduce_update_scale(self.row_amax[l], self.M, self.blocks[l].state_x, self.stream)
+
+    def _block_forward(self, b):
+        if self.fp8_up:
+            b._up_fp8(0)
+            A.fp8mlp_down_proj_fp8(self.M, self.d, self.h, b.post_fp8, b.W2q_t, b.w2_scale_inv, b.state, b.out,
+                                   self.stream)
+        else:
+            b.forward()
 
     def calibrate(self):
         for l, b in enumerate(self.blocks):
-            A.fp8mlp_rmsnorm_fwd(self.M, self.d, self.r[l], b.x, self.rstd[l], self.stream)
-            b.calibrate()
-            b.forward()
+            self._norm(l)
+            if self.fp8_up:
+                # first the x-scale from x's own amax, then post's scale
+                self._update_x_scale(l)
+                self._norm(l)
+                b._up_fp8(A.FWD_CALIBRATE)
+                A.fp8mlp_amax_reduce_update_scale(b.partial_amax, b.partial_amax.numel(), b.state, self.stream)
+            else:
+                b.calibrate()
+            self._block_forward(b)
             A.fp8mlp_residual_add(self.M, self.d, self.r[l], b.out, self.r[l + 1], self.stream)
 
     def forward(self):
         for l, b in enumerate(self.blocks):
-            A.fp8mlp_rmsnorm_fwd(self.M, self.d, self.r[l], b.x, self.rstd[l], self.stream)
-            b.forward()
+            self._norm(l)
+            self._block_forward(b)
             A.fp8mlp_residual_add(self.M, self.d, self.r[l], b.out, self.r[l + 1], self.stream)
 
     def backward(self):
@@ -244,5 +283,7 @@ class MLPStack:
             A.fp8mlp_rmsnorm_bwd(M, d, self.r[l], self.rstd[l], b.dX, self.dr, self.dr, self.stream)
 
     def update_scales(self):
-        for b in self.blocks:
-            b.update_scale()
+        for l, b in enumerate(self.blocks):
+            A.fp8mlp_amax_reduce_update_scale(b.partial_amax, b.partial_amax.numel(), b.state, self.stream)
+            if self.fp8_up:
+                self._update_x_scale(l)

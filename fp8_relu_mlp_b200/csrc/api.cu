@@ -752,6 +752,25 @@ int fp8mlp_mlp_bwd(int M, int d, int h, const uint16_t* x, const uint16_t* W1, c
                        stream);
 }
 
+int fp8mlp_rmsnorm_fwd_quant(int M, int d, const uint16_t* r, uint16_t* x, float* rstd,
+                             const fp8mlp_scale_state* st_x, uint8_t* x_fp8, float* row_amax,
+                             fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, d, 16));
+  if (M == 0) return FP8MLP_OK;
+  REQUIRE_PTR(r);
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(st_x);
+  REQUIRE_PTR(x_fp8);
+  if (rstd == nullptr || (reinterpret_cast<uintptr_t>(rstd) & 3u)) return fail(FP8MLP_ERR_INVALID_ARG, "rstd");
+  if (row_amax == nullptr || (reinterpret_cast<uintptr_t>(row_amax) & 3u))
+    return fail(FP8MLP_ERR_INVALID_ARG, "row_amax");
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  const cudaError_t e = launch_rmsnorm_fwd_quant(M, d, r, x, rstd, st_x, x_fp8, row_amax, di->num_sms, stream);
+  return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "rmsnorm_fwd_quant launch");
+}
+
 int fp8mlp_rmsnorm_fwd(int M, int d, const uint16_t* r, uint16_t* x, float* rstd, fp8mlp_stream_t stream) {
   g_detail.clear();
   TRY(check_dims(M, d, 16));

@@ -51,6 +51,9 @@ cudaError_t launch_w2_cache(int h, int d, const uint16_t* W2, uint8_t* W2q_t, fl
                             unsigned int* partial, unsigned int* status, int num_sms, cudaStream_t s);
 cudaError_t launch_rmsnorm_fwd(int M, int d, const uint16_t* r, uint16_t* x, float* rstd, int num_sms,
                                cudaStream_t s);
+cudaError_t launch_rmsnorm_fwd_quant(int M, int d, const uint16_t* r, uint16_t* x, float* rstd,
+                                     const fp8mlp_scale_state* st_x, uint8_t* x_fp8, float* row_amax, int num_sms,
+                                     cudaStream_t s);
 cudaError_t launch_rmsnorm_bwd(int M, int d, const uint16_t* r, const float* rstd, const uint16_t* dx,
                                const uint16_t* dr_in, uint16_t* dr_out, int num_sms, cudaStream_t s);
 cudaError_t launch_residual_add(int M, int d, const uint16_t* r, const uint16_t* out, uint16_t* r_next,

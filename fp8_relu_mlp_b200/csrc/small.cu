@@ -227,6 +227,64 @@ __global__ void rmsnorm_fwd_kernel(int M, int d, const uint16_t* __restrict__ r,
   }
 }
 
+// RMSNorm forward that also writes the e4m3 copy of x for an FP8
+// up-projection: x_fp8 = e4m3(fp32(x_bf16 * s_x)) under the delayed x-scale,
+// and row_amax[m] = max |x_bf16[m,:]| (the amax that drives the next scale).
+__global__ void rmsnorm_fwd_quant_kernel(int M, int d, const uint16_t* __restrict__ r, uint16_t* __restrict__ x,
+                                         float* __restrict__ rstd, const fp8mlp_scale_state* st_x,
+                                         uint2* __restrict__ xq, float* __restrict__ row_amax) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const float s = st_x->scale;
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  for (int row = blockIdx.x * warps + (threadIdx.x >> 5); row < M; row += gridDim.x * warps) {
+    const uint16_t* rr = r + static_cast<size_t>(row) * d;
+    float ss = 0.f;
+    for (int c = lane * 8; c < d; c += 256) {
+      const uint4 v = *reinterpret_cast<const uint4*>(rr + c);
+      const unsigned int w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float a = bf16lo_to_f32(w4[k]), b = bf16hi_to_f32(w4[k]);
+        ss = fmaf(a, a, ss);
+        ss = fmaf(b, b, ss);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rs = __fdiv_rn(1.f, __fsqrt_rn(__fdiv_rn(ss, static_cast<float>(d)) + 1e-6f));
+    if (lane == 0) rstd[row] = rs;
+    uint16_t* xr = x + static_cast<size_t>(row) * d;
+    uint2* qr = xq + static_cast<size_t>(row) * (d / 8);
+    unsigned int m = 0;  // max |x| as BF16 magnitude bits (integer order = value order)
+    for (int c = lane * 8; c < d; c += 256) {
+      const uint4 v = *reinterpret_cast<const uint4*>(rr + c);
+      const unsigned int w4[4] = {v.x, v.y, v.z, v.w};
+      unsigned int o4[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        o4[k] = pack_bf16x2(__fmul_rn(bf16lo_to_f32(w4[k]), rs), __fmul_rn(bf16hi_to_f32(w4[k]), rs));
+        m = max(m, o4[k] & 0x7FFFu);
+        m = max(m, (o4[k] >> 16) & 0x7FFFu);
+      }
+      *reinterpret_cast<uint4*>(xr + c) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+      uint32_t q[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const uint32_t a = pack_e4m3x2(__fmul_rn(bf16lo_to_f32(o4[2 * j]), s), __fmul_rn(bf16hi_to_f32(o4[2 * j]), s));
+        const uint32_t b = pack_e4m3x2(__fmul_rn(bf16lo_to_f32(o4[2 * j + 1]), s),
+                                       __fmul_rn(bf16hi_to_f32(o4[2 * j + 1]), s));
+        q[j] = a | (b << 16);
+      }
+      qr[c / 8] = make_uint2(q[0], q[1]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) row_amax[row] = __uint_as_float(m << 16);
+  }
+}
+
 __global__ void rmsnorm_bwd_kernel(int M, int d, const uint16_t* __restrict__ r, const float* __restrict__ rstd,
                                    const uint16_t* __restrict__ dx, const uint16_t* dr_in, uint16_t* dr_out) {
   pdl_wait();
@@ -425,6 +483,15 @@ cudaError_t launch_w1_cache(int h, int d, const uint16_t* W1, uint8_t* W1q, floa
   if (e != cudaSuccess) return e;
   e = launch_pdl(w1_quant_kernel, dim3(nparts), dim3(256), 0, s, n / 8, reinterpret_cast<const uint4*>(W1),
                  reinterpret_cast<uint2*>(W1q), w1_scale_inv, static_cast<const unsigned int*>(partial), nparts, status);
+  count_launches(1);
+  return e;
+}
+
+cudaError_t launch_rmsnorm_fwd_quant(int M, int d, const uint16_t* r, uint16_t* x, float* rstd,
+                                     const fp8mlp_scale_state* st_x, uint8_t* x_fp8, float* row_amax, int num_sms,
+                                     cudaStream_t s) {
+  const cudaError_t e = launch_pdl(rmsnorm_fwd_quant_kernel, dim3(grid_for(static_cast<size_t>(M), 8, num_sms, 8)),
+                                   dim3(256), 0, s, M, d, r, x, rstd, st_x, reinterpret_cast<uint2*>(x_fp8), row_amax);
   count_launches(1);
   return e;
 }

@@ -403,6 +403,18 @@ int fp8mlp_mlp_bwd(int M, int d, int h, const uint16_t* x, const uint16_t* W1, c
 /* x = bf16(r * rstd), rstd[m] = 1/sqrt(mean(r[m,:]^2) + 1e-6) (fp32). */
 int fp8mlp_rmsnorm_fwd(int M, int d, const uint16_t* r, uint16_t* x, float* rstd, fp8mlp_stream_t stream);
 
+/* RMSNorm forward fused with the x quantiser of the FP8 up-projection
+ * ("NanoGPT Speedrun (Track 1)", From Unoptimized, item 5: e4m3 MLP GEMMs in
+ * the training forward), so that x is read once: x and rstd as
+ * fp8mlp_rmsnorm_fwd, and
+ *   x_fp8[m,k] = e4m3_satfinite( fp32(x[m,k] * st_x->scale) )   (the BF16 x)
+ *   row_amax[m] = max_k |x[m,k]|                                (fp32, [M])
+ * -- the codes of fp8mlp_quantize_x on this x.  The next step's x-scale is
+ * fp8mlp_amax_reduce_update_scale(row_amax, M, st_x). */
+int fp8mlp_rmsnorm_fwd_quant(int M, int d, const uint16_t* r, uint16_t* x, float* rstd,
+                             const fp8mlp_scale_state* st_x, uint8_t* x_fp8, float* row_amax,
+                             fp8mlp_stream_t stream);
+
 /* dr_out = bf16( dr_in + rstd * (dx - xhat * mean(dx * xhat)) ), xhat = r * rstd.
  * dr_in may equal dr_out (in place). */
 int fp8mlp_rmsnorm_bwd(int M, int d, const uint16_t* r, const float* rstd, const uint16_t* dx,

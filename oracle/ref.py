@@ -412,6 +412,27 @@ def stack_forward(r0, layers, scales):
     return saved, r
 
 
+def stack_forward_fp8up(r0, layers, scales, x_scales):
+    """The stack with every up-projection on e4m3 copies ("NanoGPT Speedrun
+    (Track 1)", From Unoptimized, item 5): per layer x = rmsnorm(r),
+    x_q = e4m3(fp32(x s_x)) under the layer's delayed x-scale, pre from the
+    e4m3 up-projection against the W1 cache, then post, its FP8 copy and the
+    FP8 down-projection as in stack_forward.  layers: dicts with W1q and
+    w1_scale_inv as well; x_scales: list of (s_x, s_x_inv).  The saved dicts
+    also hold x_amax = max |x| (the next x-scale's amax); the backward is
+    stack_backward (BF16 x and W1)."""
+    r = r0
+    saved = []
+    for L, (s, si), (sx, sxi) in zip(layers, scales, x_scales):
+        xb, _ = rmsnorm_fwd(r)
+        xq, ax = quantise_x(xb, sx)
+        post = relu2_post(up_proj_fp8(xq, L["W1q"], sxi, L["w1_scale_inv"]))
+        out = down_proj_fp8(quantise_post(post, s), L["W2q_t"], si, L["w2_scale_inv"])
+        saved.append(dict(r=r, x=xb, post=post, amax=amax(post), x_amax=ax))
+        r = residual_add(r, out)
+    return saved, r
+
+
 def stack_backward(saved, layers, dr_top):
     """Backward through the stack; the residual gradient is carried as BF16.
     Returns (dr0 bits, list of (dW1, dW2))."""

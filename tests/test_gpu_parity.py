@@ -500,6 +500,83 @@ def test_rmsnorm_and_residual(M, d):
     assert x.intact() and rstd.intact() and dro.intact() and rn.intact()
 
 
+@pytest.mark.parametrize("M,d", [(300, 768), (1, 64), (1000, 1024)])
+def test_rmsnorm_fwd_quant(M, d):
+    g = np.random.default_rng(3 * M + d)
+    r = synth.to_bf16_bits(g.standard_normal((M, d)).astype(np.float32) * 3)
+    s_x = np.float32(448.0 / 9.0)
+    st = _state(2.0, float(s_x))
+    x, rstd = Guarded((M, d), torch.bfloat16), Guarded((M,), torch.float32)
+    xq, ra = Guarded((M, d), torch.uint8), Guarded((M,), torch.float32)
+    A.fp8mlp_rmsnorm_fwd_quant(M, d, dev_bf16(r), x.t, rstd.t, st, xq.t, ra.t)
+    x2, rstd2 = torch.empty(M, d, dtype=torch.bfloat16, device="cuda"), torch.empty(M, device="cuda")
+    A.fp8mlp_rmsnorm_fwd(M, d, dev_bf16(r), x2, rstd2)
+    torch.cuda.synchronize()
+    # x and rstd are those of the plain RMSNorm kernel
+    assert torch.equal(x.t, x2) and torch.equal(rstd.t, rstd2)
+    xg, qg = host_bits(x.t), host_bits(xq.t)
+    xo, _ = ref.rmsnorm_fwd(r)
+    qo, _ = ref.quantise_x(xo, s_x)
+    same = xg == xo
+    assert same.mean() > 0.9
+    assert np.array_equal(qg[same], qo[same])
+    # where the BF16 x is one step away from the oracle's, the code is at most
+    # one e4m3 step away (rounding is monotone)
+    signed = lambda c: (c & 0x7F).astype(np.int64) * np.where(c & 0x80, -1, 1)
+    assert (np.abs(signed(qg[~same]) - signed(qo[~same])) <= 1).all()
+    # the codes are RNE-satfinite e4m3 of the kernel's own x * s_x (torch's cast)
+    want = (x.t.float() * float(s_x)).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+    assert torch.equal(xq.t, want)
+    # per-row max |x| of the kernel's own x, exactly
+    assert torch.equal(ra.t, x.t.float().abs().amax(dim=1))
+    assert x.intact() and rstd.intact() and xq.intact() and ra.intact()
+
+
+@pytest.mark.parametrize("L,M,d,h", [(3, 300, 128, 512), (2, 1024, 768, 3072)])
+def test_stack_fp8_up_vs_oracle(L, M, d, h):
+    from fp8_relu_mlp_b200.block import MLPBlock, MLPStack
+    g = np.random.default_rng(L * 100 + M + 7)
+    r0 = synth.to_bf16_bits(g.standard_normal((M, d)).astype(np.float32))
+    dtop = synth.to_bf16_bits(g.standard_normal((M, d)).astype(np.float32))
+    layers, scales, xsc = [], [], []
+    S = MLPStack(L, M, d, h, fp8_up=True)
+    for l in range(L):
+        P = synth.make_problem(1, d, h, seed=600 + l)
+        W2q_t, _, s_wi = ref.w2_cache(P["W2"])
+        W1q, _, s1i = ref.w1_cache(P["W1"])
+        layers.append(dict(W1=P["W1"], W2=P["W2"], W2q_t=W2q_t, w2_scale_inv=s_wi, W1q=W1q, w1_scale_inv=s1i))
+        s = np.float32(30.0 + 5 * l)
+        sx = np.float32(448.0 / (9.0 + l))
+        scales.append((s, np.float32(np.float32(1) / s)))
+        xsc.append((sx, np.float32(np.float32(1) / sx)))
+        b = S.blocks[l]
+        b.W1.copy_(MLPBlock.bits_to_bf16(P["W1"], b.device))
+        b.W2.copy_(MLPBlock.bits_to_bf16(P["W2"], b.device))
+        A.fp8mlp_scale_state_init(b.state, 2.0, float(s))
+        A.fp8mlp_scale_state_init(b.state_x, 2.0, float(sx))
+    S.refresh_w2_caches()
+    S.r[0].copy_(MLPBlock.bits_to_bf16(r0, S.device))
+    S.forward()
+    S.dr.copy_(MLPBlock.bits_to_bf16(dtop, S.device))
+    S.backward()
+    torch.cuda.synchronize()
+    for l in range(L):
+        assert np.array_equal(host_bits(S.blocks[l].W1q), layers[l]["W1q"]), l
+    saved, rL = ref.stack_forward_fp8up(r0, layers, scales, xsc)
+    dr0, grads = ref.stack_backward(saved, layers, dtop)
+    assert rel_fro(ref.bf16_to_f64(host_bits(S.r[L])), ref.bf16_to_f64(rL)) < 2e-2
+    assert rel_fro(ref.bf16_to_f64(host_bits(S.dr)), ref.bf16_to_f64(dr0)) < 2e-2
+    for l in range(L):
+        assert rel_fro(host_bits(S.blocks[l].dW1), grads[l][0]) < 2e-2, l
+        assert rel_fro(host_bits(S.blocks[l].dW2), grads[l][1]) < 2e-2, l
+        # the x amax that drives the next x-scale: within one BF16 step
+        ga = float(host_bits(S.row_amax[l]).max())
+        assert abs(ga - float(saved[l]["x_amax"])) <= 2.0 ** -7 * float(saved[l]["x_amax"]), l
+    S.update_scales()
+    torch.cuda.synchronize()
+    assert A.fp8mlp_get_device_status() == 0
+
+
 # ---------------------------------------------------------------------------
 # a CUDA-graph replay of the step gives the same bits as the eager calls
 # ---------------------------------------------------------------------------

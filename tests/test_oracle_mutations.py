@@ -75,6 +75,9 @@ MUTATIONS = {
                            ["test_ce_bruteforce_with_ignored_targets", "test_ce_multi_target_is_sum_of_single_targets"]),
     "ce_out_of_range_target_clipped": ("_ce_targets", lambda orig: _ce_targets_clipped,
                                        ["test_ce_bruteforce_with_ignored_targets", "test_ce_zero_logits_closed_form"]),
+    "stack_fp8up_x_dequant_dropped": ("stack_forward_fp8up",
+                                      lambda orig: (lambda r0, ly, sc, xs: orig(r0, ly, sc, [(a, np.float32(1.0)) for a, _ in xs])),
+                                      ["test_stack_fp8up_close_to_bf16_stack"]),
     "ce_fp8_scale_dropped": ("head_logits_fp8", lambda orig: (lambda xq, Wq, a, b: orig(xq, Wq, 1.0, 1.0)),
                              ["test_ce_head_logits_fp8_bruteforce_and_exact_grid"]),
 }

@@ -704,3 +704,33 @@ def test_ce_backward_through_head_vs_torch_autograd():
     # dlogits is rounded to BF16 (relative error <= 2^-9 per element)
     assert _rel(ref.bf16_to_f64(dX), Xt.grad.numpy()) < 1e-2
     assert _rel(dW, Wt.grad.numpy()) < 1e-2
+
+
+def test_stack_fp8up_close_to_bf16_stack():
+    # the e4m3 up-projection perturbs each layer's pre by the e4m3 rounding
+    # of x and W1 (round to nearest: relative error uniform within 2^-4, RMS
+    # 2^-4/sqrt(3) per operand, so about 5% RMS on pre and twice that on
+    # post = pre^2); the residual stream carries r as well, so the two
+    # stacks stay within 10% of each other.  A missing or inverted
+    # dequantising scale (a factor 8 to 56 here), a transposed operand or a
+    # skipped layer would not
+    g = np.random.default_rng(71)
+    M, d, h, Lyr = 24, 32, 64, 3
+    r0 = _bf16(g.standard_normal((M, d)) * 2.0)
+    layers, scales, xs = [], [], []
+    for l in range(Lyr):
+        W1 = _bf16(g.standard_normal((h, d)) / np.sqrt(d))
+        W2 = _bf16(g.standard_normal((h, d)) / np.sqrt(h))
+        W2q_t, _, s_wi = ref.w2_cache(W2)
+        W1q, _, s1i = ref.w1_cache(W1)
+        layers.append(dict(W1=W1, W2=W2, W2q_t=W2q_t, w2_scale_inv=s_wi, W1q=W1q, w1_scale_inv=s1i))
+        scales.append((np.float32(448.0 / 40), np.float32(40 / 448.0)))
+        xs.append((np.float32(448.0 / 8), np.float32(8 / 448.0)))
+    sv8, r8 = ref.stack_forward_fp8up(r0, layers, scales, xs)
+    sv, r = ref.stack_forward(r0, layers, scales)
+    for l in range(Lyr):
+        d_out = ref.bf16_to_f64(sv8[l]["r"]) - ref.bf16_to_f64(sv[l]["r"])
+        assert _rel(ref.bf16_to_f64(sv8[l]["post"]), ref.bf16_to_f64(sv[l]["post"])) < 0.2
+        assert np.abs(d_out).max() <= 0.2 * np.abs(ref.bf16_to_f64(sv[l]["r"])).max()
+        assert sv8[l]["x_amax"] == np.float32(np.abs(ref.bf16_to_f64(sv8[l]["x"])).max())
+    assert _rel(ref.bf16_to_f64(r8), ref.bf16_to_f64(r)) < 0.1
