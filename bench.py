@@ -62,6 +62,9 @@ def parse():
                          "W2 cache refresh run on a second stream beside the GEMMs)")
     ap.add_argument("--fp8-up", action="store_true",
                     help="run the up-projection on e4m3 copies of x and W1 as well (x quantiser + W1 cache per step)")
+    ap.add_argument("--compare-library", action="store_true",
+                    help="time each GEMM of the step16k block against cuBLAS (torch.mm / torch._scaled_mm) on the "
+                         "same shapes, one launch at a time with L2 flushed, and print one JSON line")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's token count (small cases for profiling; not a bench line)")
     ap.add_argument("--bf16-head", action="store_true",
@@ -783,6 +786,70 @@ def run_linear(a, W, world, rank, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def run_compare_library(a, W):
+    """Each GEMM of the block next to cuBLAS on the same shapes and output
+    types (torch.mm; torch._scaled_mm for the e4m3 down-projection): a
+    reference for what a library GEMM with a plain store epilogue reaches at
+    these sizes.  One launch at a time, L2 flushed before each, median of 11."""
+    import numpy as np
+    import torch
+    from fp8_relu_mlp_b200 import _abi as A
+    from fp8_relu_mlp_b200 import synth
+    from fp8_relu_mlp_b200.block import MLPBlock
+    dev = torch.device("cuda", 0)
+    M, d, h = W.M, W.d, W.h
+    blk = MLPBlock(M, d, h, device=dev, margin=W.margin)
+    P = synth.make_problem(M, d, h, seed=0)
+    for k in ("x", "W1", "W2", "dOut"):
+        getattr(blk, k).copy_(MLPBlock.bits_to_bf16(P[k], dev))
+    blk.refresh_w2_cache()
+    blk.calibrate()
+    blk.forward()
+    blk.backward()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    one = torch.ones((), device=dev)
+    W2q = blk.W2q_t  # [d, h] e4m3, K-major: the second operand of q . W2q^T
+    ops = [
+        ("up_fused (post, e4m3 copy, partial amax)", 1,
+         lambda: A.fp8mlp_up_proj_fused(M, d, h, blk.x, blk.W1, blk.state, blk.post, blk.post_fp8,
+                                        blk.partial_amax)),
+        ("cuBLAS x . W1^T -> bf16 [M,h]", 1, lambda: torch.mm(blk.x, blk.W1.t())),
+        ("down_fp8 (e4m3, scaled epilogue)", 1,
+         lambda: A.fp8mlp_down_proj_fp8(M, d, h, blk.post_fp8, blk.W2q_t, blk.w2_scale_inv, blk.state, blk.out)),
+        ("cuBLAS e4m3 q . W2q^T -> bf16 [M,d] (torch._scaled_mm)", 1,
+         lambda: torch._scaled_mm(blk.post_fp8.view(torch.float8_e4m3fn), W2q.view(torch.float8_e4m3fn).t(),
+                                  scale_a=one, scale_b=one, out_dtype=torch.bfloat16)),
+        ("bwd_dpre (dPost GEMM + 2 sqrt(post) epilogue)", 1,
+         lambda: A.fp8mlp_bwd_dpre(M, d, h, blk.dOut, blk.W2, blk.post, blk.dPre)),
+        ("cuBLAS dOut . W2^T -> bf16 [M,h]", 1, lambda: torch.mm(blk.dOut, blk.W2.t())),
+        ("bwd_dx", 1, lambda: A.fp8mlp_bwd_dx(M, d, h, blk.dPre, blk.W1, blk.dX)),
+        ("cuBLAS dPre . W1 -> bf16 [M,d]", 1, lambda: torch.mm(blk.dPre, blk.W1)),
+        ("bwd_dw (dW1 and dW2, fp32, one launch)", 2,
+         lambda: A.fp8mlp_bwd_dw(M, d, h, blk.x, blk.dPre, blk.post, blk.dOut, blk.dW1, blk.dW2)),
+        ("cuBLAS dPre^T . x -> fp32 [h,d] (dW1 only)", 1,
+         lambda: torch.mm(blk.dPre.t(), blk.x, out_dtype=torch.float32)),
+    ]
+    F = 2 * M * d * h
+    res = []
+    for name, nF, f in ops:
+        for _ in range(3):
+            f()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(11):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        us = float(np.median(ts)) * 1e3
+        res.append({"gemm": name, "us": round(us, 1), "tflops": round(nF * F / us / 1e6, 1)})
+    print(json.dumps({"compare_library": res, "config": config_of(W), "clocks_note": "single launches, L2 flushed",
+                      "torch": torch.__version__}), flush=True)
+
+
 def ce_work(M, d, V, fp8):
     """FLOPs (by precision) and minimum HBM bytes of each call of a head step."""
     F = 2 * M * d * V
@@ -1262,6 +1329,10 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if a.impl == "reference":
         run_reference(a, W, world, rank)
+        return 0
+    if a.compare_library:
+        if rank == 0:
+            run_compare_library(a, W)
         return 0
     if W.name.startswith("qkv"):
         run_linear(a, W, world, rank, local_rank)
