@@ -61,7 +61,13 @@ cudaError_t launch_one(const GemmParams& p, int num_tiles, int num_sms, cudaStre
 
 }  // namespace
 
-int up_partial_cols() { return CfgUp::BN / CfgUp::EPI_SPLIT; }
+int up_partial_cols() {
+  // fp8mlp_partial_amax_shape serves both up-projections
+  static_assert(CfgUp::BN / CfgUp::EPI_SPLIT == CfgUpQ::BN / CfgUpQ::EPI_SPLIT &&
+                    CfgUp::TILE_M == CfgUpQ::TILE_M,
+                "the BF16 and e4m3 up-projections share one partial-amax layout");
+  return CfgUp::BN / CfgUp::EPI_SPLIT;
+}
 
 int ce_partial_cols() {
   static_assert(CfgCeF::BN / CfgCeF::EPI_SPLIT == CfgCeF8::BN / CfgCeF8::EPI_SPLIT, "same partial layout");
