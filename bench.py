@@ -69,6 +69,8 @@ def parse():
                     help="override the workload's token count (small cases for profiling; not a bench line)")
     ap.add_argument("--bf16-head", action="store_true",
                     help="ce16k: BF16 logits instead of the e4m3 LM head")
+    ap.add_argument("--shard-grads", action="store_true",
+                    help="with N>1, reduce-scatter dW1/dW2 (each rank keeps h/N rows) instead of all-reducing them")
     ap.add_argument("--replicas", action="store_true",
                     help="with N>1, run independent replicas (no partial-amax / dW all-reduce)")
     return ap.parse_args()
@@ -601,7 +603,7 @@ def run_dp(a, W, world, rank, local_rank, blk, flush, dist, peaks, fp8_peak, fp8
     from fp8_relu_mlp_b200 import _abi as A
     from fp8_relu_mlp_b200.dp import DataParallelStep
     M, d, h = W.M, W.d, W.h
-    stepper = DataParallelStep(blk)
+    stepper = DataParallelStep(blk, shard_grads=a.shard_grads)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     for _ in range(max(a.warmup, 3)):
         flush.zero_()
@@ -644,7 +646,8 @@ def run_dp(a, W, world, rank, local_rank, blk, flush, dist, peaks, fp8_peak, fp8
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16+e4m3 (fp32 accumulate)",
             "data": "synthetic (seeded; shapes of the 768-dim GPT-2-small / nanochat MLP)",
             "config": dict(config_of(W), parallelism=f"dp{world}: NCCL all-reduce of partial amax (MAX) "
-                                                     f"and dW1/dW2 (mean), overlapped with dX"),
+                                                     f"and {'reduce-scatter' if a.shard_grads else 'all-reduce'} "
+                                                     f"of dW1/dW2 (mean), overlapped with dX"),
             "roofline": {"bound": "tensor", "kernel": "bwd_dw", "achieved": achieved, "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
                          "traffic": load_traffic(W.name).get("bwd_dw"),

@@ -9,7 +9,9 @@ A training step then needs two exchanges:
   with data parallelism that amax is over all ranks' tokens);
 * dW1 and dW2 are all-reduced (summed, optionally averaged), the gradient
   exchange of data-parallel training that the pages' 8-GPU runs do in their
-  optimizer.
+  optimizer -- or reduce-scattered, so that each rank keeps the reduced rows
+  of its own shard (h/N rows of each), for an optimizer whose state is
+  sharded by rank; that moves half the bytes of an all-reduce.
 
 The dW exchange is issued on a side stream as soon as the dW GEMM is done and
 overlaps the dX GEMM, which does not depend on it.  These helpers only move
@@ -37,6 +39,19 @@ def allreduce_grads(dW1: torch.Tensor, dW2: torch.Tensor, group=None, average: b
             t.div_(world)
 
 
+def reduce_scatter_grads(dW1: torch.Tensor, dW2: torch.Tensor, shard1: torch.Tensor, shard2: torch.Tensor,
+                         group=None, average: bool = True):
+    """SUM (or mean) over ranks of dW1 and dW2 [h,d], of which this rank keeps
+    rows [r h/N, (r+1) h/N) in shard1 / shard2 [h/N, d]."""
+    world = dist.get_world_size(group)
+    for full, part in ((dW1, shard1), (dW2, shard2)):
+        if full.shape[0] % world != 0 or part.shape[0] * world != full.shape[0]:
+            raise ValueError("h must be a multiple of the world size, shards of h/N rows")
+        dist.reduce_scatter_tensor(part, full, op=dist.ReduceOp.SUM, group=group)
+        if average and world > 1:
+            part.div_(world)
+
+
 def max_over_ranks(x: float, device=None, group=None) -> float:
     """The maximum of a host scalar over all ranks (e.g. a timing)."""
     t = torch.tensor([float(x)], dtype=torch.float64, device=device)
@@ -53,11 +68,21 @@ class DataParallelStep:
     updates the delayed scale from the all-reduced amax and refreshes the W2
     cache (after the caller's optimizer update, in a real training loop)."""
 
-    def __init__(self, blk, group=None, average: bool = True):
+    def __init__(self, blk, group=None, average: bool = True, shard_grads: bool = False):
+        """``shard_grads``: reduce-scatter dW1/dW2 into ``self.dW1_shard`` /
+        ``self.dW2_shard`` ([h/N, d], this rank's rows) instead of
+        all-reducing the full tensors."""
         self.blk = blk
         self.group = group
         self.average = average
         self.side = torch.cuda.Stream(blk.device)
+        self.shard_grads = shard_grads
+        if shard_grads:
+            n = dist.get_world_size(group)
+            if blk.h % n != 0:
+                raise ValueError("h must be a multiple of the world size to shard the gradients")
+            self.dW1_shard = torch.empty(blk.h // n, blk.d, dtype=torch.float32, device=blk.device)
+            self.dW2_shard = torch.empty_like(self.dW1_shard)
 
     def __call__(self, refresh_w2: bool = True, mark=None):
         """``mark(i)``, if given, is called on the main stream at 0 (start),
@@ -77,7 +102,10 @@ class DataParallelStep:
         self.side.wait_stream(main)
         with torch.cuda.stream(self.side):
             allreduce_amax(b.partial_amax, self.group)
-            allreduce_grads(b.dW1, b.dW2, self.group, self.average)
+            if self.shard_grads:
+                reduce_scatter_grads(b.dW1, b.dW2, self.dW1_shard, self.dW2_shard, self.group, self.average)
+            else:
+                allreduce_grads(b.dW1, b.dW2, self.group, self.average)
         A.fp8mlp_bwd_dx(M, d, h, b.dPre, b.W1, b.dX)
         main.wait_stream(self.side)
         b.update_scale()

@@ -38,7 +38,13 @@ def _worker(rank, world, port, out_q):
         dW2 = torch.full((4, 3), float(10 * (rank + 1)))
         dp.allreduce_grads(dW1, dW2, average=True)
         t = dp.max_over_ranks(0.25 * (rank + 1))
-        out_q.put((rank, local_max, float(pa.max()), float(st["scale"]), dW1.numpy().copy(), dW2.numpy().copy(), t))
+        # reduce-scatter: rank r keeps rows [2r, 2r+2) of the mean over ranks
+        G1 = torch.arange(12, dtype=torch.float32).reshape(4, 3) * (rank + 1)
+        G2 = -G1
+        s1, s2 = torch.empty(2, 3), torch.empty(2, 3)
+        dp.reduce_scatter_grads(G1, G2, s1, s2, average=True)
+        out_q.put((rank, local_max, float(pa.max()), float(st["scale"]), dW1.numpy().copy(), dW2.numpy().copy(), t,
+                   s1.numpy().copy(), s2.numpy().copy()))
     finally:
         dist.destroy_process_group()
 
@@ -58,8 +64,10 @@ def test_two_rank_exchange():
         assert p.exitcode == 0
     res.sort()
     global_max = max(r[1] for r in res)
-    for rank, local_max, reduced_max, scale, dW1, dW2, t in res:
+    full = np.arange(12, dtype=np.float32).reshape(4, 3) * 1.5   # mean of x1 and x2
+    for rank, local_max, reduced_max, scale, dW1, dW2, t, s1, s2 in res:
         assert reduced_max == global_max           # every rank sees the global amax
         assert np.all(dW1 == 1.5) and np.all(dW2 == 15.0)   # mean over ranks
         assert t == 0.5                             # max over ranks
+        assert np.array_equal(s1, full[2 * rank:2 * rank + 2]) and np.array_equal(s2, -full[2 * rank:2 * rank + 2])
     assert res[0][3] == res[1][3]                   # identical delayed scale on both ranks

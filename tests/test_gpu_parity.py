@@ -763,11 +763,16 @@ def test_data_parallel_step_single_rank():
     try:
         b = make()
         DataParallelStep(b)()
+        bs = make()
+        sharded = DataParallelStep(bs, shard_grads=True)
+        sharded()
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()
     for k in ("post", "post_fp8", "out", "dPre", "dX", "dW1", "dW2", "state", "W2q_t"):
         assert torch.equal(getattr(plain, k), getattr(b, k)), k
+    # one rank owns every row: the reduce-scattered shards are the whole gradients
+    assert torch.equal(sharded.dW1_shard, plain.dW1) and torch.equal(sharded.dW2_shard, plain.dW2)
 
 
 # ---------------------------------------------------------------------------
