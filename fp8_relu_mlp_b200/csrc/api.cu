@@ -304,6 +304,9 @@ int ce_bwd_impl(bool fp8, int M, int d, int V, int T, const void* x, const void*
   TRY(map_kmajor(&p.tmB[0], W, dt, es, V, d, kGemmBN * kGemmBM / gemm_tile_m(kind), "W"));
   TRY(map_tile32(&p.tmOut[0], dlogits, BF16, 2, M, V, "dlogits"));
   fill_common(p, kind, di, M, V, d, 1);
+  // the pairs at work share one vocabulary tile of the head, which then stays
+  // in L2 while the dlogits stream passes through
+  p.n_major = 1;
   p.ce_lse = lse;
   p.ce_loss = loss;
   p.ce_dloss = dloss;

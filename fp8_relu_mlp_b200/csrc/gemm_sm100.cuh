@@ -57,6 +57,7 @@ struct alignas(64) GemmParams {
   unsigned long long timeout_ns;
   int debug_flags;
   int launch_flags;  // FP8MLP_LAUNCH_OVERLAP_PREVIOUS: wait for the previous grid only before finishing
+  int n_major;       // tile order: 0 = row blocks outer (consecutive tiles share A), 1 = column blocks outer
   // softcapped cross-entropy (CeFwd / CeBwd); the logits are y = acc (BF16
   // inputs) or acc * s_x^-1 * s_w^-1 (e4m3 inputs, scales in st_in / w_in_scale_inv)
   int ce_T;                  // targets per row (1..4)
@@ -191,6 +192,20 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 }  // namespace dev
 
+// (row block, column block) of tile tt within its group.  With n_major the
+// CTA pairs working at the same time share a column block, i.e. one B tile,
+// which then leaves DRAM once even while a large output stream runs through
+// L2; otherwise they share row blocks (A tiles).
+__device__ __forceinline__ void tile_coords(const GemmParams& p, int tt, int& mb, int& nb) {
+  if (p.n_major) {
+    nb = tt / p.tiles_m;
+    mb = tt - nb * p.tiles_m;
+  } else {
+    mb = tt / p.tiles_n;
+    nb = tt - mb * p.tiles_n;
+  }
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_constant__ GemmParams p) {
   using namespace dev;
@@ -275,8 +290,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
       for (int t = pair; t < num_tiles; t += npairs) {
         const int g = t / tiles_per_group;
         const int tt = t - g * tiles_per_group;
-        const int m0 = (tt / p.tiles_n) * C::TILE_M + static_cast<int>(rank) * C::BM;  // this CTA's A rows
-        const int n0 = (tt % p.tiles_n) * C::BN + static_cast<int>(rank) * C::B_ROWS;  // this CTA's B rows
+        int mb, nb;
+        tile_coords(p, tt, mb, nb);
+        const int m0 = mb * C::TILE_M + static_cast<int>(rank) * C::BM;  // this CTA's A rows
+        const int n0 = nb * C::BN + static_cast<int>(rank) * C::B_ROWS;  // this CTA's B rows
         const CUtensorMap* mA = &p.tmA[g];
         const CUtensorMap* mB = &p.tmB[g];
         bool ok = true;
@@ -425,12 +442,14 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
     uint8_t* aux_ring = sAux + e * C::AUX_WARP;
     uint64_t* my_auxb = auxb + e * C::NAUX;
     auto tile_rows = [&](int tile) {  // first row of this warp's 32 rows in `tile`
-      const int tt2 = tile - (tile / tiles_per_group) * tiles_per_group;
-      return (tt2 / p.tiles_n) * C::TILE_M + static_cast<int>(rank) * C::BM + q * 32;
+      int mb2, nb2;
+      tile_coords(p, tile - (tile / tiles_per_group) * tiles_per_group, mb2, nb2);
+      return mb2 * C::TILE_M + static_cast<int>(rank) * C::BM + q * 32;
     };
     auto tile_cols = [&](int tile) {
-      const int tt2 = tile - (tile / tiles_per_group) * tiles_per_group;
-      return (tt2 % p.tiles_n) * C::BN;
+      int mb2, nb2;
+      tile_coords(p, tile - (tile / tiles_per_group) * tiles_per_group, mb2, nb2);
+      return nb2 * C::BN;
     };
     if constexpr (C::EPI == Epi::DPre) {
       if (pair < num_tiles) {
@@ -449,7 +468,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
     for (int t = pair; t < num_tiles; t += npairs) {
       const int g = t / tiles_per_group;
       const int tt = t - g * tiles_per_group;
-      const int mb = tt / p.tiles_n, nb = tt % p.tiles_n;
+      int mb, nb;
+      tile_coords(p, tt, mb, nb);
       const int row0 = tile_rows(t);
       const int n0 = nb * C::BN;
       const int next_tile = t + npairs;
