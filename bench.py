@@ -1133,7 +1133,7 @@ def run_stack(a, W, world, rank, local_rank):
         b.W1.copy_(MLPBlock.bits_to_bf16(P["W1"], dev))
         b.W2.copy_(MLPBlock.bits_to_bf16(P["W2"], dev))
     S.r[0].copy_(MLPBlock.bits_to_bf16(r0, dev))
-    dtop_d = MLPBlock.bits_to_bf16(dtop, dev)
+    io = {"dtop": MLPBlock.bits_to_bf16(dtop, dev)}  # dL/dr_L of the step (an input, like r_0)
     S.refresh_w2_caches()
     S.calibrate()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -1145,7 +1145,7 @@ def run_stack(a, W, world, rank, local_rank):
                 ev[i].record()
         mark(0)
         S.forward()
-        S.dr.copy_(dtop_d)
+        S.dr.copy_(io["dtop"])
         # backward of the top layer, with its dW launch marked
         A.fp8mlp_bwd_dpre(M, d, h, S.dr, last.W2, last.post, last.dPre)
         A.fp8mlp_bwd_dx(M, d, h, last.dPre, last.W1, last.dX)
@@ -1222,37 +1222,39 @@ def run_stack(a, W, world, rank, local_rank):
     peak_sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     e2e = None
     if not a.no_e2e:
+        # r_0 and dL/dr_L in from pinned host memory, r_L and dL/dr_0 back,
+        # every step; copies overlapped with the neighbouring steps
+        # (hostio.HostPipeline over two sets of those four buffers)
+        from fp8_relu_mlp_b200.hostio import HostPipeline
         r0h = torch.from_numpy(r0.view(np.int16)).view(torch.bfloat16).pin_memory()
         dth = torch.from_numpy(dtop.view(np.int16)).view(torch.bfloat16).pin_memory()
         rLh = torch.empty(M, d, dtype=torch.bfloat16).pin_memory()
         dr0h = torch.empty(M, d, dtype=torch.bfloat16).pin_memory()
+        sets = [dict(r0=S.r[0], dtop=io["dtop"], rL=S.r[L], dr=S.dr)]
+        sets.append({k: v.clone() for k, v in sets[0].items()})
 
-        def body():
-            S.r[0].copy_(r0h, non_blocking=True)
-            dtop_d.copy_(dth, non_blocking=True)
+        def set_step(k):
+            S.r[0], io["dtop"], S.r[L], S.dr = sets[k]["r0"], sets[k]["dtop"], sets[k]["rL"], sets[k]["dr"]
             step()
-            rLh.copy_(S.r[L], non_blocking=True)
-            dr0h.copy_(S.dr, non_blocking=True)
 
-        body()
+        pipe = HostPipeline(set_step, [[sb["r0"], sb["dtop"]] for sb in sets], [[sb["rL"], sb["dr"]] for sb in sets],
+                            device=dev, graph=not a.eager)
+        S.r[0], io["dtop"], S.r[L], S.dr = sets[0]["r0"], sets[0]["dtop"], sets[0]["rL"], sets[0]["dr"]
+        pipe.run([r0h, dth], [rLh, dr0h], 2)
         torch.cuda.synchronize()
-        g2 = None if a.eager else S.blocks[0].capture(body)
-        for _ in range(2):
-            g2.replay() if g2 is not None else body()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
-        e0.record()
-        for _ in range(a.steps):
-            g2.replay() if g2 is not None else body()
-        e1.record()
-        e1.synchronize()
-        t2 = e0.elapsed_time(e1) * 1e-3
+        if dist:
+            dist.barrier()
+        timer = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        pipe.run([r0h, dth], [rLh, dr0h], a.steps, timer)
+        timer[1].synchronize()
+        t2 = timer[0].elapsed_time(timer[1]) * 1e-3
         if dist:
             tt = torch.tensor([t2], device=dev, dtype=torch.float64)
             dist.all_reduce(tt, op=dist.ReduceOp.MAX)
             t2 = float(tt.item())
         e2e = {"value": M * world * a.steps / t2, "unit": "tokens/s", "h2d_bytes_per_step": 4 * M * d,
-               "d2h_bytes_per_step": 4 * M * d}
+               "d2h_bytes_per_step": 4 * M * d,
+               "overlap": "copies on two streams beside the compute, double-buffered device sets"}
     if rank == 0:
         traffic = load_traffic(W.name).get("bwd_dw")
         line = {
