@@ -172,3 +172,45 @@ def test_heavytail_spike_saturates_and_matches():
     blk.update_scale()
     A_spike = _oracle_amax(xs, P["W1"])
     assert abs(blk.read_state()["amax_prev"] / float(A_spike) - 1) <= 2.0 ** -7
+
+
+def test_fullsize_fp8_up_overlapped_step_sampled():
+    """The e4m3 up-projection at the benchmark's size (bench.py --fp8-up,
+    M=16384), through the overlapped training step the benchmark times: the
+    x-scale bit-exact from the oracle's own max |x|, the W1 cache and the x
+    codes bit-exact, sampled rows of post, out and dX against the oracle's
+    same FP8 pipeline (the BF16 backward of its own post)."""
+    W = synth.WORKLOADS["step16k"]
+    M, d, h = W.M, W.d, W.h
+    P = synth.make_problem(M, d, h, seed=0)
+    blk = MLPBlock(M, d, h, margin=W.margin, fp8_up=True)
+    _load(blk, P)
+    blk.refresh_w2_cache()
+    blk.refresh_w1_cache()
+    blk.calibrate()
+    torch.cuda.synchronize()
+    ax = np.float32(np.abs(ref.bf16_to_f64(P["x"])).max())
+    st_x = ref.scale_update(ref.scale_state_init(W.margin, 1.0), ax)
+    assert np.float32(blk.read_state(blk.state_x)["scale"]) == st_x["scale"]
+    W1q_o, _, s_w1i = ref.w1_cache(P["W1"])
+    assert np.array_equal(host_bits(blk.W1q), W1q_o)
+    # the step at a known post scale
+    s_o = np.float32(448.0 / 50.0)
+    A.fp8mlp_scale_state_init(blk.state, W.margin, float(s_o))
+    side = torch.cuda.Stream()
+    blk.train_step_overlapped(side)
+    torch.cuda.synchronize()
+    rows = _sample_rows(M, 48, seed=3)
+    xq_o, _ = ref.quantise_x(P["x"][rows], st_x["scale"])
+    assert np.array_equal(host_bits(blk.x_fp8)[rows], xq_o)
+    post_o = ref.relu2_post(ref.up_proj_fp8(xq_o, W1q_o, st_x["scale_inv"], s_w1i))
+    assert rel_fro(ref.bf16_to_f64(host_bits(blk.post)[rows]), ref.bf16_to_f64(post_o)) < 1e-2
+    W2q_o, _, s_w2i = ref.w2_cache(P["W2"])
+    out_o = ref.down_proj_fp8(ref.quantise_post(post_o, s_o), W2q_o, np.float32(np.float32(1) / s_o), s_w2i)
+    assert rel_fro(ref.bf16_to_f64(host_bits(blk.out)[rows]), ref.bf16_to_f64(out_o)) < 2e-2
+    # BF16 backward from the GPU's own post is the straight-through gradient;
+    # the oracle's backward uses its own post (from the e4m3 up-projection)
+    dPre_o = ref.bwd_dpre(post_o, P["dOut"][rows], P["W2"])
+    dX_o = ref.bwd_dx(dPre_o, P["W1"])
+    assert rel_fro(ref.bf16_to_f64(host_bits(blk.dX)[rows]), ref.bf16_to_f64(dX_o)) < 2e-2
+    assert A.fp8mlp_get_device_status() == 0
