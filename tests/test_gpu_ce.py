@@ -314,3 +314,32 @@ def test_ce_fullsize_sampled_rows(fp8):
     tol = 2.0 ** -8 * np.abs(want) + (1e-4 + 4 * eps[:, None]) * scale + 1e-30
     assert not (np.abs(got - want) > tol).any()
     assert h.intact() and dl.intact()
+
+
+@pytest.mark.parametrize("cap", [1.0, 40.0])
+def test_ce_cap_extremes(cap):
+    # logits far beyond the cap: with c = 40 the smallest terms exp(z - c)
+    # reach e^-80 (still normal fp32), with c = 1 every z is within [-1, 1].
+    # The exponent arguments grow with c (|c log2(e) (t - 1)| <= 2c log2(e)),
+    # so the transcendental part of the tolerance scales with c / 15.
+    M, d, V, T = 257, 64, 1040, 2
+    P = synth.make_head_problem(M, d, V, T=T, seed=int(cap) + 29, logit_std=100.0)
+    h = Head(P, T, WEIGHTS, cap=cap)
+    h.fwd()
+    dl = h.bwd(reduction=A.CE_MEAN)
+    torch.cuda.synchronize()
+    X, Wm = ref.bf16_to_f64(h.x_bits), ref.bf16_to_f64(h.W_bits)
+    y = X @ Wm.T
+    eps = _eps_y(X, Wm)
+    f = ref.ce_forward(y, h.tg, h.w, cap)
+    tol = TOL_TR * max(1.0, cap / 15.0) + eps
+    lse = host_bits(h.lse.t).astype(np.float64)
+    np.testing.assert_array_less(np.abs(lse - f["lse"]), tol + 1e-6 * np.abs(f["lse"]))
+    row = host_bits(h.row.t).astype(np.float64)
+    _, we = ref._ce_targets(h.tg, h.w, V)
+    np.testing.assert_array_less(np.abs(row - f["row_loss"]), we.sum(axis=1) * 2 * tol + 1e-6 * np.abs(f["row_loss"]) + 1e-12)
+    want = ref.ce_backward_dlogits(y, h.tg, h.w, cap, f["lse"], ref.ce_grad_scale(1.0, f["weight_sum"], True))
+    got = ref.bf16_to_f64(host_bits(dl.t))
+    assert rel_fro(got, want) < 4e-3
+    assert np.isfinite(lse).all() and np.isfinite(got).all()
+    assert h.intact() and dl.intact()
