@@ -214,3 +214,50 @@ def test_fullsize_fp8_up_overlapped_step_sampled():
     dX_o = ref.bwd_dx(dPre_o, P["W1"])
     assert rel_fro(ref.bf16_to_f64(host_bits(blk.dX)[rows]), ref.bf16_to_f64(dX_o)) < 2e-2
     assert A.fp8mlp_get_device_status() == 0
+
+
+@pytest.mark.parametrize("fp8_up", [False, True])
+def test_stack9_fullsize_sampled_rows(fp8_up):
+    """The 9-layer stack at the benchmark's size (M=131072), in the launch
+    configuration bench.py times.  With every layer's delayed scales fixed
+    the stack is row-wise independent (RMSNorm, the MLP and the residual act
+    per token), so the oracle runs sampled rows through all nine layers,
+    forward (r_L) and backward (dL/dr_0)."""
+    from fp8_relu_mlp_b200.block import MLPStack
+    W = synth.WORKLOADS["stack9"]
+    L, M, d, h = W.layers, W.M, W.d, W.h
+    g = synth.rng(1000)
+    r0 = synth.to_bf16_bits(synth.make_x(g, M, d, "normal"))
+    dtop = synth.to_bf16_bits(synth.make_x(g, M, d, "normal"))
+    S = MLPStack(L, M, d, h, margin=W.margin, fp8_up=fp8_up)
+    layers, scales, xsc = [], [], []
+    for l, b in enumerate(S.blocks):
+        P = synth.make_problem(1, d, h, seed=100 + l)
+        b.W1.copy_(MLPBlock.bits_to_bf16(P["W1"], b.device))
+        b.W2.copy_(MLPBlock.bits_to_bf16(P["W2"], b.device))
+        W2q_t, _, s_wi = ref.w2_cache(P["W2"])
+        lay = dict(W1=P["W1"], W2=P["W2"], W2q_t=W2q_t, w2_scale_inv=s_wi)
+        s = np.float32(448.0 / (2.0 * (20.0 + 3 * l)))
+        A.fp8mlp_scale_state_init(b.state, W.margin, float(s))
+        scales.append((s, np.float32(np.float32(1) / s)))
+        if fp8_up:
+            lay["W1q"], _, lay["w1_scale_inv"] = ref.w1_cache(P["W1"])
+            sx = np.float32(448.0 / (2.0 * 5.0))
+            A.fp8mlp_scale_state_init(b.state_x, W.margin, float(sx))
+            xsc.append((sx, np.float32(np.float32(1) / sx)))
+        layers.append(lay)
+    S.refresh_w2_caches()
+    S.r[0].copy_(MLPBlock.bits_to_bf16(r0, S.device))
+    S.forward()
+    S.dr.copy_(MLPBlock.bits_to_bf16(dtop, S.device))
+    S.backward()
+    torch.cuda.synchronize()
+    rows = _sample_rows(M, 24, seed=5)
+    if fp8_up:
+        saved, rL = ref.stack_forward_fp8up(r0[rows], layers, scales, xsc)
+    else:
+        saved, rL = ref.stack_forward(r0[rows], layers, scales)
+    dr0, _ = ref.stack_backward(saved, layers, dtop[rows])
+    assert rel_fro(ref.bf16_to_f64(host_bits(S.r[L])[rows]), ref.bf16_to_f64(rL)) < 2e-2
+    assert rel_fro(ref.bf16_to_f64(host_bits(S.dr)[rows]), ref.bf16_to_f64(dr0)) < 2e-2
+    assert A.fp8mlp_get_device_status() == 0
