@@ -370,6 +370,7 @@ def run_ours(a, W, world, rank, local_rank):
     if world > 1:
         import torch.distributed as dist
         import datetime
+        torch.cuda.set_device(local_rank)  # before the communicator binds a device
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -675,6 +676,12 @@ def run_linear(a, W, world, rank, local_rank):
     from fp8_relu_mlp_b200 import _abi as A
     from fp8_relu_mlp_b200 import synth
     from fp8_relu_mlp_b200.block import MLPBlock
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local_rank)  # before the communicator binds a device
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     A.fp8mlp_set_programmatic_launch(not a.no_pdl)
@@ -736,6 +743,9 @@ def run_linear(a, W, world, rank, local_rank):
         flush.zero_()
         run()
     torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
     step_ms, fwd_ms = [], []
     with ClockSampler(local_rank) as clk:
         for _ in range(a.steps):
@@ -745,6 +755,10 @@ def run_linear(a, W, world, rank, local_rank):
             step_ms.append(ev[0].elapsed_time(ev[3]))
             fwd_ms.append(ev[1].elapsed_time(ev[2]))
     total_s = sum(step_ms) * 1e-3
+    if dist:
+        t = torch.tensor([total_s], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_s = float(t.item())
     F = 2 * M * K * N
     fwd_s = statistics.mean(fwd_ms) * 1e-3
     achieved = F / fwd_s / 1e12
@@ -762,21 +776,28 @@ def run_linear(a, W, world, rank, local_rank):
                             [[sb[2], sb[3]] for sb in sets], device=dev, graph=not a.eager)
         pipe.run([xh, dyh], [yh, dxh], max(a.warmup, 3))
         torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
         timer = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
         pipe.run([xh, dyh], [yh, dxh], a.steps, timer)
         timer[1].synchronize()
         te = timer[0].elapsed_time(timer[1]) * 1e-3
-        e2e = {"value": M * a.steps / te, "unit": "tokens/s",
+        if dist:
+            tt = torch.tensor([te], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            te = float(tt.item())
+        e2e = {"value": M * world * a.steps / te, "unit": "tokens/s",
                "h2d_bytes_per_step": int(2 * (xh.numel() + dyh.numel())),
                "d2h_bytes_per_step": int(2 * (yh.numel() + dxh.numel())),
                "overlap": "copies on two streams beside the compute, double-buffered device sets"}
     if rank == 0:
         line = {
             "metric": LINEAR_METRIC,
-            "value": M * a.steps / total_s, "unit": "tokens/s", "n_gpus": 1, "steps": a.steps, "warmup": a.warmup,
+            "value": M * world * a.steps / total_s, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup,
             "ms_per_step": total_s / a.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3 forward, bf16 backward (fp32 accumulate)", "data": "synthetic",
-            "config": dict(config_of(W), K=K, N=N),
+            "config": dict(config_of(W), K=K, N=N, parallelism=f"dp{world} replicas" if world > 1 else "single GPU"),
             "roofline": {"bound": "tensor", "kernel": "linear_fwd_fp8", "achieved": achieved, "peak": fp8_peak,
                          "unit": "TFLOP/s", "frac": achieved / fp8_peak, "traffic": None, "peak_source": fp8_src},
             "step_roofline": {"roofline_ms": roof * 1e3, "measured_ms": total_s / a.steps * 1e3,
@@ -787,6 +808,9 @@ def run_linear(a, W, world, rank, local_rank):
         if e2e:
             line["e2e"] = e2e
         print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 def run_compare_library(a, W):
@@ -887,6 +911,7 @@ def run_ce(a, W, world, rank, local_rank):
     if world > 1:
         import torch.distributed as dist
         import datetime
+        torch.cuda.set_device(local_rank)  # before the communicator binds a device
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -1117,6 +1142,7 @@ def run_stack(a, W, world, rank, local_rank):
     if world > 1:
         import torch.distributed as dist
         import datetime
+        torch.cuda.set_device(local_rank)  # before the communicator binds a device
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
