@@ -734,3 +734,31 @@ def test_stack_fp8up_close_to_bf16_stack():
         assert np.abs(d_out).max() <= 0.2 * np.abs(ref.bf16_to_f64(sv[l]["r"])).max()
         assert sv8[l]["x_amax"] == np.float32(np.abs(ref.bf16_to_f64(sv8[l]["x"])).max())
     assert _rel(ref.bf16_to_f64(r8), ref.bf16_to_f64(r)) < 0.1
+
+
+def test_ce_closed_form_at_exact_tanh_points():
+    # c = 2 and y = +-ln 3: tanh(ln(3)/2) = (3-1)/(3+1) = 1/2 exactly, so the
+    # softcapped logits are z = [1, 0, -1] (and 0 for y = 0), and everything
+    # downstream has a closed form:
+    #   lse(row 0) = ln(e + 1 + 1/e) = ln(1 + 2 cosh 1),  lse(row 1) = ln 3
+    #   losses with w = (1, 0.5), targets row 0 = (0, 2), row 1 = (1, ignored):
+    #   row 0 = (lse0 - 1) + 0.5 (lse0 + 1),  row 1 = ln 3,  weight 2.5
+    #   dL/dy = (W_m softmax(z) - sum_t w_t onehot) (1 - tanh^2), with
+    #   1 - tanh^2 = 3/4 at +-ln 3 and 1 at 0; W_0 = 1.5, W_1 = 1
+    import math
+    ln3 = math.log(3.0)
+    y = np.array([[ln3, 0.0, -ln3], [0.0, 0.0, 0.0]])
+    tg = np.array([[0, 2], [1, -1]])
+    w = [1.0, 0.5]
+    np.testing.assert_allclose(ref.softcap(y, 2.0), [[1.0, 0.0, -1.0], [0.0, 0.0, 0.0]], atol=1e-15)
+    f = ref.ce_forward(y, tg, w, 2.0)
+    lse0 = math.log(1.0 + 2.0 * math.cosh(1.0))
+    np.testing.assert_allclose(f["lse"], [lse0, ln3], rtol=1e-14)
+    np.testing.assert_allclose(f["row_loss"], [(lse0 - 1.0) + 0.5 * (lse0 + 1.0), ln3], rtol=1e-14)
+    assert f["weight_sum"] == 2.5
+    np.testing.assert_allclose(f["mean"], ((lse0 - 1.0) + 0.5 * (lse0 + 1.0) + ln3) / 2.5, rtol=1e-14)
+    e = math.e
+    p0 = np.array([e, 1.0, 1.0 / e]) / (e + 1.0 + 1.0 / e)
+    want = np.array([[(1.5 * p0[0] - 1.0) * 0.75, 1.5 * p0[1], (1.5 * p0[2] - 0.5) * 0.75],
+                     [1 / 3, 1 / 3 - 1.0, 1 / 3]])
+    np.testing.assert_allclose(ref.ce_backward_dlogits(y, tg, w, 2.0, f["lse"], 1.0), want, rtol=1e-13, atol=1e-15)
