@@ -35,8 +35,11 @@
  *   - Ownership: the caller owns and allocates every buffer; the library
  *     allocates no device memory and keeps no pointer after the call.
  *   - Device pointers must be 16-byte aligned (TMA).  Tensors are dense.
- *   - Shapes: M >= 0 is arbitrary (M = 0 is a no-op that returns FP8MLP_OK);
- *     d and h must be multiples of 16 and at least 16.
+ *   - Shapes: M >= 0 is arbitrary; d and h must be multiples of 16 and at
+ *     least 16.  M = 0 returns FP8MLP_OK and writes nothing, except the
+ *     results an empty batch defines: zero weight gradients (fp8mlp_bwd_dw,
+ *     fp8mlp_mlp_bwd, fp8mlp_linear_bwd) and zero cross-entropy totals
+ *     (fp8mlp_ce_fwd, fp8mlp_ce_fwd_fp8).
  *   - Asynchrony: every call enqueues work on `stream` (NULL = the legacy
  *     default stream) of the current device and returns without waiting.
  *     No call reads device data back to the host, except

@@ -27,6 +27,8 @@ SHAPES = [  # (M, d, h): several tiles, ragged tails in every dimension
     (1, 64, 256),
     (129, 128, 512),
     (1000, 768, 3072),
+    (17, 16, 16),     # the smallest d and h: K and N inside one partial block
+    (260, 48, 144),   # K under one k-block, N ending inside a 32-column chunk
 ]
 
 
@@ -362,6 +364,61 @@ def test_bwd_dw_empty_batch_zeroes():
     dW2 = torch.full((h, d), 3.0, device="cuda")
     A.fp8mlp_bwd_dw(0, d, h, None, None, None, None, dW1, dW2)
     assert (dW1 == 0).all() and (dW2 == 0).all()
+
+
+def test_empty_batch_every_entry_point():
+    """M = 0 through every call that takes a batch: nothing is written, except
+    the results an empty batch defines (zero weight gradients, zero
+    cross-entropy totals)."""
+    d, h, V, T = 64, 256, 512, 1
+
+    def buf(nbytes, dtype=torch.uint8):  # a sentinel byte pattern
+        return torch.full((nbytes,), 0x5A, dtype=torch.uint8, device="cuda").view(dtype)
+
+    x, W1, W2, post, dOut, dPre, dX, out = (buf(8192, torch.bfloat16) for _ in range(8))
+    q, W2q, W1q, xq = (buf(4096) for _ in range(4))
+    pa, rstd, ramax, lse, rowl, ws = (buf(4096, torch.float32) for _ in range(6))
+    inv = torch.ones(4, dtype=torch.float32, device="cuda")
+    st, st_x = _state(), _state()
+    tg = torch.zeros(16, dtype=torch.int32, device="cuda")
+    untouched = [x, W1, W2, post, dOut, dPre, dX, out, q, W2q, W1q, xq, pa, rstd, ramax, lse, rowl, ws]
+    before = [t.clone() for t in untouched]
+    dW1 = torch.full((h * d,), 3.0, device="cuda")
+    dW2 = torch.full((h * d,), 3.0, device="cuda")
+    dW = torch.full((h * d,), 3.0, device="cuda")
+    loss = torch.full((4,), 3.0, device="cuda")
+    loss8 = torch.full((4,), 3.0, device="cuda")
+    st_before = st.clone()
+
+    A.fp8mlp_up_proj_fused(0, d, h, x, W1, st, post, q, pa)
+    A.fp8mlp_up_proj_fused_fp8(0, d, h, xq, W1q, inv, st_x, st, post, q, pa)
+    A.fp8mlp_down_proj_fp8(0, d, h, q, W2q, inv, st, out)
+    A.fp8mlp_down_proj_bf16(0, d, h, post, W2, out)
+    A.fp8mlp_mlp_fwd(0, d, h, x, W1, W2q, inv, W2, st, post, q, pa, out)
+    A.fp8mlp_quantize_x(0, d, x, st_x, xq, pa)
+    A.fp8mlp_linear_fwd_fp8(0, d, h, xq, W1q, inv, st_x, out)
+    A.fp8mlp_linear_bwd(0, d, h, x, W1, dPre, dX, dW)
+    A.fp8mlp_bwd_dpre(0, d, h, dOut, W2, post, dPre)
+    A.fp8mlp_bwd_dx(0, d, h, dPre, W1, dX)
+    A.fp8mlp_bwd_dw(0, d, h, x, dPre, post, dOut, dW1, dW2)
+    A.fp8mlp_rmsnorm_fwd(0, d, x, out, rstd)
+    A.fp8mlp_rmsnorm_fwd_quant(0, d, x, out, rstd, st_x, xq, ramax)
+    A.fp8mlp_rmsnorm_bwd(0, d, x, rstd, dX, dOut, out)
+    A.fp8mlp_residual_add(0, d, x, out, dPre)
+    A.fp8mlp_ce_fwd(0, d, V, T, x, W1, tg, None, 15.0, lse, rowl, loss, ws)
+    A.fp8mlp_ce_fwd_fp8(0, d, V, T, xq, st_x, W1q, inv, tg, None, 15.0, lse, rowl, loss8, ws)
+    A.fp8mlp_ce_bwd_dlogits(0, d, V, T, x, W1, tg, None, 15.0, lse, loss, None, A.CE_MEAN, dPre)
+    A.fp8mlp_ce_bwd_dlogits_fp8(0, d, V, T, xq, st_x, W1q, inv, tg, None, 15.0, lse, loss, None, A.CE_MEAN, dPre)
+    torch.cuda.synchronize()
+    for t, b in zip(untouched, before):
+        assert torch.equal(t.view(torch.uint8), b.view(torch.uint8)), "a call with M = 0 wrote an output"
+    assert torch.equal(st, st_before)
+    assert (dW1 == 0).all() and (dW2 == 0).all() and (dW == 0).all()
+    assert (loss[:3] == 0).all() and loss[3] == 3.0 and (loss8[:3] == 0).all()
+    A.fp8mlp_mlp_bwd(0, d, h, x, W1, W2, post, dOut, dPre, dX, dW1.fill_(3.0), dW2.fill_(3.0))
+    torch.cuda.synchronize()
+    assert (dW1 == 0).all() and (dW2 == 0).all()
+    assert A.fp8mlp_get_device_status() == 0
 
 
 # ---------------------------------------------------------------------------
@@ -886,10 +943,10 @@ def test_fp8_up_forward_normal_inputs(M, d, h):
 # generic FP8 linear layer (attention projections)
 # ---------------------------------------------------------------------------
 
-LINEAR_SHAPES = [(300, 768, 2304), (1000, 768, 768), (129, 512, 768), (16384, 768, 2304)]
+LINEAR_SHAPES = [(300, 768, 2304), (1000, 768, 768), (129, 512, 768), (33, 16, 48), (16384, 768, 2304)]
 
 
-@pytest.mark.parametrize("M,K,N", LINEAR_SHAPES[:3])
+@pytest.mark.parametrize("M,K,N", LINEAR_SHAPES[:4])
 def test_linear_fwd_fp8_bit_exact_grid(M, K, N):
     P = synth.make_problem(M, K, N, seed=M + N, x_dist="grid", w_dist="grid")   # W1 is [N,K]
     st_x = _state(2.0, 16.0)
