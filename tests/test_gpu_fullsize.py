@@ -53,18 +53,19 @@ def _forward_checks(blk, P, W, rows, s_o):
     assert np.array_equal(host_bits(blk.W2q_t), W2q_o)
     s_inv = np.float32(np.float32(1) / s_o)
     f = ref.forward_rows(rows, P["x"], P["W1"], W2q_o, s_wi, s_o, s_inv)
-    post_g = host_bits(blk.post)[rows]
+    idx = torch.as_tensor(rows, device=blk.post.device)
+    post_g = host_bits(blk.post.index_select(0, idx))
     ok, frac = post_within_accumulation_bound(post_g, P["x"], P["W1"], rows=rows)
     assert ok and frac < 1e-2, frac
-    q_g = host_bits(blk.post_fp8)[rows]
+    q_g = host_bits(blk.post_fp8.index_select(0, idx))
     # equal wherever post agrees; elsewhere one FP8 step at most
     same = post_g == f["post"]
     assert np.array_equal(q_g[same], f["q"][same])
-    out_g = ref.bf16_to_f64(host_bits(blk.out)[rows])
+    out_g = ref.bf16_to_f64(host_bits(blk.out.index_select(0, idx)))
     assert rel_fro(out_g, ref.bf16_to_f64(f["out"])) < 2e-2
     # partial amax: block max of the GPU's own post, and its max is the global max
     pa = blk.partial_amax
-    assert float(pa.max()) == float(blk.post.float().max())
+    assert float(pa.max()) == float(blk.post.max())
     return f
 
 
@@ -260,4 +261,49 @@ def test_stack9_fullsize_sampled_rows(fp8_up):
     dr0, _ = ref.stack_backward(saved, layers, dtop[rows])
     assert rel_fro(ref.bf16_to_f64(host_bits(S.r[L])[rows]), ref.bf16_to_f64(rL)) < 2e-2
     assert rel_fro(ref.bf16_to_f64(host_bits(S.dr)[rows]), ref.bf16_to_f64(dr0)) < 2e-2
+    assert A.fp8mlp_get_device_status() == 0
+
+
+def test_batch_past_2_31_elements_sampled():
+    """M = 704512 tokens at d = 768, h = 3072: post and dPre hold 2.16e9
+    elements, so the rows from 699051 on sit past element 2^31 and every
+    offset into them needs 64-bit arithmetic.  Forward rows (at a scale the
+    oracle takes from the sampled rows; any s_t serves when both sides use
+    it) and backward rows against the oracle; dX and out past 2^31 bytes too.
+
+    The token rows repeat with a period of 16381 rows (a prime: no tile
+    boundary and no 2^32-byte wrap maps a row onto a copy of itself), so the
+    inputs are drawn in seconds; the oracle takes the sampled rows' own
+    values.  post and dPre are filled with NaN first, so an element left
+    unwritten shows."""
+    M, d, h = 704512, 768, 3072
+    assert M * h > 2 ** 31
+    period = 16381
+    P = synth.make_problem(period, d, h, seed=5)
+    reps = -(-M // period)
+    for k in ("x", "dOut"):
+        P[k] = np.ascontiguousarray(np.tile(P[k], (reps, 1))[:M])
+    blk = MLPBlock(M, d, h, margin=2.0, with_backward=True)
+    _load(blk, P)
+    blk.refresh_w2_cache()
+    rows = np.array(sorted(set(_sample_rows(M, 24, seed=3).tolist()) | {699050, 699051, 699052}))
+    A_rows = ref.amax(ref.relu2_post(ref.up_proj(P["x"][rows], P["W1"])))
+    st_o = ref.scale_update(ref.scale_state_init(2.0, 1.0), A_rows)
+
+    class _W:
+        margin = 2.0
+
+    blk.post.fill_(float("nan"))
+    blk.dPre.fill_(float("nan"))
+    _forward_checks(blk, P, _W, rows, st_o["scale"])
+    assert A.fp8mlp_get_device_status() == 0
+    blk.backward()
+    torch.cuda.synchronize()
+    idx = torch.as_tensor(rows, device=blk.dPre.device)
+    dPre_o, dX_o = ref.dx_rows(rows, P["x"], P["W1"], P["W2"], P["dOut"])
+    assert rel_fro(ref.bf16_to_f64(host_bits(blk.dPre.index_select(0, idx))), ref.bf16_to_f64(dPre_o)) < 1e-2
+    assert rel_fro(ref.bf16_to_f64(host_bits(blk.dX.index_select(0, idx))), ref.bf16_to_f64(dX_o)) < 1e-2
+    # every element past 2^31 was written
+    assert not bool(blk.post[699050:].isnan().any())
+    assert not bool(blk.dPre[699050:].isnan().any())
     assert A.fp8mlp_get_device_status() == 0
