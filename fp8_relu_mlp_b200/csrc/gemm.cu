@@ -6,7 +6,9 @@ namespace fp8mlp {
 
 // 2-CTA UMMA (cluster pairs, 256x256 tiles): each SM streams its 128 rows of
 // A and half of B, a third less operand traffic per FLOP than 1-CTA tiles
-using CfgUp = GemmCfg<2, kGemmBN, 5, false, false, false, Epi::UpFused>;
+// up-projection: the MMA waits on operand stages far more often than on the
+// epilogue, so one staging slot per epilogue warp pays for a sixth stage
+using CfgUp = GemmCfg<2, kGemmBN, 6, false, false, false, Epi::UpFused, 8, 4, 1>;
 using CfgDown8 = GemmCfg<2, kGemmBN, 6, true, false, false, Epi::DownScaled>;
 using CfgBf16MnB = GemmCfg<2, kGemmBN, 6, false, false, true, Epi::StoreBf16>;
 using CfgUpQ = GemmCfg<2, kGemmBN, 5, true, false, false, Epi::UpFused>;

@@ -75,7 +75,7 @@ struct alignas(64) GemmParams {
 };
 
 template <int CG_, int BN_, int STAGES_, bool FP8_, bool A_MN_, bool B_MN_, Epi EPI_, int NEPI_ = 8,
-          int AUX_RING_ = 4>
+          int AUX_RING_ = 4, int NSLOT_ = 2>
 struct GemmCfg {
   static constexpr int CG = CG_;           // CTAs per UMMA (1, or 2 = the pair of a cluster)
   static constexpr int BM = 128;           // accumulator rows per CTA (TMEM lanes)
@@ -115,7 +115,12 @@ struct GemmCfg {
   static constexpr bool STORES = EPI != Epi::CeFwd;  // the epilogue writes a tile with TMA
   static constexpr int OUT_BUF = !STORES ? 0 : 32 * ECOLS * (EPI == Epi::StoreF32 ? 4 : 2);
   static constexpr int OUT2_BUF = EPI == Epi::UpFused ? 32 * ECOLS : 0;
-  static constexpr int SLOT = OUT_BUF + OUT2_BUF;  // one output staging slot (two per epilogue warp)
+  static constexpr int SLOT = OUT_BUF + OUT2_BUF;  // one output staging slot
+  // staging slots per epilogue warp: with 2 a chunk is written while the
+  // previous chunk's store still reads the other slot; 1 leaves that shared
+  // memory to the operand ring
+  static constexpr int NSLOT = NSLOT_;
+  static_assert(NSLOT == 1 || NSLOT == 2, "staging slots");
   static_assert(SLOT % 1024 == 0, "slot alignment");
   // DPre: each epilogue warp streams its 32x32 blocks of post through a ring
   // of NAUX slots of its own, loaded NAUX chunks ahead of use
@@ -126,7 +131,7 @@ struct GemmCfg {
   static constexpr int TMEM_COLS = 512;
   static_assert(2 * BN <= TMEM_COLS, "two accumulators");
   static constexpr int NUM_BARS = 2 * STAGES + 4 + NEPI * NAUX + 1;
-  static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * (A_BYTES + B_BYTES) + 2 * NEPI * SLOT +
+  static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * (A_BYTES + B_BYTES) + NSLOT * NEPI * SLOT +
                                     NEPI * AUX_WARP + NUM_BARS * 8 + 16;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
@@ -216,7 +221,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
   uint8_t* sA = smem;
   uint8_t* sB = sA + C::STAGES * C::A_BYTES;
   uint8_t* sEpi = sB + C::STAGES * C::B_BYTES;
-  uint8_t* sAux = sEpi + 2 * C::NEPI * C::SLOT;
+  uint8_t* sAux = sEpi + C::NSLOT * C::NEPI * C::SLOT;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sAux + C::NEPI * C::AUX_WARP);
   uint64_t* full = bars;                // [STAGES] (the leader's are used)
   uint64_t* empty = bars + C::STAGES;   // [STAGES]
@@ -519,10 +524,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
               mbar_arrive_cluster(tempty_addr0 + acc * 8u);
           }
         }
-        uint8_t* slot = sEpi + (e * 2 + (ctr & 1u)) * C::SLOT;
+        uint8_t* slot = sEpi + (e * C::NSLOT + (C::NSLOT == 2 ? (ctr & 1u) : 0u)) * C::SLOT;
         const uint32_t sbase = smem_u32(slot);
         if constexpr (C::STORES) {
-          if (lane == 0) bulk_wait_read<1>();  // the store issued from this slot two chunks ago has read it
+          // the store issued from this slot NSLOT chunks ago has read it
+          if (lane == 0) bulk_wait_read<C::NSLOT - 1>();
           __syncwarp();
         }
         const int col0 = n0 + c * C::ECOLS;
