@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "internal.h"
@@ -51,8 +52,11 @@ int check_dims(int M, int d, int h) {
 
 // ---- device info --------------------------------------------------------
 constexpr int kMaxDevices = 64;
+// filled once per device under g_dev_mutex; g_dev_ok (release / acquire)
+// lets later calls from any thread read the entry without the lock
 DeviceInfo g_dev[kMaxDevices];
-bool g_dev_ok[kMaxDevices] = {};
+std::atomic<bool> g_dev_ok[kMaxDevices] = {};
+std::mutex g_dev_mutex;
 
 // ---- tensor maps ---------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -155,7 +159,12 @@ int current_device(DeviceInfo** info) {
     return fail(FP8MLP_ERR_NO_DEVICE, std::string("no CUDA device: ") + cudaGetErrorString(e));
   }
   if (dev < 0 || dev >= kMaxDevices) return fail(FP8MLP_ERR_NO_DEVICE, "device index out of range");
-  if (!g_dev_ok[dev]) {
+  if (!g_dev_ok[dev].load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (g_dev_ok[dev].load(std::memory_order_relaxed)) {
+      *info = &g_dev[dev];
+      return FP8MLP_OK;
+    }
     int major = 0, minor = 0, sms = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
@@ -175,7 +184,7 @@ int current_device(DeviceInfo** info) {
     g_dev[dev].device = dev;
     g_dev[dev].num_sms = sms;
     g_dev[dev].status = st;
-    g_dev_ok[dev] = true;
+    g_dev_ok[dev].store(true, std::memory_order_release);
   }
   *info = &g_dev[dev];
   return FP8MLP_OK;

@@ -1,5 +1,7 @@
 // Instantiations of the tcgen05 GEMM for the roles of the MLP block, the FP8
 // linear layer and the softcapped cross-entropy head.
+#include <atomic>
+
 #include "internal.h"
 
 namespace fp8mlp {
@@ -28,14 +30,16 @@ constexpr int kMaxDevices = 64;
 
 template <class C>
 cudaError_t launch_one(const GemmParams& p, int num_tiles, int num_sms, cudaStream_t s) {
-  static bool attr_done[kMaxDevices] = {};
+  // the attribute is set once per device; two threads racing here both set
+  // the same value, which CUDA allows
+  static std::atomic<bool> attr_done[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < kMaxDevices && !attr_done[dev]) {
+  if (dev < 0 || dev >= kMaxDevices || !attr_done[dev].load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(gemm_sm100_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr_done[dev] = true;
+    if (dev >= 0 && dev < kMaxDevices) attr_done[dev].store(true, std::memory_order_release);
   }
   // persistent: one CTA (pair) per SM (pair), never more than the tiles
   const int units = num_sms / C::CG;

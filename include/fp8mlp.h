@@ -327,8 +327,8 @@ int fp8mlp_w2_fp8_cache_refresh(int h, int d, const uint16_t* W2, uint8_t* W2q_t
                                 void* workspace, fp8mlp_stream_t stream);
 
 /*
- * The same refresh for callers that cannot allocate device memory.  The paper
- * has no counterpart: this entry point exists for integration only.  Some
+ * The same refresh for callers that cannot allocate device memory.  The
+ * pages describe no such call: this entry point exists for integration only.  Some
  * callers cannot provide a workspace: code inside another framework's
  * operator hook that owns every device allocation through its own pool and
  * exposes none to the op, or a runtime that forbids cudaMalloc/cudaFree on its

@@ -502,6 +502,62 @@ def test_tiny_three_steps_normal_perturbed():
         W2 = synth.perturb(W2, 0, step, W.perturb_var, "W2")
 
 
+_THREADS_SCRIPT = r"""
+import threading, torch
+from fp8_relu_mlp_b200 import _abi as A
+M, d, h, n = 1000, 128, 512, 8
+g = torch.Generator(device="cpu").manual_seed(7)
+W1 = (torch.randn(h, d, generator=g) / d ** 0.5).bfloat16().cuda()
+W2 = (torch.randn(h, d, generator=g) / h ** 0.5).bfloat16().cuda()
+xs = [torch.randn(M, d, generator=g).bfloat16().cuda() for _ in range(n)]
+rb, cb, _, _ = A.fp8mlp_partial_amax_shape(M, h)
+bufs = [dict(st=torch.zeros(8, device="cuda"), post=torch.empty(M, h, dtype=torch.bfloat16, device="cuda"),
+             q=torch.empty(M, h, dtype=torch.uint8, device="cuda"), pa=torch.empty(rb, cb, device="cuda"),
+             out=torch.empty(M, d, dtype=torch.bfloat16, device="cuda"), s=torch.cuda.Stream()) for _ in range(n)]
+torch.cuda.synchronize()
+go = threading.Barrier(n)
+errs = []
+def work(i):
+    b = bufs[i]
+    try:
+        go.wait()   # every thread's first library call at once
+        A.fp8mlp_scale_state_init(b["st"], 2.0, 4.0, stream=b["s"])
+        A.fp8mlp_up_proj_fused(M, d, h, xs[i], W1, b["st"], b["post"], b["q"], b["pa"], stream=b["s"])
+        A.fp8mlp_down_proj_bf16(M, d, h, b["post"], W2, b["out"], stream=b["s"])
+    except Exception as e:
+        errs.append(repr(e))
+ts = [threading.Thread(target=work, args=(i,)) for i in range(n)]
+[t.start() for t in ts]
+[t.join() for t in ts]
+torch.cuda.synchronize()
+assert not errs, errs
+for i in range(n):   # the same calls again, one at a time, must agree bit for bit
+    b = bufs[i]
+    post, q, out = b["post"].clone(), b["q"].clone(), b["out"].clone()
+    A.fp8mlp_up_proj_fused(M, d, h, xs[i], W1, b["st"], b["post"], b["q"], b["pa"])
+    A.fp8mlp_down_proj_bf16(M, d, h, b["post"], W2, b["out"])
+    torch.cuda.synchronize()
+    assert torch.equal(post.view(torch.int16), b["post"].view(torch.int16)), i
+    assert torch.equal(q, b["q"]), i
+    assert torch.equal(out.view(torch.int16), b["out"].view(torch.int16)), i
+assert A.fp8mlp_get_device_status() == 0
+print("ok")
+"""
+
+
+def test_first_calls_from_many_threads_at_once():
+    """A fresh process whose first library calls come from 8 host threads at
+    once, each on its own stream: the per-device set-up is done once and every
+    thread's results equal the same calls made one at a time."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _THREADS_SCRIPT], cwd=root, capture_output=True, text=True,
+                       timeout=300, env=dict(os.environ, PYTHONPATH=root))
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
+
+
 # ---------------------------------------------------------------------------
 # failure detection: a bounded wait runs out, the context stays usable
 # ---------------------------------------------------------------------------
