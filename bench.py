@@ -179,7 +179,7 @@ def kernel_work(M, d, h):
         "bwd_dpre": dict(bf16=F, fp8=0, bytes=2 * M * d + 2 * h * d + 2 * M * h + 2 * M * h),
         "bwd_dx": dict(bf16=F, fp8=0, bytes=2 * M * h + 2 * h * d + 2 * M * d),
         "bwd_dw": dict(bf16=2 * F, fp8=0, bytes=2 * M * h + 2 * M * d + 2 * M * h + 2 * M * d + 8 * h * d),
-        "amax_scale": dict(bf16=0, fp8=0, bytes=4 * (4 * -(-M // 128)) * -(-h // 256)),
+        "amax_scale": dict(bf16=0, fp8=0, bytes=4 * (8 * -(-M // 256)) * (4 * -(-h // 256))),
         "w2_cache": dict(bf16=0, fp8=0, bytes=2 * (2 * h * d) + d * h),
     }
 

@@ -13,7 +13,9 @@ namespace fp8mlp {
 using CfgUp = GemmCfg<2, kGemmBN, 6, false, false, false, Epi::UpFused, 8, 4, 1>;
 using CfgDown8 = GemmCfg<2, kGemmBN, 6, true, false, false, Epi::DownScaled>;
 using CfgBf16MnB = GemmCfg<2, kGemmBN, 6, false, false, true, Epi::StoreBf16>;
-using CfgUpQ = GemmCfg<2, kGemmBN, 5, true, false, false, Epi::UpFused>;
+// e4m3 up-projection: the mainloop is twice as fast, so the epilogue sets the
+// pace; 16 epilogue warps (96 registers each, one staging slot)
+using CfgUpQ = GemmCfg<2, kGemmBN, 5, true, false, false, Epi::UpFused, 16, 4, 1>;
 using CfgDPre = GemmCfg<2, kGemmBN, 4, false, false, false, Epi::DPre>;
 // dW: one long tile per CTA pair, so a light epilogue (4 warps) and more stages
 using CfgDW = GemmCfg<2, kGemmBN, 6, false, true, true, Epi::StoreF32, 4>;
@@ -68,11 +70,12 @@ cudaError_t launch_one(const GemmParams& p, int num_tiles, int num_sms, cudaStre
 }  // namespace
 
 int up_partial_cols() {
-  // fp8mlp_partial_amax_shape serves both up-projections
-  static_assert(CfgUp::BN / CfgUp::EPI_SPLIT == CfgUpQ::BN / CfgUpQ::EPI_SPLIT &&
+  // fp8mlp_partial_amax_shape serves both up-projections: blocks of 32 rows
+  // x 64 columns, whatever their epilogue warp counts
+  static_assert(CfgUp::PA_PER_TILE == CfgUpQ::PA_PER_TILE && CfgUp::BN == CfgUpQ::BN &&
                     CfgUp::TILE_M == CfgUpQ::TILE_M,
                 "the BF16 and e4m3 up-projections share one partial-amax layout");
-  return CfgUp::BN / CfgUp::EPI_SPLIT;
+  return CfgUp::BN / CfgUp::PA_PER_TILE;
 }
 
 int ce_partial_cols() {

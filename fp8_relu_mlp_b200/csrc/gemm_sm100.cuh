@@ -112,6 +112,10 @@ struct GemmCfg {
   static constexpr int NCH_W = NCHUNK / EPI_SPLIT;  // chunks per epilogue warp per tile
   static constexpr int THREADS = 64 + 32 * NEPI;
   static_assert(NEPI % 4 == 0 && NCHUNK % EPI_SPLIT == 0, "chunks per warp");
+  // up-projection: partial-amax entries per tile row block of 32 (one per 64
+  // columns: two chunks of one warp)
+  static constexpr int PA_PER_TILE = BN / 64;
+  static_assert(EPI != Epi::UpFused || NCH_W % 2 == 0, "whole 64-column blocks per warp");
   static constexpr bool STORES = EPI != Epi::CeFwd;  // the epilogue writes a tile with TMA
   static constexpr int OUT_BUF = !STORES ? 0 : 32 * ECOLS * (EPI == Epi::StoreF32 ? 4 : 2);
   static constexpr int OUT2_BUF = EPI == Epi::UpFused ? 32 * ECOLS : 0;
@@ -716,18 +720,23 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
             bulk_commit();
           }
         }
+        if constexpr (C::EPI == Epi::UpFused) {
+          if (cw & 1) {
+            // this warp's 32 rows x 64 columns of post are complete: one
+            // partial-amax entry (row block of 32, column block of 64)
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
+            if (lane == 0)
+              p.partial_amax[((mb * CG + static_cast<int>(rank)) * 4 + q) * (p.tiles_n * C::PA_PER_TILE) +
+                             nb * C::PA_PER_TILE + (c >> 1)] = round_bf16(tmax);
+            tmax = 0.f;
+          }
+        }
         ++ctr;
       }
       if (!ok) break;
       if constexpr (C::EPI == Epi::CeFwd) {
         if (ce_m < p.M) p.ce_partial[static_cast<size_t>(nb * C::EPI_SPLIT + half) * p.M + ce_m] = ce_sum;
-      }
-      if constexpr (C::EPI == Epi::UpFused) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
-        if (lane == 0)
-          p.partial_amax[((mb * CG + static_cast<int>(rank)) * 4 + q) * (p.tiles_n * C::EPI_SPLIT) +
-                         nb * C::EPI_SPLIT + half] = round_bf16(tmax);
       }
       if (++acc == 2) {
         acc = 0;

@@ -118,9 +118,9 @@ typedef struct fp8mlp_scale_state {
  *   post[m,i]     = bf16( fp32(r*r) ),  r = max(fp32(x[m,:] . W1[i,:]), 0)
  *   post_fp8[m,i] = e4m3_satfinite( fp32(post[m,i] * st->scale) )
  *   partial_amax  = max of post over blocks of block_rows x block_cols
- *                   (32 x 128), fp32, row-major [row_blocks][col_blocks]
+ *                   (32 x 64), fp32, row-major [row_blocks][col_blocks]
  *                   with the sizes of fp8mlp_partial_amax_shape
- *                   (8*ceil(M/256) x 2*ceil(h/256)); blocks that lie
+ *                   (8*ceil(M/256) x 4*ceil(h/256)); blocks that lie
  *                   wholly past row M or column h hold 0
  *   pre_debug     = optional fp32 pre [M,h] (NULL to skip; slow, for tests)
  *

@@ -101,10 +101,10 @@ def test_empty_batch_is_a_no_op():
 
 
 def test_partial_amax_shape():
-    assert A.fp8mlp_partial_amax_shape(16384, 3072) == (512, 24, 32, 128)
-    assert A.fp8mlp_partial_amax_shape(129, 256) == (8, 2, 32, 128)
-    assert A.fp8mlp_partial_amax_shape(300, 272) == (16, 4, 32, 128)
-    assert A.fp8mlp_partial_amax_shape(0, 256) == (0, 2, 32, 128)
+    assert A.fp8mlp_partial_amax_shape(16384, 3072) == (512, 48, 32, 64)
+    assert A.fp8mlp_partial_amax_shape(129, 256) == (8, 4, 32, 64)
+    assert A.fp8mlp_partial_amax_shape(300, 272) == (16, 8, 32, 64)
+    assert A.fp8mlp_partial_amax_shape(0, 256) == (0, 4, 32, 64)
     assert A.fp8mlp_workspace_size(16384, 768, 3072) >= 4
 
 
