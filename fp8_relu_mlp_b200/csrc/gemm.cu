@@ -16,7 +16,10 @@ using CfgBf16MnB = GemmCfg<2, kGemmBN, 6, false, false, true, Epi::StoreBf16>;
 // e4m3 up-projection: the mainloop is twice as fast, so the epilogue sets the
 // pace; 16 epilogue warps (96 registers each, one staging slot)
 using CfgUpQ = GemmCfg<2, kGemmBN, 5, true, false, false, Epi::UpFused, 16, 4, 1>;
-using CfgDPre = GemmCfg<2, kGemmBN, 4, false, false, false, Epi::DPre>;
+// dPre: 16 epilogue warps (two 32-column chunks each per tile) with a
+// one-chunk post ring and one staging slot, which leaves room for a fifth
+// operand stage
+using CfgDPre = GemmCfg<2, kGemmBN, 5, false, false, false, Epi::DPre, 16, 1, 1>;
 // dW: one long tile per CTA pair, so a light epilogue (4 warps) and more stages
 using CfgDW = GemmCfg<2, kGemmBN, 6, false, true, true, Epi::StoreF32, 4>;
 // LM head with the softcapped cross-entropy in the epilogue; the forward
