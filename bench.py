@@ -124,13 +124,16 @@ class ClockSampler:
 
     def __init__(self, index):
         self.samples, self.reasons, self.ok = [], set(), False
-        self.max_mhz = None
+        self.max_mhz = self.gpu = self.driver = None
         try:
             import pynvml
             pynvml.nvmlInit()
             self.nv = pynvml
             self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            name, drv = pynvml.nvmlDeviceGetName(self.h), pynvml.nvmlSystemGetDriverVersion()
+            self.gpu = name.decode() if isinstance(name, bytes) else name
+            self.driver = drv.decode() if isinstance(drv, bytes) else drv
             self.ok = True
         except Exception:
             self.ok = False
@@ -160,10 +163,9 @@ class ClockSampler:
             self.t.join()
 
     def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "gpu": self.gpu,
+                "driver": self.driver}
 
 
 # ---------------------------------------------------------------------------
@@ -306,18 +308,34 @@ def metric_of(W):
     return METRIC
 
 
-def cpu_baseline(W, seconds, tokens=None, fp8_up=False):
-    tokens = tokens or oracle_tokens(W, "baseline")
-    step, threads = oracle_step_timer(W, tokens, fp8_up=fp8_up)
+def _time_steps(step, seconds, max_reps=50):
     t0 = time.perf_counter()
     reps = 0
     while True:
         step()
         reps += 1
         el = time.perf_counter() - t0
-        if el >= seconds or reps >= 50:
-            break
+        if el >= seconds or reps >= max_reps:
+            return reps, el
+
+
+def cpu_baseline(W, seconds, tokens=None, fp8_up=False):
+    """The oracle on the host cores: all of them (the BLAS pool's threads),
+    then one thread on a third of the budget."""
+    tokens = tokens or oracle_tokens(W, "baseline")
+    step, threads = oracle_step_timer(W, tokens, fp8_up=fp8_up)
+    step()  # untimed: first-touch of the inputs and numpy's buffers
+    reps, el = _time_steps(step, seconds)
+    single = None
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            r1, e1 = _time_steps(step, seconds / 3)
+        single = {"value": tokens * r1 / e1, "unit": "tokens/s", "cores": 1, "sample": f"{r1} steps, {e1:.1f} s"}
+    except Exception:  # pragma: no cover
+        pass
     return {"value": tokens * reps / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "single_thread": single,
             "sample": ("each step also re-quantises its token share of the head's rows (weight cache); "
                        if W.name.startswith("ce") else "") +
                       f"{reps} oracle steps of {tokens} tokens of the {W.name} workload "
