@@ -29,6 +29,7 @@ SHAPES = [  # (M, d, h): several tiles, ragged tails in every dimension
     (1000, 768, 3072),
     (17, 16, 16),     # the smallest d and h: K and N inside one partial block
     (260, 48, 144),   # K under one k-block, N ending inside a 32-column chunk
+    (1700, 64, 2800),  # 77 tiles on 74 CTA pairs: the last 3 run as half-width units
 ]
 
 
