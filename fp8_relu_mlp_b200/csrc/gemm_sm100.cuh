@@ -2,16 +2,18 @@
 //
 //   D[m, n] = sum_k A[m, k] * B[n, k]      (fp32 accumulate in TMEM)
 //
-// One CTA per SM (320 threads); with CG = 2 the CTAs of a cluster pair share
-// a 2-CTA UMMA over a 256-row tile (each CTA loads its 128 rows of A and half
-// of B; the leader issues the UMMA; each CTA drains its own 128 TMEM lanes):
+// One CTA per SM (64 + 32*NEPI threads); with CG = 2 the CTAs of a cluster
+// pair share a 2-CTA UMMA over a 256-row tile (each CTA loads its 128 rows of
+// A and half of B; the leader issues the UMMA; each CTA drains its own 128
+// TMEM lanes):
 //   warp 0      TMA producer: streams A/B k-blocks into a STAGES-deep smem ring
 //   warp 1      allocates 512 TMEM columns (two 256-column accumulators) and
 //               issues the UMMAs from one thread
-//   warps 2..9  epilogue: TMEM -> registers -> fused math -> swizzled smem ->
-//               TMA store, 32 columns at a time; warp w owns TMEM lanes
-//               32*(w%4) .. +31 (tile rows 32*(w%4) .. +31) and one half of
-//               the tile's columns, so two warps share each SM sub-partition
+//   warps 2..   NEPI epilogue warps (4, 8 or 16): TMEM -> registers -> fused
+//               math -> swizzled smem -> TMA store, 32 columns at a time; warp
+//               w owns TMEM lanes 32*(w%4) .. +31 (tile rows 32*(w%4) .. +31)
+//               and one of NEPI/4 column groups of the tile, so NEPI/4 warps
+//               share each SM sub-partition
 // The two accumulators let the epilogue of tile i overlap the mainloop of
 // tile i+1.  Operands are BF16 (kind::f16) or e4m3 (kind::f8f6f4), each
 // K-major or MN-major, staged with 128-byte swizzle.  TMA zero-fills rows and
@@ -131,7 +133,7 @@ struct GemmCfg {
   static constexpr int AUX_CHUNK = EPI == Epi::DPre ? 32 * ECOLS * 2 : 0;
   static constexpr int NAUX = EPI == Epi::DPre ? AUX_RING_ : 0;  // ring slots per warp
   static constexpr int AUX_WARP = AUX_CHUNK * NAUX;
-  static_assert(NAUX == 0 || (NAUX <= NCH_W && NCH_W % NAUX == 0), "post ring");
+  static_assert(NAUX == 0 || (NAUX <= NCH_W && NCH_W % (NAUX > 0 ? NAUX : 1) == 0), "post ring");
   static constexpr int TMEM_COLS = 512;
   static_assert(2 * BN <= TMEM_COLS, "two accumulators");
   static constexpr int NUM_BARS = 2 * STAGES + 4 + NEPI * NAUX + 1;
@@ -588,7 +590,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
           }
           store_row_bf16<64>(sbase, lane, pk);
         } else if constexpr (C::EPI == Epi::DPre) {
-          // post of this chunk was loaded one tile ahead into ring slot c
+          // post of this chunk was loaded NAUX chunks ahead of its use into
+          // ring slot q_aux % NAUX
           const uint32_t q_aux = iter * C::NCH_W + cw;
           const int slot_aux = static_cast<int>(q_aux % C::NAUX);
           if (!mbar_wait(&my_auxb[slot_aux], (q_aux / C::NAUX) & 1u, w)) {
