@@ -1331,6 +1331,40 @@ def run_stack(a, W, world, rank, local_rank):
         dist.destroy_process_group()
 
 
+def copy_bound(torch, dev, host_in, host_out, tokens, reps=5):
+    """Tokens/s if a step were nothing but its copies: the same pinned host
+    tensors copied in (host to device) and out (device to host) at once on
+    two streams, as the pipelined end-to-end step overlaps them."""
+    din = [torch.empty_like(h, device=dev) for h in host_in]
+    dout = [torch.empty_like(h, device=dev) for h in host_out]
+    s1, s2 = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    cur = torch.cuda.current_stream(dev)
+
+    def once():
+        with torch.cuda.stream(s1):
+            for h, d in zip(host_in, din):
+                d.copy_(h, non_blocking=True)
+        with torch.cuda.stream(s2):
+            for h, d in zip(host_out, dout):
+                h.copy_(d, non_blocking=True)
+
+    s1.wait_stream(cur)
+    s2.wait_stream(cur)
+    once()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    s1.wait_stream(cur)
+    s2.wait_stream(cur)
+    for _ in range(reps):
+        once()
+    cur.wait_stream(s1)
+    cur.wait_stream(s2)
+    e1.record(cur)
+    e1.synchronize()
+    return tokens * reps / (e0.elapsed_time(e1) * 1e-3)
+
+
 def measure_e2e(a, blk, P, torch, dev, stream, M, world, dist, step_fn=None):
     """Same step through the public API with host buffers: every step's
     inputs (x, dOut) come from pinned host memory and its results (out, dX)
@@ -1358,10 +1392,13 @@ def measure_e2e(a, blk, P, torch, dev, stream, M, world, dist, step_fn=None):
         tt = torch.tensor([t], device=dev, dtype=torch.float64)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         t = float(tt.item())
+    cb = copy_bound(torch, dev, [xh, gh], [oh, dxh], M * world)
     return {"value": M * world * a.steps / t, "unit": "tokens/s",
             "h2d_bytes_per_step": int(xh.numel() * 2 + gh.numel() * 2),
             "d2h_bytes_per_step": int(oh.numel() * 2 + dxh.numel() * 2),
-            "overlap": "copies on two streams beside the compute, double-buffered device sets"}
+            "overlap": "copies on two streams beside the compute, double-buffered device sets",
+            "copy_bound": {"value": cb, "unit": "tokens/s",
+                           "note": "the same pinned copies alone, both directions at once (this rank's link)"}}
 
 
 def main():

@@ -39,6 +39,8 @@ def test_bench_line_step16k():
     e = d["e2e"]
     assert e["value"] > 0 and e["unit"] == d["unit"] and e["value"] < d["value"]
     assert e["h2d_bytes_per_step"] == 2 * 16384 * 768 * 2 and e["d2h_bytes_per_step"] == 2 * 16384 * 768 * 2
+    # the copies alone bound the end-to-end step
+    assert 0 < e["value"] <= 1.1 * e["copy_bound"]["value"]
     c = d["cpu_baseline"]
     assert c["kind"] == "oracle" and c["value"] > 0 and c["cores"] >= 1 and c["sample"]
     clk = d["clocks"]
