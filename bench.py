@@ -723,6 +723,7 @@ def run_linear(a, W, world, rank, local_rank):
     y = torch.empty(M, N, dtype=bf, device=dev)
     dX = torch.empty(M, K, dtype=bf, device=dev)
     dW = torch.empty(N, K, dtype=torch.float32, device=dev)
+    wsl = torch.empty(max(16, A.fp8mlp_linear_bwd_workspace_size(M, K, N)), dtype=u8, device=dev)
     flush = torch.empty(256 << 20, dtype=u8, device=dev)
     A.fp8mlp_weight_fp8_cache_refresh(N, K, Wt, Wq, winv, ws)
     A.fp8mlp_quantize_x(M, K, x, st, xq, pax)
@@ -739,7 +740,7 @@ def run_linear(a, W, world, rank, local_rank):
         A.fp8mlp_linear_fwd_fp8(M, K, N, xq, Wq, winv, st, yb)
         mark(2)
         A.fp8mlp_amax_reduce_update_scale(pax, npx, st)
-        A.fp8mlp_linear_bwd(M, K, N, xb, Wt, dYb, dXb, dW)
+        A.fp8mlp_linear_bwd(M, K, N, xb, Wt, dYb, dXb, dW, workspace=wsl)
         A.fp8mlp_weight_fp8_cache_refresh(N, K, Wt, Wq, winv, ws)
         mark(3)
 
@@ -817,7 +818,8 @@ def run_linear(a, W, world, rank, local_rank):
             "dtype": "e4m3 forward, bf16 backward (fp32 accumulate)", "data": "synthetic",
             "config": dict(config_of(W), K=K, N=N, parallelism=f"dp{world} replicas" if world > 1 else "single GPU"),
             "roofline": {"bound": "tensor", "kernel": "linear_fwd_fp8", "achieved": achieved, "peak": fp8_peak,
-                         "unit": "TFLOP/s", "frac": achieved / fp8_peak, "traffic": None, "peak_source": fp8_src},
+                         "unit": "TFLOP/s", "frac": achieved / fp8_peak,
+                         "traffic": load_traffic(W.name).get("linear_fwd_fp8"), "peak_source": fp8_src},
             "step_roofline": {"roofline_ms": roof * 1e3, "measured_ms": total_s / a.steps * 1e3,
                               "frac": roof / (total_s / a.steps)},
             "clocks": clk.summary(), "gpu_launches": int(kps * a.steps),

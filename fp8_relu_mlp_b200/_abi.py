@@ -67,7 +67,7 @@ _SIGS = {
     "fp8mlp_up_proj_fused_fp8": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _p],
     "fp8mlp_linear_fwd_fp8": [_i, _i, _i, _p, _p, _p, _p, _p, _p],
     "fp8mlp_weight_fp8_cache_refresh": [_i, _i, _p, _p, _p, _p, _p],
-    "fp8mlp_linear_bwd": [_i, _i, _i, _p, _p, _p, _p, _p, _i, _p],
+    "fp8mlp_linear_bwd": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _i, _p],
     "fp8mlp_ce_fwd": [_i, _i, _i, _i, _p, _p, _p, _p, _f, _p, _p, _p, _p, _p],
     "fp8mlp_ce_fwd_fp8": [_i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _f, _p, _p, _p, _p, _p],
     "fp8mlp_ce_bwd_dlogits": [_i, _i, _i, _i, _p, _p, _p, _p, _f, _p, _p, _p, _i, _p, _p],
@@ -93,6 +93,8 @@ lib.fp8mlp_workspace_size.argtypes = [_i, _i, _i]
 lib.fp8mlp_workspace_size.restype = _sz
 lib.fp8mlp_ce_workspace_size.argtypes = [_i, _i, _i]
 lib.fp8mlp_ce_workspace_size.restype = _sz
+lib.fp8mlp_linear_bwd_workspace_size.argtypes = [_i, _i, _i]
+lib.fp8mlp_linear_bwd_workspace_size.restype = _sz
 lib.fp8mlp_kernel_launch_count.argtypes = []
 lib.fp8mlp_kernel_launch_count.restype = ctypes.c_ulonglong
 for _n in ("fp8mlp_error_string",):
@@ -231,8 +233,12 @@ def fp8mlp_weight_fp8_cache_refresh(N, K, W, Wq, w_scale_inv, workspace, stream=
                  _stream(stream))
 
 
-def fp8mlp_linear_bwd(M, K, N, x, W, dY, dX, dW, flags=0, stream=None):
-    return _call("fp8mlp_linear_bwd", M, K, N, _ptr(x), _ptr(W), _ptr(dY), _ptr(dX), _ptr(dW), flags,
+def fp8mlp_linear_bwd_workspace_size(M, K, N):
+    return int(lib.fp8mlp_linear_bwd_workspace_size(M, K, N))
+
+
+def fp8mlp_linear_bwd(M, K, N, x, W, dY, dX, dW, flags=0, stream=None, workspace=None):
+    return _call("fp8mlp_linear_bwd", M, K, N, _ptr(x), _ptr(W), _ptr(dY), _ptr(dX), _ptr(dW), _ptr(workspace), flags,
                  _stream(stream))
 
 

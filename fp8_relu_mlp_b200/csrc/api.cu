@@ -588,8 +588,13 @@ int fp8mlp_linear_fwd_fp8(int M, int K, int N, const uint8_t* x_fp8, const uint8
   return launch(GemmKind::Down8, p, di, stream, "linear_fwd_fp8 launch");
 }
 
+size_t fp8mlp_linear_bwd_workspace_size(int M, int K, int N) {
+  if (M < 2 * kLinearSplitRows || K <= 0 || N <= 0) return 0;
+  return sizeof(float) * static_cast<size_t>(N) * K;
+}
+
 int fp8mlp_linear_bwd(int M, int K, int N, const uint16_t* x, const uint16_t* W, const uint16_t* dY, uint16_t* dX,
-                      float* dW, int flags, fp8mlp_stream_t stream) {
+                      float* dW, void* workspace, int flags, fp8mlp_stream_t stream) {
   g_detail.clear();
   TRY(check_dims(M, N, K));
   TRY(check_launch_flags(flags));
@@ -618,13 +623,31 @@ int fp8mlp_linear_bwd(int M, int K, int N, const uint16_t* x, const uint16_t* W,
   }
   // dW[N,K] = dY^T . x: contraction over the M tokens, both operands MN-major
   GemmParams p{};
-  TRY(map_mnmajor(&p.tmA[0], dY, M, N, "dY"));
-  TRY(map_mnmajor(&p.tmB[0], x, M, K, "x"));
+  // with few output tiles (a third of the CTA pairs for 768 -> 2304) and a
+  // workspace, the tokens are split in two: rows [0, M0) accumulate into dW,
+  // rows [M0, M) into the workspace (the second group of one launch), and
+  // the workspace is added to dW afterwards, in that order
+  const int tiles = cdiv(N, kGemmBN) * cdiv(K, kGemmBN);
+  const bool split = workspace != nullptr && M >= 2 * kLinearSplitRows && 2 * tiles <= di->num_sms / 2;
+  if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 15u))
+    return fail(FP8MLP_ERR_INVALID_ARG, "workspace misaligned");
+  const int M0 = split ? cdiv(cdiv(M, 2), kLinearSplitRows) * kLinearSplitRows : M;
+  TRY(map_mnmajor(&p.tmA[0], dY, M0, N, "dY"));
+  TRY(map_mnmajor(&p.tmB[0], x, M0, K, "x"));
   TRY(map_tile32(&p.tmOut[0], dW, F32, 4, N, K, "dW"));
-  fill_common(p, GemmKind::DW, di, N, K, M, 1);
+  if (split) {
+    TRY(map_mnmajor(&p.tmA[1], dY + static_cast<size_t>(M0) * N, M - M0, N, "dY"));
+    TRY(map_mnmajor(&p.tmB[1], x + static_cast<size_t>(M0) * K, M - M0, K, "x"));
+    TRY(map_tile32(&p.tmOut[1], workspace, F32, 4, N, K, "workspace"));
+  }
+  fill_common(p, GemmKind::DW, di, N, K, M0, split ? 2 : 1);
   // dW neither reads dX nor writes what dX reads: it may overlap its tail
   p.launch_flags = dX != nullptr ? FP8MLP_LAUNCH_OVERLAP_PREVIOUS : flags;
-  return launch(GemmKind::DW, p, di, stream, "linear_bwd dW launch");
+  TRY(launch(GemmKind::DW, p, di, stream, "linear_bwd dW launch"));
+  if (!split) return FP8MLP_OK;
+  const cudaError_t e =
+      launch_add_f32(static_cast<size_t>(N) * K, dW, static_cast<const float*>(workspace), di->num_sms, stream);
+  return e == cudaSuccess ? FP8MLP_OK : cuda_fail(e, "linear_bwd dW add");
 }
 
 size_t fp8mlp_ce_workspace_size(int M, int V, int T) {

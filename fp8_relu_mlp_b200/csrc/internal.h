@@ -24,6 +24,7 @@ enum class GemmKind : int {
 };
 constexpr int kGemmBM = 128;  // accumulator rows per CTA
 constexpr int kGemmBN = 256;  // output tile columns
+constexpr int kLinearSplitRows = 64;  // the linear dW's token split falls on a k-block (64 BF16 rows)
 
 // rows of one output tile of `kind` (128 per CTA times the CTA-group size)
 int gemm_tile_m(GemmKind kind);
@@ -43,6 +44,7 @@ cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int num_tiles, int n
 
 // small kernels
 cudaError_t launch_state_init(fp8mlp_scale_state* st, float margin, float s0, cudaStream_t s);
+cudaError_t launch_add_f32(size_t n, float* dst, const float* src, int num_sms, cudaStream_t s);
 cudaError_t launch_amax_scale(const float* pa, int n, fp8mlp_scale_state* st, unsigned int* status, cudaStream_t s);
 // the W2 cache refresh reduces |W2| in blocks of kW2ElemsPerBlock elements,
 // one partial maximum per block in the caller's workspace

@@ -343,6 +343,18 @@ __global__ void residual_add_kernel(size_t n_vec, const uint4* __restrict__ r, c
   }
 }
 
+// dst += src over n fp32 values (n a multiple of 4): the second half of a
+// weight gradient split over the tokens, added in a fixed order
+__global__ void add_f32_kernel(size_t n4, float4* __restrict__ dst, const float4* __restrict__ src) {
+  pdl_wait();
+  pdl_launch_dependents();
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 a = dst[i], b = __ldcs(src + i);
+    dst[i] = make_float4(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y), __fadd_rn(a.z, b.z), __fadd_rn(a.w, b.w));
+  }
+}
+
 // x_q = e4m3(fp32(x * s_x)) with s_x = st->scale; block b also writes the
 // max |x| over its kXElemsPerBlock elements (BF16 magnitude bits: integer
 // order = value order) as the partial amax of x's delayed scale.
@@ -435,6 +447,14 @@ int grid_for(size_t work, int per_block, int num_sms, int blocks_per_sm) {
 }
 
 }  // namespace
+
+cudaError_t launch_add_f32(size_t n, float* dst, const float* src, int num_sms, cudaStream_t s) {
+  const size_t n4 = n / 4;
+  const cudaError_t e = launch_pdl(add_f32_kernel, dim3(grid_for(n4, 256, num_sms, 4)), dim3(256), 0, s, n4,
+                                   reinterpret_cast<float4*>(dst), reinterpret_cast<const float4*>(src));
+  count_launches(1);
+  return e;
+}
 
 cudaError_t launch_state_init(fp8mlp_scale_state* st, float margin, float s0, cudaStream_t s) {
   const cudaError_t e = launch_pdl(state_init_kernel, dim3(1), dim3(1), 0, s, st, margin, s0);

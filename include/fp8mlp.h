@@ -216,9 +216,22 @@ int fp8mlp_weight_fp8_cache_refresh(int N, int K, const uint16_t* W, uint8_t* Wq
  * The dW GEMM, which does not depend on dX, starts while the dX GEMM
  * finishes.  flags: 0, or FP8MLP_LAUNCH_OVERLAP_PREVIOUS for the first GEMM
  * launched (dX, or dW when dX is NULL), with the meaning given at
- * fp8mlp_bwd_dpre. */
+ * fp8mlp_bwd_dpre.
+ * workspace: NULL, or fp8mlp_linear_bwd_workspace_size(M, K, N) bytes
+ * (16-byte aligned, no initial contents needed).  When dW has so few
+ * 256x256 output tiles that they would keep at most half of the CTA pairs
+ * busy (768 -> 2304: 27 tiles for 74 pairs), the tokens are split in two at
+ * a multiple of 64 rows: the first part accumulates into dW, the second
+ * into the workspace in the same launch, and a last kernel adds the
+ * workspace to dW (dW = fp32(first part) + fp32(second part), a fixed
+ * order).  With NULL, or when the split does not apply, the workspace is
+ * not touched. */
 int fp8mlp_linear_bwd(int M, int K, int N, const uint16_t* x, const uint16_t* W, const uint16_t* dY, uint16_t* dX,
-                      float* dW, int flags, fp8mlp_stream_t stream);
+                      float* dW, void* workspace, int flags, fp8mlp_stream_t stream);
+
+/* Bytes of the optional workspace of fp8mlp_linear_bwd: 4*N*K when M >= 128,
+ * else 0. */
+size_t fp8mlp_linear_bwd_workspace_size(int M, int K, int N);
 
 /* ------------------------------------------------------------------------
  * Softcapped cross-entropy over a language-model head, without [M,V] logits.

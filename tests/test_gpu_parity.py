@@ -1020,8 +1020,13 @@ def test_linear_fwd_fp8_bit_exact_grid(M, K, N):
     assert y.intact()
 
 
+@pytest.mark.parametrize("split", [False, True])
 @pytest.mark.parametrize("M,K,N", LINEAR_SHAPES)
-def test_linear_fp8_fwd_bwd_normal(M, K, N):
+def test_linear_fp8_fwd_bwd_normal(M, K, N, split):
+    """With a workspace (split) dW of the shapes with few output tiles is
+    summed in two halves over the tokens: (300, 768, 2304) at row 192,
+    (1000, 768, 768) at 512, (129, 512, 768) at 128 (one row in the second
+    half), 16384 x 768 -> 2304 at 8192; M = 33 is below the split size."""
     P = synth.make_problem(M, K, N, seed=7 * M + N)
     s_x = np.float32(448.0 / 9.0)
     st_x = _state(2.0, float(s_x))
@@ -1038,8 +1043,12 @@ def test_linear_fp8_fwd_bwd_normal(M, K, N):
     dY = synth.to_bf16_bits(g.standard_normal((M, N)).astype(np.float32))
     dX = Guarded((M, K), torch.bfloat16)
     dW = Guarded((N, K), torch.float32)
-    A.fp8mlp_linear_bwd(M, K, N, dev_bf16(P["x"]), dev_bf16(P["W1"]), dev_bf16(dY), dX.t, dW.t)
+    wsl = Guarded((max(1, A.fp8mlp_linear_bwd_workspace_size(M, K, N)),), torch.uint8) if split else None
+    A.fp8mlp_linear_bwd(M, K, N, dev_bf16(P["x"]), dev_bf16(P["W1"]), dev_bf16(dY), dX.t, dW.t,
+                        workspace=wsl.t if split else None)
     torch.cuda.synchronize()
+    if split:
+        assert wsl.intact()
     rows = np.arange(M) if M <= 1000 else np.unique(np.r_[0, M - 1, np.random.default_rng(1).integers(0, M, 64)])
     xq_o, _ = ref.quantise_x(P["x"][rows], s_x)
     Wq_o, _, swi = ref.w1_cache(P["W1"])
