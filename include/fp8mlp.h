@@ -218,7 +218,8 @@ int fp8mlp_weight_fp8_cache_refresh(int N, int K, const uint16_t* W, uint8_t* Wq
  * launched (dX, or dW when dX is NULL), with the meaning given at
  * fp8mlp_bwd_dpre.
  * workspace: NULL, or fp8mlp_linear_bwd_workspace_size(M, K, N) bytes
- * (16-byte aligned, no initial contents needed).  When dW has so few
+ * (16-byte aligned, no initial contents needed; calls that may overlap on
+ * the GPU need workspaces of their own).  When dW has so few
  * 256x256 output tiles that they would keep at most half of the CTA pairs
  * busy (768 -> 2304: 27 tiles for 74 pairs), the tokens are split in two at
  * a multiple of 64 rows: the first part accumulates into dW, the second
