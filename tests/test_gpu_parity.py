@@ -121,6 +121,20 @@ def post_within_accumulation_bound(post_gpu, x, W1, rows=None):
     return bool(ok.all()), float((post_gpu != post_o).mean())
 
 
+def within_accumulation_bound(got, exact, absprod, K, bf16_out, extra=0.0):
+    """Element by element: a result accumulated in fp32 over K products, in
+    any order, lies within K 2^-24 sum_k |a_k b_k| of the exact sum (the
+    recursive-summation bound); a BF16 output adds half a BF16 step (2^-8
+    relative); `extra` covers a scaling applied after the sum."""
+    g = np.asarray(got, np.float64)
+    e = np.asarray(exact, np.float64)
+    bound = K * 2.0 ** -24 * absprod * (1 + extra) + extra * np.abs(e) + 1e-30
+    if bf16_out:
+        bound = bound + 2.0 ** -8 * np.maximum(np.abs(g), np.abs(e))
+    bad = np.abs(g - e) > bound
+    return (not bad.any()), int(bad.sum())
+
+
 @pytest.mark.parametrize("M,d,h", [(256, 64, 256), (1000, 768, 3072)])
 def test_up_proj_fused_normal_inputs(M, d, h):
     P = synth.make_problem(M, d, h, seed=11)
@@ -243,6 +257,11 @@ def test_down_proj_fp8(M, d, h):
     got = host_bits(out.t)
     # only the fp32 accumulation order and the final BF16 rounding differ
     assert rel_fro(ref.bf16_to_f64(got), ref.bf16_to_f64(want)) < 4e-3
+    Q, Wd = ref.e4m3_to_f64(q), ref.e4m3_to_f64(Wq)
+    comb = float(np.float32(np.float32(s_now["scale_inv"]) * swinv))
+    ok, nbad = within_accumulation_bound(ref.bf16_to_f64(got), (Q @ Wd.T) * comb,
+                                         (np.abs(Q) @ np.abs(Wd).T) * comb, h, True, extra=2.0 ** -23)
+    assert ok, nbad
     assert out.intact()
 
 
@@ -310,6 +329,13 @@ def test_bwd_dpre(M, d, h):
     want = ref.bwd_dpre(post, P["dOut"], P["W2"])
     got = host_bits(dPre.t)
     assert rel_fro(ref.bf16_to_f64(got), ref.bf16_to_f64(want)) < 4e-3
+    # dPre = 2 sqrt(post) dPost: the accumulation bound of dPost times
+    # 2 sqrt(post), plus the approximate square root (relative 2^-21 allowed)
+    G, W2 = ref.bf16_to_f64(P["dOut"]), ref.bf16_to_f64(P["W2"])
+    r2 = 2.0 * np.sqrt(ref.bf16_to_f64(post))
+    ok, nbad = within_accumulation_bound(ref.bf16_to_f64(got), r2 * (G @ W2.T), r2 * (np.abs(G) @ np.abs(W2).T),
+                                         d, True, extra=2.0 ** -21)
+    assert ok, nbad
     # zero post gives exactly zero dPre (relu'(pre) = 0 there)
     assert (ref.bf16_to_f64(got)[ref.bf16_to_f64(post) == 0] == 0).all()
     assert dPre.intact()
@@ -325,6 +351,9 @@ def test_bwd_dx(M, d, h):
     torch.cuda.synchronize()
     want = ref.bwd_dx(dPre, P["W1"])
     assert rel_fro(ref.bf16_to_f64(host_bits(dX.t)), ref.bf16_to_f64(want)) < 4e-3
+    D, W1 = ref.bf16_to_f64(dPre), ref.bf16_to_f64(P["W1"])
+    ok, nbad = within_accumulation_bound(ref.bf16_to_f64(host_bits(dX.t)), D @ W1, np.abs(D) @ np.abs(W1), h, True)
+    assert ok, nbad
     assert dX.intact()
 
 
@@ -339,6 +368,11 @@ def test_bwd_dw(M, d, h):
     torch.cuda.synchronize()
     assert rel_fro(host_bits(dW1.t), ref.bwd_dw1(dPre, P["x"])) < 1e-4
     assert rel_fro(host_bits(dW2.t), ref.bwd_dw2(post, P["dOut"])) < 1e-4
+    D, X = ref.bf16_to_f64(dPre), ref.bf16_to_f64(P["x"])
+    Pp, G = ref.bf16_to_f64(post), ref.bf16_to_f64(P["dOut"])
+    ok1, n1 = within_accumulation_bound(host_bits(dW1.t), D.T @ X, np.abs(D).T @ np.abs(X), M, False)
+    ok2, n2 = within_accumulation_bound(host_bits(dW2.t), Pp.T @ G, np.abs(Pp).T @ np.abs(G), M, False)
+    assert ok1 and ok2, (n1, n2)
     assert dW1.intact() and dW2.intact()
 
 
