@@ -1089,13 +1089,29 @@ def test_linear_fp8_fwd_bwd_normal(M, K, N, split):
     assert np.array_equal(host_bits(Wq), Wq_o)
     y_o = ref.linear_fp8(xq_o, Wq_o, np.float32(np.float32(1) / s_x), swi)
     assert rel_fro(ref.bf16_to_f64(host_bits(y.t)[rows]), ref.bf16_to_f64(y_o)) < 4e-3
+    # element by element: the exact product of the e4m3 operands, scaled
+    Xq, Wqd = ref.e4m3_to_f64(xq_o), ref.e4m3_to_f64(Wq_o)
+    comb = float(np.float32(np.float32(np.float32(1) / s_x) * np.float32(swi[0] if np.ndim(swi) else swi)))
+    ok, nbad = within_accumulation_bound(ref.bf16_to_f64(host_bits(y.t)[rows]), (Xq @ Wqd.T) * comb,
+                                         (np.abs(Xq) @ np.abs(Wqd).T) * comb, K, True, extra=2.0 ** -23)
+    assert ok, nbad
     exact = ref.bf16_to_f64(P["x"][rows]) @ ref.bf16_to_f64(P["W1"]).T
     assert rel_fro(ref.bf16_to_f64(host_bits(y.t)[rows]), exact) < 6e-2
     dX_o = ref.bf16_bits_from_f32(ref.f32(ref.bf16_to_f64(dY[rows]) @ ref.bf16_to_f64(P["W1"])))
     assert rel_fro(ref.bf16_to_f64(host_bits(dX.t)[rows]), ref.bf16_to_f64(dX_o)) < TOL_GRAD
+    Gr, Wd = ref.bf16_to_f64(dY[rows]), ref.bf16_to_f64(P["W1"])
+    ok, nbad = within_accumulation_bound(ref.bf16_to_f64(host_bits(dX.t)[rows]), Gr @ Wd, np.abs(Gr) @ np.abs(Wd), N,
+                                         True)
+    assert ok, nbad
     if M <= 1000:
         _, dW_o = ref.linear_bwd(P["x"], P["W1"], dY)
         assert rel_fro(host_bits(dW.t), dW_o) < TOL_GRAD
+        # with the token split, each half is within its own bound and the
+        # final add rounds once more (relative 2^-24)
+        G, X = ref.bf16_to_f64(dY), ref.bf16_to_f64(P["x"])
+        ok, nbad = within_accumulation_bound(host_bits(dW.t), G.T @ X, np.abs(G).T @ np.abs(X), M, False,
+                                             extra=2.0 ** -23)
+        assert ok, nbad
     else:
         G, X = ref.bf16_to_f64(dY), ref.bf16_to_f64(P["x"])
         pairs = [(0, 0), (N - 1, K - 1), (N // 2, 17), (5, K // 3)]
