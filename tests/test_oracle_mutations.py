@@ -81,7 +81,31 @@ MUTATIONS = {
                                       ["test_stack_fp8up_close_to_bf16_stack"]),
     "ce_fp8_scale_dropped": ("head_logits_fp8", lambda orig: (lambda xq, Wq, a, b: orig(xq, Wq, 1.0, 1.0)),
                              ["test_ce_head_logits_fp8_bruteforce_and_exact_grid"]),
+    "quantise_x_scale_dropped": ("quantise_x", lambda orig: (lambda x, s: orig(x, 1.0)),
+                                 ["test_quantise_x_matches_library_and_amax"]),
+    "w1_cache_scales_swapped": ("w1_cache", lambda orig: (lambda W1: (lambda r: (r[0], r[2], r[1]))(orig(W1))),
+                                ["test_w1_cache_matches_library"]),
+    "up_proj_fp8_dequant_dropped": ("up_proj_fp8", lambda orig: (lambda xq, Wq, a, b: orig(xq, Wq, 1.0, 1.0)),
+                                    ["test_up_proj_fp8_bruteforce_and_exact_grid"]),
+    "linear_bwd_dw_transposed": ("linear_bwd", lambda orig: (lambda x, W, dY: (lambda r: (r[0], r[1].T.copy()))(orig(x, W, dY))),
+                                 ["test_linear_fp8_and_bwd_bruteforce"]),
+    "rmsnorm_eps_dropped": ("rmsnorm_fwd", lambda orig: _rmsnorm_no_eps,
+                            ["test_rmsnorm_constant_rows_and_autograd"]),
+    "residual_add_drops_out": ("residual_add", lambda orig: (lambda r, out: np.asarray(r).copy()),
+                               ["test_residual_add_rounds_the_fp32_sum"]),
+    "residual_add_truncates": ("residual_add", lambda orig: (lambda r, out: _trunc_bf16(ref.f32(ref.bf16_to_f64(r) + ref.bf16_to_f64(out)))),
+                               ["test_residual_add_rounds_the_fp32_sum"]),
+    "reduce_partials_skips_nan": ("reduce_partials", lambda orig: (lambda pa: np.float32(np.nanmax(pa)) if np.size(pa) else np.float32(0.0)),
+                                  ["test_reduce_partials_nan_and_empty"]),
+    "down_proj_bf16_w2_reversed": ("down_proj_bf16", lambda orig: (lambda post, W2: orig(post, np.asarray(W2)[::-1].copy())),
+                                   ["test_down_proj_bf16_bruteforce"]),
 }
+
+
+def _rmsnorm_no_eps(r):
+    R = ref.bf16_to_f64(r)
+    rstd = 1.0 / np.sqrt(np.mean(R * R, axis=1))
+    return ref.bf16_bits_from_f32(ref.f32(R * rstd[:, None])), ref.f32(rstd)
 
 
 def _ce_grad_no_onehot(y, tg, w, c, lse, g):

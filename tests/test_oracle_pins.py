@@ -384,11 +384,15 @@ def test_backward_exact_integers_and_finite_differences():
 # ---------------------------------------------------------------------------
 
 def test_rmsnorm_constant_rows_and_autograd():
-    r = _bf16(np.array([[3.0] * 8, [-0.5] * 8], np.float32))
+    # a constant row c normalises to c / sqrt(c^2 + eps); at c ~ 1e-3 the
+    # eps = 1e-6 term halves the mean square's reciprocal
+    r = _bf16(np.array([[3.0] * 8, [-0.5] * 8, [1e-3] * 8], np.float32))
     x, _ = ref.rmsnorm_fwd(r)
     X = ref.bf16_to_f64(x)
     np.testing.assert_allclose(X[0], 3 / np.sqrt(9 + 1e-6), rtol=2 ** -8)
     np.testing.assert_allclose(X[1], -0.5 / np.sqrt(0.25 + 1e-6), rtol=2 ** -8)
+    c = ref.bf16_to_f64(r)[2, 0]
+    np.testing.assert_allclose(X[2], c / np.sqrt(c * c + 1e-6), rtol=2 ** -8)
     g = np.random.default_rng(12)
     r = _bf16(g.standard_normal((6, 16)))
     dx = _bf16(g.standard_normal((6, 16)))
@@ -396,6 +400,30 @@ def test_rmsnorm_constant_rows_and_autograd():
     y = R * torch.rsqrt(R.pow(2).mean(dim=1, keepdim=True) + 1e-6)
     y.backward(torch.tensor(ref.bf16_to_f64(dx)))
     np.testing.assert_allclose(ref.rmsnorm_bwd(r, dx), R.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_residual_add_rounds_the_fp32_sum():
+    # BF16 has 7 stored mantissa bits: next to 1.0 a step is 2^-7
+    r = _bf16(np.array([[1.0, 1.0, 1.0, -2.0]], np.float32))
+    o = _bf16(np.array([[2.0 ** -9, 2.0 ** -8, 3 * 2.0 ** -8, 2.0 ** -7]], np.float32))
+    got = ref.bf16_to_f64(ref.residual_add(r, o))[0]
+    # below half a step: down; a tie: to even (1.0); 1.5 steps: the tie goes
+    # to the even neighbour 1 + 2^-6; -2 + 2^-7 = -1.9921875 is representable
+    assert list(got) == [1.0, 1.0, 1.0 + 2.0 ** -6, -2.0 + 2.0 ** -7]
+    g = np.random.default_rng(14)
+    a, b = _bf16(g.standard_normal((32, 40))), _bf16(g.standard_normal((32, 40)) * 0.01)
+    want = (torch.tensor(ref.bf16_to_f64(a), dtype=torch.float32) + torch.tensor(ref.bf16_to_f64(b), dtype=torch.float32))
+    want = want.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ref.residual_add(a, b), want)
+
+
+def test_down_proj_bf16_bruteforce():
+    g = np.random.default_rng(15)
+    post = _bf16(np.abs(g.standard_normal((5, 12))))
+    W2 = _bf16(g.standard_normal((12, 7)))
+    got = ref.bf16_to_f64(ref.down_proj_bf16(post, W2))
+    want = _brute(ref.bf16_to_f64(post), ref.bf16_to_f64(W2).T)
+    np.testing.assert_allclose(got, want, rtol=2 ** -8)
 
 
 # ---------------------------------------------------------------------------
