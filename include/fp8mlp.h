@@ -175,6 +175,7 @@ int fp8mlp_mlp_fwd(int M, int d, int h, const uint16_t* x, const uint16_t* W1, c
  * fp8mlp_amax_reduce_update_scale into st_x for the next step). */
 int fp8mlp_quantize_x(int M, int d, const uint16_t* x, const fp8mlp_scale_state* st_x, uint8_t* x_fp8,
                       float* partial_amax_x, fp8mlp_stream_t stream);
+/* Entries of fp8mlp_quantize_x's partial_amax_x: ceil(M*d / 8192). */
 int fp8mlp_x_partial_amax_count(int M, int d);
 
 /* Exact FP8 copy of W1 (not transposed; W1 [h,d] is K-major for the
@@ -464,6 +465,7 @@ int fp8mlp_set_wait_timeout_ns(unsigned long long ns);
 #define FP8MLP_DEBUG_STALL_PRODUCER 1
 int fp8mlp_set_debug_flags(int flags);
 
+/* Static text of a return code. */
 const char* fp8mlp_error_string(int code);
 /* Text of the last error on this thread (empty if none). */
 const char* fp8mlp_last_error_detail(void);
