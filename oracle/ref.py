@@ -27,7 +27,7 @@ Sources, cited by page title and section:
          refresh is viable; BF16 post is kept for backward; amax(t-1) with a
          margin instead of a rolling window.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
   * scale s = 448 / (margin * amax), 448 being the largest finite e4m3 value;
   * the FP8 copy quantises the BF16-rounded post;
   * amax/scale keep the previous value when amax is zero or not finite;
@@ -514,7 +514,7 @@ def linear_bwd(x, W, dY):
 #         through an FP8 soft-capped cross-entropy kernel.
 #   [R83-1] "NanoGPT Speedrun (Track 1)", Changes vs Record #83, item 1: the
 #         earlier record ran FP8 only in the LM head.
-# Readings where the pages are silent (each also listed in the design doc):
+# Readings where the pages are silent:
 #   * softcap z = c * tanh(y / c), c > 0 (a cap of the form 2c * sigmoid(y/c')
 #     differs from it by a per-row constant, which cross-entropy ignores);
 #   * T targets per position, weights w_t; a target outside [0, V) is ignored;
