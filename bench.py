@@ -39,6 +39,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "ReLU² MLP fwd+bwd tokens/s and % of FP8/BF16 roofline at d=768,h=3072"
+FWD_METRIC = "ReLU² MLP fwd tokens/s and % of FP8/BF16 roofline at d=768,h=3072"
 LINEAR_METRIC = "FP8 linear (attention QKV projection) fwd+bwd tokens/s and % of FP8/BF16 roofline"
 CE_METRIC = "softcapped cross-entropy LM head fwd+bwd tokens/s and % of FP8/BF16 roofline at d=768,V=50304"
 CE_CAP = 15.0
@@ -50,7 +51,8 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="step16k", choices=["step16k", "train49k", "heavytail", "stack9", "qkv16k", "ce16k"])
+    ap.add_argument("--workload", default="step16k",
+                    choices=["step16k", "fwd16k", "train49k", "heavytail", "stack9", "qkv16k", "ce16k"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -281,6 +283,14 @@ def oracle_step_timer(W, tokens, seed=0, fp8_up=False):
         return step, threads
     P = synth.make_problem(tokens, W.d, W.h, seed=seed)
     st = {"s": ref.scale_state_init(W.margin, 1.0)}
+    if not W.backward:
+        W2q_t, _, s_wi = ref.w2_cache(P["W2"])
+
+        def step():  # forward with the delayed scale, then the scale update
+            f = ref.forward(P["x"], P["W1"], W2q_t, s_wi, st["s"]["scale"], st["s"]["scale_inv"])
+            st["s"] = ref.scale_update(st["s"], f["amax"])
+            return np
+        return step, threads
 
     def step():
         W2q_t, s_w, s_wi = ref.w2_cache(P["W2"])
@@ -301,6 +311,8 @@ def oracle_tokens(W, kind):
 
 
 def metric_of(W):
+    if not W.backward:
+        return FWD_METRIC
     if W.name.startswith("ce"):
         return CE_METRIC
     if W.name.startswith("qkv"):
@@ -340,7 +352,7 @@ def cpu_baseline(W, seconds, tokens=None, fp8_up=False):
                        if W.name.startswith("ce") else "") +
                       f"{reps} oracle steps of {tokens} tokens of the {W.name} workload "
                       f"(d={W.d}, {'V' if W.name.startswith('ce') else 'h'}={W.h}, {W.layers} layer(s); "
-                      f"the whole fwd+bwd step), {el:.1f} s"}
+                      f"the whole {'fwd+bwd' if W.backward else 'forward'} step), {el:.1f} s"}
 
 
 def run_reference(a, W, world, rank):
@@ -682,6 +694,148 @@ def run_dp(a, W, world, rank, local_rank, blk, flush, dist, peaks, fp8_peak, fp8
     dist.barrier()
     dist.destroy_process_group()
     return None
+
+
+def run_fwd(a, W, world, rank, local_rank):
+    """The forward alone (inference with delayed scaling): per step the fused
+    BF16 up-projection (post, its e4m3 copy, partial amax), the e4m3
+    down-projection and the scale update for the next step; one CUDA graph
+    per step.  The weights do not change, so the W2 cache is refreshed once."""
+    import numpy as np
+    import torch
+    from fp8_relu_mlp_b200 import _abi as A
+    from fp8_relu_mlp_b200 import synth
+    from fp8_relu_mlp_b200.block import MLPBlock
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local_rank)  # before the communicator binds a device
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    A.fp8mlp_set_programmatic_launch(not a.no_pdl)
+    M, d, h = W.M, W.d, W.h
+    peaks = load_peaks()
+    fp8_peak, fp8_src = measure_fp8_peak(torch, peaks["bf16_tflops"])
+    blk = MLPBlock(M, d, h, device=dev, margin=W.margin, with_backward=False)
+    P = synth.make_problem(M, d, h, seed=rank, x_dist=W.x_dist)
+    for k in ("x", "W1", "W2"):
+        getattr(blk, k).copy_(MLPBlock.bits_to_bf16(P[k], dev))
+    blk.refresh_w2_cache()
+    blk.calibrate()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    npa = blk.partial_amax.numel()
+
+    def step(ev=None, bufs=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record()
+        xb, ob = bufs if bufs is not None else (blk.x, blk.out)
+        mark(0)
+        A.fp8mlp_up_proj_fused(M, d, h, xb, blk.W1, blk.state, blk.post, blk.post_fp8, blk.partial_amax)
+        mark(1)
+        A.fp8mlp_down_proj_fp8(M, d, h, blk.post_fp8, blk.W2q_t, blk.w2_scale_inv, blk.state, ob)
+        mark(2)
+        A.fp8mlp_amax_reduce_update_scale(blk.partial_amax, npa, blk.state)
+        mark(3)
+
+    step()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True, external=not a.eager) for _ in range(4)]
+    n_cap0 = A.fp8mlp_kernel_launch_count()
+    graph = None
+    if not a.eager:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step(ev)
+    kps = A.fp8mlp_kernel_launch_count() - n_cap0 if graph is not None else 3
+
+    def run():
+        graph.replay() if graph is not None else step(ev)
+
+    for _ in range(max(a.warmup, 3)):
+        flush.zero_()
+        run()
+    torch.cuda.synchronize()
+    A.fp8mlp_clear_device_status()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms, up_ms, down_ms = [], [], []
+    with ClockSampler(local_rank) as clk:
+        for _ in range(a.steps):
+            flush.zero_()
+            run()
+            ev[3].synchronize()
+            step_ms.append(ev[0].elapsed_time(ev[3]))
+            up_ms.append(ev[0].elapsed_time(ev[1]))
+            down_ms.append(ev[1].elapsed_time(ev[2]))
+    status = A.fp8mlp_get_device_status()
+    total_s = sum(step_ms) * 1e-3
+    if dist:
+        t = torch.tensor([total_s], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_s = float(t.item())
+    work = kernel_work(M, d, h)
+    up_s = statistics.mean(up_ms) * 1e-3
+    achieved = work["up_fused"]["bf16"] / up_s / 1e12
+    roof = sum(max(work[k]["bf16"] / (peaks["bf16_tflops"] * 1e12) + work[k]["fp8"] / (fp8_peak * 1e12),
+                   work[k]["bytes"] / (peaks["hbm_gbs"] * 1e9)) for k in ("up_fused", "down_fp8", "amax_scale"))
+    e2e = None
+    if not a.no_e2e:
+        # x in from pinned host memory and out back, every step; copies
+        # overlapped with the neighbouring steps (two device buffer sets)
+        from fp8_relu_mlp_b200.hostio import HostPipeline
+        xh = blk.x.cpu().pin_memory()
+        oh = torch.empty_like(blk.out, device="cpu").pin_memory()
+        sets = [(blk.x, blk.out), (blk.x.clone(), torch.empty_like(blk.out))]
+        pipe = HostPipeline(lambda k: step(bufs=sets[k]), [[sb[0]] for sb in sets], [[sb[1]] for sb in sets],
+                            device=dev, graph=not a.eager)
+        pipe.run([xh], [oh], max(a.warmup, 3))
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        timer = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        pipe.run([xh], [oh], a.steps, timer)
+        timer[1].synchronize()
+        te = timer[0].elapsed_time(timer[1]) * 1e-3
+        if dist:
+            tt = torch.tensor([te], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            te = float(tt.item())
+        e2e = {"value": M * world * a.steps / te, "unit": "tokens/s",
+               "h2d_bytes_per_step": int(2 * xh.numel()), "d2h_bytes_per_step": int(2 * oh.numel()),
+               "overlap": "copies on two streams beside the compute, double-buffered device sets",
+               "copy_bound": {"value": copy_bound(torch, dev, [xh], [oh], M * world), "unit": "tokens/s",
+                              "note": "the same pinned copies alone, both directions at once (this rank's link)"}}
+    if rank == 0:
+        line = {
+            "metric": FWD_METRIC,
+            "value": M * world * a.steps / total_s, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup,
+            "ms_per_step": total_s / a.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 up-projection, e4m3 down-projection (fp32 accumulate)",
+            "data": "synthetic (seeded; shapes of the 768-dim GPT-2-small / nanochat MLP)",
+            "config": dict(config_of(W), parallelism=f"dp{world} replicas" if world > 1 else "single GPU"),
+            "roofline": {"bound": "tensor", "kernel": "up_fused", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "traffic": load_traffic(W.name).get("up_fused"),
+                         "peak_source": "bf16_tflops burst of measured peaks"},
+            "step_roofline": {"roofline_ms": roof * 1e3, "measured_ms": total_s / a.steps * 1e3,
+                              "frac": roof / (total_s / a.steps), "peaks": {**peaks, "fp8_tflops": fp8_peak}},
+            "kernels_ms": {"up_fused": statistics.median(up_ms), "down_fp8": statistics.median(down_ms)},
+            "clocks": clk.summary(), "gpu_launches": int(kps * a.steps), "device_status": status,
+            "launch_mode": "eager" if graph is None else "cuda_graph",
+        }
+        if e2e is not None:
+            line["e2e"] = e2e
+        if not a.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(W, a.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 def run_linear(a, W, world, rank, local_rank):
@@ -1422,7 +1576,9 @@ def main():
         if rank == 0:
             run_compare_library(a, W)
         return 0
-    if W.name.startswith("qkv"):
+    if not W.backward:
+        run_fwd(a, W, world, rank, local_rank)
+    elif W.name.startswith("qkv"):
         run_linear(a, W, world, rank, local_rank)
     elif W.name.startswith("ce"):
         run_ce(a, W, world, rank, local_rank)

@@ -12,7 +12,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 @pytest.mark.timeout(300)
-@pytest.mark.parametrize("workload", ["step16k", "qkv16k"])
+@pytest.mark.parametrize("workload", ["step16k", "fwd16k", "qkv16k"])
 def test_reference_arm_json_line(workload):
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
                         "--warmup", "1", "--workload", workload],

@@ -55,3 +55,15 @@ def test_bench_line_ce16k_small():
     assert d["config"]["workload"].startswith("ce16k") and d["value"] > 0
     assert d["roofline"]["kernel"] in ("ce_fwd", "ce_bwd_dlogits", "dx", "dw")
     assert d["gpu_launches"] > 0 and d["device_status"] == 0
+
+
+@pytest.mark.timeout(900)
+def test_bench_line_fwd16k():
+    d = _run("--workload", "fwd16k", "--steps", "5", "--warmup", "3", "--cpu-seconds", "2")
+    assert d["config"]["workload"].startswith("fwd16k") and d["value"] > 0
+    assert d["roofline"]["kernel"] == "up_fused" and 0 < d["roofline"]["frac"] < 1.3
+    e = d["e2e"]
+    assert e["h2d_bytes_per_step"] == 16384 * 768 * 2 and e["d2h_bytes_per_step"] == 16384 * 768 * 2
+    assert 0 < e["value"] <= 1.1 * e["copy_bound"]["value"]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["gpu_launches"] >= 3 * d["steps"]
+    assert d["device_status"] == 0
