@@ -608,29 +608,30 @@ int fp8mlp_linear_bwd(int M, int K, int N, const uint16_t* x, const uint16_t* W,
   REQUIRE_PTR(x);
   REQUIRE_PTR(W);
   REQUIRE_PTR(dY);
+  if (dX != nullptr) REQUIRE_PTR(dX);
+  if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 15u))
+    return fail(FP8MLP_ERR_INVALID_ARG, "workspace misaligned");
   DeviceInfo* di = nullptr;
   TRY(current_device(&di));
+  // both launches are set up (and their tensor maps checked) before either
+  // is enqueued
+  // dX[M,K] = dY[M,N] . W[N,K]: contraction over N, W as an MN-major B operand
+  GemmParams px{};
   if (dX != nullptr) {
-    REQUIRE_PTR(dX);
-    // dX[M,K] = dY[M,N] . W[N,K]: contraction over N, W as an MN-major B operand
-    GemmParams p{};
-    TRY(map_kmajor(&p.tmA[0], dY, BF16, 2, M, N, kGemmBM, "dY"));
-    TRY(map_mnmajor(&p.tmB[0], W, N, K, "W"));
-    TRY(map_tile32(&p.tmOut[0], dX, BF16, 2, M, K, "dX"));
-    fill_common(p, GemmKind::Bf16MnB, di, M, K, N, 1);
-    p.launch_flags = flags;
-    TRY(launch(GemmKind::Bf16MnB, p, di, stream, "linear_bwd dX launch"));
+    TRY(map_kmajor(&px.tmA[0], dY, BF16, 2, M, N, kGemmBM, "dY"));
+    TRY(map_mnmajor(&px.tmB[0], W, N, K, "W"));
+    TRY(map_tile32(&px.tmOut[0], dX, BF16, 2, M, K, "dX"));
+    fill_common(px, GemmKind::Bf16MnB, di, M, K, N, 1);
+    px.launch_flags = flags;
   }
-  // dW[N,K] = dY^T . x: contraction over the M tokens, both operands MN-major
-  GemmParams p{};
-  // with few output tiles (a third of the CTA pairs for 768 -> 2304) and a
+  // dW[N,K] = dY^T . x: contraction over the M tokens, both operands MN-major.
+  // With few output tiles (a third of the CTA pairs for 768 -> 2304) and a
   // workspace, the tokens are split in two: rows [0, M0) accumulate into dW,
   // rows [M0, M) into the workspace (the second group of one launch), and
   // the workspace is added to dW afterwards, in that order
+  GemmParams p{};
   const int tiles = cdiv(N, kGemmBN) * cdiv(K, kGemmBN);
   const bool split = workspace != nullptr && M >= 2 * kLinearSplitRows && 2 * tiles <= di->num_sms / 2;
-  if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 15u))
-    return fail(FP8MLP_ERR_INVALID_ARG, "workspace misaligned");
   const int M0 = split ? cdiv(cdiv(M, 2), kLinearSplitRows) * kLinearSplitRows : M;
   TRY(map_mnmajor(&p.tmA[0], dY, M0, N, "dY"));
   TRY(map_mnmajor(&p.tmB[0], x, M0, K, "x"));
@@ -643,6 +644,7 @@ int fp8mlp_linear_bwd(int M, int K, int N, const uint16_t* x, const uint16_t* W,
   fill_common(p, GemmKind::DW, di, N, K, M0, split ? 2 : 1);
   // dW neither reads dX nor writes what dX reads: it may overlap its tail
   p.launch_flags = dX != nullptr ? FP8MLP_LAUNCH_OVERLAP_PREVIOUS : flags;
+  if (dX != nullptr) TRY(launch(GemmKind::Bf16MnB, px, di, stream, "linear_bwd dX launch"));
   TRY(launch(GemmKind::DW, p, di, stream, "linear_bwd dW launch"));
   if (!split) return FP8MLP_OK;
   const cudaError_t e =

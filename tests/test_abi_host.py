@@ -86,6 +86,18 @@ def test_launch_flag_checks():
     assert _rc("fp8mlp_bwd_dw", 16, 64, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, None) == A.ERR_INVALID_ARG
 
 
+def test_linear_bwd_checks_before_enqueueing():
+    # host-side checks (pointers, dX alignment, workspace alignment) come
+    # before the device query, so they answer without a GPU
+    args = [300, 768, 2304, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, None]
+    for pos, bad in ((3, None), (4, FAKE + 8), (5, None), (6, FAKE + 4), (8, FAKE + 8)):
+        a = list(args)
+        a[pos] = bad
+        assert _rc("fp8mlp_linear_bwd", *a) == A.ERR_INVALID_ARG, pos
+    assert A.fp8mlp_linear_bwd_workspace_size(300, 768, 2304) == 4 * 768 * 2304
+    assert A.fp8mlp_linear_bwd_workspace_size(100, 768, 2304) == 0
+
+
 def test_scale_state_init_checks():
     assert _rc("fp8mlp_scale_state_init", FAKE, ctypes.c_float(0.0), ctypes.c_float(1.0), None) == A.ERR_INVALID_ARG
     assert _rc("fp8mlp_scale_state_init", FAKE, ctypes.c_float(2.0), ctypes.c_float(-1.0), None) == A.ERR_INVALID_ARG
