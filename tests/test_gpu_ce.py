@@ -31,6 +31,7 @@ SHAPES = [  # (M, d, V, T): ragged rows, columns and vocabulary tiles
     (256, 64, 256, 1),
     (1, 64, 16, 1),
     (513, 768, 4096, 2),
+    (200, 96, 528, 4),    # the most targets per row; d and V end inside a block
 ]
 WEIGHTS = [1.0, 0.5, 0.25, 0.125]
 

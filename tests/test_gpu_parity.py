@@ -1119,3 +1119,11 @@ def test_linear_fp8_fwd_bwd_normal(M, K, N, split):
         want = np.array([G[:, i] @ X[:, j] for i, j in pairs])
         assert rel_fro(got, want) < TOL_GRAD
     assert y.intact() and dX.intact() and dW.intact()
+
+
+def test_smoke_entry_point():
+    """The entry point the driver runs: one small training step through the
+    C ABI on cuda:0, checked against the oracle inside."""
+    import __graft_entry__
+    __graft_entry__.smoke()
+    assert A.fp8mlp_get_device_status() == 0
