@@ -97,9 +97,51 @@ MUTATIONS = {
                                ["test_residual_add_rounds_the_fp32_sum"]),
     "reduce_partials_skips_nan": ("reduce_partials", lambda orig: (lambda pa: np.float32(np.nanmax(pa)) if np.size(pa) else np.float32(0.0)),
                                   ["test_reduce_partials_nan_and_empty"]),
+    # the sampled evaluators of the full-size GPU tests
+    "forward_rows_takes_leading_rows": ("forward_rows",
+                                        lambda orig: (lambda rows, *a: orig(np.arange(len(rows)), *a)),
+                                        ["test_forward_rows_equal_whole_batch"]),
+    "dx_rows_dout_not_sliced": ("dx_rows", lambda orig: _dx_rows_dout_prefix,
+                                ["test_dx_rows_equal_whole_batch"]),
+    "dpre_column_reads_w2_column": ("dpre_column",
+                                    lambda orig: (lambda i, pc, dOut, W2: orig(i, pc, dOut, np.asarray(W2).T.copy())),
+                                    ["test_post_and_dpre_columns_equal_whole_batch"]),
+    "dpre_column_factor_two_dropped": ("dpre_column", lambda orig: _dpre_column_no_two,
+                                       ["test_post_and_dpre_columns_equal_whole_batch"]),
+    "post_column_off_by_one": ("post_column",
+                               lambda orig: (lambda i, x, W1: orig((i + 1) % np.shape(W1)[0], x, W1)),
+                               ["test_post_and_dpre_columns_equal_whole_batch"]),
+    "dw_entries_dw2_from_dpre": ("dw_entries", lambda orig: _dw_entries_mut("dw2_dpre"),
+                                 ["test_dw_entries_equal_whole_batch"]),
+    "dw_entries_dw1_reads_dout": ("dw_entries", lambda orig: _dw_entries_mut("dw1_dout"),
+                                  ["test_dw_entries_equal_whole_batch"]),
     "down_proj_bf16_w2_reversed": ("down_proj_bf16", lambda orig: (lambda post, W2: orig(post, np.asarray(W2)[::-1].copy())),
                                    ["test_down_proj_bf16_bruteforce"]),
 }
+
+
+def _dx_rows_dout_prefix(rows, x, W1, W2, dOut):
+    post = ref.relu2_post(ref.up_proj(x[rows], W1))
+    dPre = ref.bwd_dpre(post, dOut[:len(rows)], W2)
+    return dPre, ref.bwd_dx(dPre, W1)
+
+
+def _dpre_column_no_two(i, post_col, dOut, W2):
+    dPost = ref.bf16_to_f64(dOut) @ ref.bf16_to_f64(W2[i])
+    return ref.bf16_bits_from_f32(ref.f32(np.sqrt(ref.bf16_to_f64(post_col)) * dPost))
+
+
+def _dw_entries_mut(kind):
+    def f(pairs, x, W1, W2, dOut):
+        X, G = ref.bf16_to_f64(x), ref.bf16_to_f64(dOut)
+        o1, o2 = [], []
+        for i, j in pairs:
+            pc = ref.post_column(i, x, W1)
+            dc = ref.dpre_column(i, pc, dOut, W2)
+            o1.append(np.float32(ref.bf16_to_f64(dc) @ (G if kind == "dw1_dout" else X)[:, j]))
+            o2.append(np.float32(ref.bf16_to_f64(dc if kind == "dw2_dpre" else pc) @ G[:, j]))
+        return np.array(o1, np.float32), np.array(o2, np.float32)
+    return f
 
 
 def _rmsnorm_no_eps(r):
@@ -132,7 +174,12 @@ def _ce_targets_clipped(targets, weights, V):
 
 PARAMS = {"test_e4m3_exhaustive_over_bf16": dict(s=3.7),
           "test_scale_update_closed_form": dict(A=3.0, margin=2.0),
-          "test_scale_keeps_previous_on_degenerate_amax": dict(A=0.0)}
+          "test_scale_keeps_previous_on_degenerate_amax": dict(A=0.0),
+          # the square case: a transposed operand has the right shape
+          "test_forward_rows_equal_whole_batch": dict(M=130, d=96, h=96),
+          "test_dx_rows_equal_whole_batch": dict(M=130, d=96, h=96),
+          "test_post_and_dpre_columns_equal_whole_batch": dict(M=130, d=96, h=96),
+          "test_dw_entries_equal_whole_batch": dict(M=130, d=96, h=96)}
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))

@@ -790,3 +790,68 @@ def test_ce_closed_form_at_exact_tanh_points():
     want = np.array([[(1.5 * p0[0] - 1.0) * 0.75, 1.5 * p0[1], (1.5 * p0[2] - 0.5) * 0.75],
                      [1 / 3, 1 / 3 - 1.0, 1 / 3]])
     np.testing.assert_allclose(ref.ce_backward_dlogits(y, tg, w, 2.0, f["lse"], 1.0), want, rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# Sampled evaluators.  The full-size GPU tests take their expected values from
+# forward_rows, dx_rows, post_column, dpre_column and dw_entries, which
+# evaluate the block's definitions at chosen rows, columns or entries.  Here
+# they are held, bit for bit, to the whole-batch functions above (forward,
+# backward, relu2_post of up_proj), which the pins in this file tie to
+# libraries, brute force and closed forms.  A square case (d == h) makes a
+# transposed operand shape-compatible, so only the values can catch it.
+# ---------------------------------------------------------------------------
+
+SAMPLED_SHAPES = [(300, 64, 256), (130, 96, 96)]
+
+
+def _whole_batch(M, d, h, seed):
+    from fp8_relu_mlp_b200 import synth
+    P = synth.make_problem(M, d, h, seed=seed)
+    W2q, _, s_wi = ref.w2_cache(P["W2"])
+    post = ref.relu2_post(ref.up_proj(P["x"], P["W1"]))
+    st = ref.scale_update(ref.scale_state_init(2.0, 1.0), ref.amax(post))
+    f = ref.forward(P["x"], P["W1"], W2q, s_wi, st["scale"], st["scale_inv"])
+    b = ref.backward(P["x"], P["W1"], P["W2"], f["post"], P["dOut"])
+    return P, W2q, s_wi, st, f, b
+
+
+def _rows(M):
+    # unsorted, with both ends and a repeat-free middle
+    return np.array([M - 1, 0, 7, M // 2, 3, M - 2])
+
+
+@pytest.mark.parametrize("M,d,h", SAMPLED_SHAPES)
+def test_forward_rows_equal_whole_batch(M, d, h):
+    P, W2q, s_wi, st, f, _ = _whole_batch(M, d, h, seed=31)
+    rows = _rows(M)
+    fr = ref.forward_rows(rows, P["x"], P["W1"], W2q, s_wi, st["scale"], st["scale_inv"])
+    for k in ("post", "q", "out"):
+        assert np.array_equal(fr[k], f[k][rows]), k
+
+
+@pytest.mark.parametrize("M,d,h", SAMPLED_SHAPES)
+def test_dx_rows_equal_whole_batch(M, d, h):
+    P, _, _, _, f, b = _whole_batch(M, d, h, seed=32)
+    rows = _rows(M)
+    dPre, dX = ref.dx_rows(rows, P["x"], P["W1"], P["W2"], P["dOut"])
+    assert np.array_equal(dPre, b["dPre"][rows])
+    assert np.array_equal(dX, b["dX"][rows])
+
+
+@pytest.mark.parametrize("M,d,h", SAMPLED_SHAPES)
+def test_post_and_dpre_columns_equal_whole_batch(M, d, h):
+    P, _, _, _, f, b = _whole_batch(M, d, h, seed=33)
+    for i in (0, 5, h // 2, h - 1):
+        pc = ref.post_column(i, P["x"], P["W1"])
+        assert np.array_equal(pc, f["post"][:, i]), i
+        assert np.array_equal(ref.dpre_column(i, pc, P["dOut"], P["W2"]), b["dPre"][:, i]), i
+
+
+@pytest.mark.parametrize("M,d,h", SAMPLED_SHAPES)
+def test_dw_entries_equal_whole_batch(M, d, h):
+    P, _, _, _, _, b = _whole_batch(M, d, h, seed=34)
+    pairs = [(0, 0), (h - 1, d - 1), (5, d - 1), (h // 2, 3), (h - 1, 0), (7, 11)]
+    w1, w2 = ref.dw_entries(pairs, P["x"], P["W1"], P["W2"], P["dOut"])
+    assert np.array_equal(w1, np.array([b["dW1"][i, j] for i, j in pairs]))
+    assert np.array_equal(w2, np.array([b["dW2"][i, j] for i, j in pairs]))
