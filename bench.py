@@ -16,9 +16,13 @@ breakdown comes from separate untimed steps.  ``e2e`` repeats the measurement th
 with the step's inputs copied in from pinned host memory and its results
 (out, dX) copied back, inside the timed region.
 
-Multi-GPU (torchrun, one process per GPU): every rank runs its own batch
-(weak scaling, data-parallel replicas, no collective on the data path); the
-time is the max over ranks.  Rank 0 prints one JSON line.
+Multi-GPU: one process per GPU under torchrun; ``--gpus N`` run without a
+torchrun environment starts the N ranks itself (and ``--gpus N`` under a
+different WORLD_SIZE is an error, so a scaling run cannot silently time one
+GPU).  Every rank runs its own batch of M tokens (weak scaling): by default
+the data-parallel step (partial amax all-reduced with MAX, dW1/dW2
+all-reduced on a side stream beside dX), ``--replicas`` for independent
+replicas; the time is the max over ranks.  Rank 0 prints one JSON line.
 
 ``--impl reference`` times the CPU oracle on the host cores on a bounded
 sample of the same workload (rank 0 only; other ranks exit 0).
@@ -371,7 +375,7 @@ def run_reference(a, W, world, rank):
     if W.name.startswith("ce"):
         sample += (f"; each step also re-quantises {tokens}/{W.M} of the head's rows, its share of the "
                    f"once-per-step weight-cache refresh")
-    line = {"metric": metric_of(W), "value": v, "unit": "tokens/s", "n_gpus": a.gpus, "steps": a.steps,
+    line = {"metric": metric_of(W), "value": v, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": el / a.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64 (bf16/e4m3 rounding emulated)", "data": "synthetic",
             "config": config_of(W), "impl": "reference",
@@ -1557,6 +1561,20 @@ def measure_e2e(a, blk, P, torch, dev, stream, M, world, dist, step_fn=None):
                            "note": "the same pinned copies alone, both directions at once (this rank's link)"}}
 
 
+def relaunch(n):
+    """--gpus N > 1 outside a torchrun environment: start N ranks of this same
+    command, one process per GPU on this node, rendezvous on 127.0.0.1, and
+    return the exit status of the launcher (non-zero if any rank failed)."""
+    import socket
+    import subprocess
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.run(cmd).returncode
+
+
 def main():
     a = parse()
     from fp8_relu_mlp_b200 import synth
@@ -1566,7 +1584,14 @@ def main():
         # traffic figures are per full-size launch, so they are not looked up
         import dataclasses
         W = dataclasses.replace(W, M=a.tokens, name=f"{W.name}@{a.tokens}")
+    if "WORLD_SIZE" not in os.environ and a.gpus > 1:
+        return relaunch(a.gpus)
     world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != a.gpus:
+        print(f"bench.py: --gpus {a.gpus} but WORLD_SIZE={world}: launch one rank per GPU "
+              f"(torchrun --nproc-per-node {a.gpus}), or run without WORLD_SIZE set and bench.py starts them",
+              file=sys.stderr, flush=True)
+        return 2
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if a.impl == "reference":

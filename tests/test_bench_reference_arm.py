@@ -28,3 +28,30 @@ def test_reference_arm_json_line(workload):
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["workload"].startswith(workload)
+
+
+@pytest.mark.timeout(120)
+def test_gpus_flag_disagreeing_with_world_size_is_refused():
+    """--gpus 2 in a one-rank environment must not print a one-GPU line."""
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "1"], capture_output=True, text=True, cwd=ROOT, env=env,
+                       timeout=100)
+    assert r.returncode != 0
+    assert not [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert "WORLD_SIZE=1" in r.stderr
+
+
+@pytest.mark.timeout(300)
+def test_gpus_flag_starts_one_rank_per_gpu():
+    """--gpus 2 without torchrun's environment starts two ranks (rendezvous on
+    127.0.0.1); the reference arm runs on rank 0 and reports n_gpus = 2."""
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "1", "--workload", "fwd16k"],
+                       capture_output=True, text=True, cwd=ROOT, env=env, timeout=280)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2
