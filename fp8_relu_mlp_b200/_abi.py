@@ -37,6 +37,7 @@ CE_SUM = 0
 CE_MEAN = 1
 LAUNCH_OVERLAP_PREVIOUS = 1
 DEBUG_STALL_PRODUCER = 1
+DEBUG_STALL_AUX = 2
 E4M3_MAX = 448.0
 
 
@@ -56,6 +57,7 @@ _SIGS = {
     "fp8mlp_down_proj_bf16": [_i, _i, _i, _p, _p, _p, _p],
     "fp8mlp_mlp_fwd": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _p],
     "fp8mlp_partial_amax_shape": [_i, _i, _p, _p, _p, _p],
+    "fp8mlp_partial_amax_count": [_i, _i],
     "fp8mlp_scale_state_init": [_p, _f, _f, _p],
     "fp8mlp_amax_reduce_update_scale": [_p, _i, _p, _p],
     "fp8mlp_w2_fp8_cache_refresh": [_i, _i, _p, _p, _p, _p, _p],
@@ -178,6 +180,10 @@ def fp8mlp_partial_amax_shape(M, h):
     v = [ctypes.c_int() for _ in range(4)]
     _call("fp8mlp_partial_amax_shape", M, h, *[ctypes.addressof(x) for x in v])
     return tuple(x.value for x in v)
+
+
+def fp8mlp_partial_amax_count(M, h):
+    return int(lib.fp8mlp_partial_amax_count(M, h))
 
 
 def fp8mlp_scale_state_init(st, margin, initial_scale, stream=None):

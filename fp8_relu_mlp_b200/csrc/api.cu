@@ -338,6 +338,13 @@ int fp8mlp_partial_amax_shape(int M, int h, int* row_blocks, int* col_blocks, in
   return FP8MLP_OK;
 }
 
+int fp8mlp_partial_amax_count(int M, int h) {
+  if (M < 0 || h < 0) return 0;
+  int rb = 0, cb = 0;
+  fp8mlp_partial_amax_shape(M, h, &rb, &cb, nullptr, nullptr);
+  return rb * cb;
+}
+
 size_t fp8mlp_workspace_size(int M, int d, int h) {
   (void)M;
   if (d <= 0 || h <= 0) return 256;
@@ -881,7 +888,8 @@ int fp8mlp_set_programmatic_launch(int enable) {
 }
 
 int fp8mlp_set_debug_flags(int flags) {
-  if (flags & ~FP8MLP_DEBUG_STALL_PRODUCER) return fail(FP8MLP_ERR_INVALID_ARG, "unknown debug flags");
+  if (flags & ~(FP8MLP_DEBUG_STALL_PRODUCER | FP8MLP_DEBUG_STALL_AUX))
+    return fail(FP8MLP_ERR_INVALID_ARG, "unknown debug flags");
   g_debug_flags.store(flags);
   return FP8MLP_OK;
 }

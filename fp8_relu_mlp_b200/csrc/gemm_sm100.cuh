@@ -452,6 +452,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
     uint32_t aux_issued = 0;
     uint8_t* aux_ring = sAux + e * C::AUX_WARP;
     uint64_t* my_auxb = auxb + e * C::NAUX;
+    // test hook: issue no loads of post, so that the waits for them run out
+    const bool stall_aux = (p.debug_flags & FP8MLP_DEBUG_STALL_AUX) != 0;
     auto tile_rows = [&](int tile) {  // first row of this warp's 32 rows in `tile`
       int mb2, nb2;
       tile_coords(p, tile - (tile / tiles_per_group) * tiles_per_group, mb2, nb2);
@@ -463,7 +465,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
       return nb2 * C::BN;
     };
     if constexpr (C::EPI == Epi::DPre) {
-      if (pair < num_tiles) {
+      if (pair < num_tiles && !stall_aux) {
         const int r0 = tile_rows(pair), c0 = tile_cols(pair);
         if (lane == 0) {
           for (int c = 0; c < C::NAUX; ++c) {
@@ -607,7 +609,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) gemm_sm100_kernel(const __grid_
             // chunk cw + NAUX of this tile, or of the next one)
             const int cw_n = cw + C::NAUX;
             const int t_n = cw_n < C::NCH_W ? t : next_tile;
-            if (t_n < num_tiles) {
+            if (t_n < num_tiles && !stall_aux) {
               const int cn = cw_n < C::NCH_W ? cw_n : cw_n - C::NCH_W;
               if (lane == 0) {
                 mbar_arrive_expect_tx(&my_auxb[slot_aux], C::AUX_CHUNK);

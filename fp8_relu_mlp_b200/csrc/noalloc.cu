@@ -8,7 +8,9 @@
 // calls can synchronise the whole device.  This entry point therefore takes
 // no workspace argument.  Its scratch -- one partial maximum of |W2| per
 // reduction block -- lives in the fixed array below, which every GPU that
-// loads the library holds until the process exits.
+// loads the library holds until the process exits.  It runs the same two
+// kernels as fp8mlp_w2_fp8_cache_refresh, with the array's address in place
+// of the workspace, so the two entry points give the same bits.
 //
 // The array is shared by every call on a device and keeps what the last
 // call wrote.  Nothing in it has to start at zero: each call writes every
@@ -26,97 +28,17 @@
 namespace fp8mlp {
 namespace {
 
-using namespace dev;
-
-constexpr int kScratchEntries = 2048;          // partial maxima the array holds
-constexpr int kElemsPerBlock = 8192;           // W2 elements one reduction block covers
-constexpr long long kMaxElems = static_cast<long long>(kScratchEntries) * kElemsPerBlock;  // 16,777,216
+constexpr int kScratchEntries = 2048;  // partial maxima the array holds
+// one partial maximum per kW2ElemsPerBlock (8192) elements of W2, as in the
+// workspace version, whose two kernels this entry point launches
+constexpr long long kMaxElems = static_cast<long long>(kScratchEntries) * kW2ElemsPerBlock;  // 16,777,216
+static_assert(kMaxElems == 16777216, "the documented limit");
 
 static __device__ __align__(256) unsigned int g_w2_partial_amax[kScratchEntries];
 
 constexpr int kMaxDev = 64;
 unsigned int* g_partial_ptr[kMaxDev] = {};
 std::mutex g_setup_mutex;
-
-// Block b writes max |W2| (as BF16 magnitude bits, whose integer order is
-// the value order, NaN above infinity) over elements [b*8192, (b+1)*8192).
-__global__ void __launch_bounds__(256) noalloc_w2_block_amax(const uint4* __restrict__ W, long long n_vec,
-                                                             unsigned int* __restrict__ partial) {
-  __shared__ unsigned int wmax[8];
-  const long long base = static_cast<long long>(blockIdx.x) * (kElemsPerBlock / 8);
-  unsigned int m = 0;
-#pragma unroll
-  for (int k = 0; k < kElemsPerBlock / 8 / 256; ++k) {
-    const long long i = base + k * 256 + threadIdx.x;
-    if (i < n_vec) {
-      const uint4 v = W[i];
-      const unsigned int w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        m = max(m, w4[j] & 0x7FFFu);
-        m = max(m, (w4[j] >> 16) & 0x7FFFu);
-      }
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    unsigned int r = 0;
-    for (int w = 0; w < 8; ++w) r = max(r, wmax[w]);
-    partial[blockIdx.x] = r;
-  }
-}
-
-// Every block reduces the partial maxima to s_w, then writes its 64x64 tile
-// of W2q_t[j, i] = e4m3(W2[i, j] * s_w).
-__global__ void __launch_bounds__(256) noalloc_w2_quant_t(int h, int d, const uint16_t* __restrict__ W2,
-                                                          uint8_t* __restrict__ W2q_t, float* w2_scale_inv,
-                                                          const unsigned int* __restrict__ partial, int nparts,
-                                                          unsigned int* status) {
-  __shared__ float tile[64][65];
-  __shared__ unsigned int wmax[8];
-  unsigned int m = 0;
-  for (int i = threadIdx.x; i < nparts; i += 256) m = max(m, partial[i]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
-  __syncthreads();
-  m = 0;
-  for (int w = 0; w < 8; ++w) m = max(m, wmax[w]);
-  const float a = __uint_as_float(m << 16);
-  const bool ok = isfinite(a) && a > 0.f;
-  const float s_w = ok ? __fdiv_rn(FP8MLP_E4M3_MAX, a) : 1.f;
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
-    w2_scale_inv[0] = __fdiv_rn(1.f, s_w);
-    if (!ok) atomicOr(status, STATUS_W2_DEGENERATE);
-  }
-  const int i0 = blockIdx.y * 64;  // rows of W2 (h)
-  const int j0 = blockIdx.x * 64;  // columns of W2 (d)
-  for (int t = threadIdx.x; t < 64 * 8; t += 256) {
-    const int r = t >> 3, c8 = (t & 7) * 8;
-    const int i = i0 + r, j = j0 + c8;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (i < h && j < d) v = *reinterpret_cast<const uint4*>(W2 + static_cast<size_t>(i) * d + j);
-    const unsigned int w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      tile[r][c8 + 2 * k] = bf16lo_to_f32(w4[k]);
-      tile[r][c8 + 2 * k + 1] = bf16hi_to_f32(w4[k]);
-    }
-  }
-  __syncthreads();
-  for (int t = threadIdx.x; t < 64 * 16; t += 256) {
-    const int jr = t >> 4, i4 = (t & 15) * 4;
-    const int j = j0 + jr, i = i0 + i4;
-    if (j < d && i < h) {
-      const uint32_t lo = pack_e4m3x2(__fmul_rn(tile[i4][jr], s_w), __fmul_rn(tile[i4 + 1][jr], s_w));
-      const uint32_t hi = pack_e4m3x2(__fmul_rn(tile[i4 + 2][jr], s_w), __fmul_rn(tile[i4 + 3][jr], s_w));
-      *reinterpret_cast<uint32_t*>(W2q_t + static_cast<size_t>(j) * h + i) = lo | (hi << 16);
-    }
-  }
-}
 
 int noalloc_fail(int code, const char* what) {
   set_error_detail(what);
@@ -163,17 +85,9 @@ extern "C" int fp8mlp_w2_fp8_cache_refresh_noalloc(int h, int d, const uint16_t*
     }
     partial = g_partial_ptr[dev];
   }
-  const long long n = static_cast<long long>(h) * d;
-  const int nparts = static_cast<int>((n + kElemsPerBlock - 1) / kElemsPerBlock);
-  cudaStream_t s = stream;
-  noalloc_w2_block_amax<<<nparts, 256, 0, s>>>(reinterpret_cast<const uint4*>(W2), n / 8, partial);
-  count_launches(1);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return noalloc_fail(FP8MLP_ERR_CUDA, cudaGetErrorString(e));
-  dim3 grid((d + 63) / 64, (h + 63) / 64);
-  noalloc_w2_quant_t<<<grid, 256, 0, s>>>(h, d, W2, W2q_t, w2_scale_inv, partial, nparts, di->status);
-  count_launches(1);
-  e = cudaGetLastError();
+  // the two kernels of fp8mlp_w2_fp8_cache_refresh, with the fixed array in
+  // place of the caller's workspace: the results are the same bits
+  const cudaError_t e = launch_w2_cache(h, d, W2, W2q_t, w2_scale_inv, partial, di->status, di->num_sms, stream);
   if (e != cudaSuccess) return noalloc_fail(FP8MLP_ERR_CUDA, cudaGetErrorString(e));
   return FP8MLP_OK;
 }

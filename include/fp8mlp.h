@@ -303,6 +303,10 @@ int fp8mlp_ce_bwd_dlogits_fp8(int M, int d, int V, int T, const uint8_t* x_fp8, 
  * [M,h] post, and the block size in rows / columns.  Returns FP8MLP_OK. */
 int fp8mlp_partial_amax_shape(int M, int h, int* row_blocks, int* col_blocks, int* block_rows,
                               int* block_cols);
+/* Number of fp32 entries of that tensor, row_blocks * col_blocks: the n to
+ * pass to fp8mlp_amax_reduce_update_scale and the length of the buffer to
+ * allocate for partial_amax (0 for negative sizes). */
+int fp8mlp_partial_amax_count(int M, int h);
 
 /* ------------------------------------------------------------------------
  * Delayed scaling and the W2 cache
@@ -347,8 +351,9 @@ int fp8mlp_w2_fp8_cache_refresh(int h, int d, const uint16_t* W2, uint8_t* W2q_t
  * callers cannot provide a workspace: code inside another framework's
  * operator hook that owns every device allocation through its own pool and
  * exposes none to the op, or a runtime that forbids cudaMalloc/cudaFree on its
- * hot path because they can synchronise the whole device.  Results equal
- * fp8mlp_w2_fp8_cache_refresh's bit for bit.
+ * hot path because they can synchronise the whole device.  It launches the
+ * same two kernels as fp8mlp_w2_fp8_cache_refresh, so the results are the
+ * same bits.
  *   - Scratch: a fixed 8 KiB device array owned by the library (2048 partial
  *     maxima, one per 8192 elements of W2); every GPU that loads the library
  *     holds it until the process exits.  h*d above 16,777,216 elements is
@@ -459,10 +464,16 @@ int fp8mlp_clear_device_status(fp8mlp_stream_t stream);
 int fp8mlp_set_programmatic_launch(int enable);
 /* Per-wait limit of the kernels' bounded waits, in ns (default 2e9). */
 int fp8mlp_set_wait_timeout_ns(unsigned long long ns);
-/* Test hook: FP8MLP_DEBUG_STALL_PRODUCER makes the next GEMM launches'
- * load warp issue nothing, so the MMA warp's bounded wait runs out and the
- * kernel returns with FP8MLP_STATUS_TIMEOUT set.  0 restores normal runs. */
+/* Test hooks for the bounded waits.  FP8MLP_DEBUG_STALL_PRODUCER makes the
+ * next GEMM launches' load warp issue nothing, so the MMA warp's bounded wait
+ * runs out.  FP8MLP_DEBUG_STALL_AUX makes the epilogue of the next
+ * fp8mlp_bwd_dpre launches issue none of its loads of post, so the
+ * epilogue's own waits for them run out (and then the MMA warp's wait for a
+ * free accumulator).  Either way the kernel returns with
+ * FP8MLP_STATUS_TIMEOUT set and the context stays usable.  0 restores normal
+ * runs. */
 #define FP8MLP_DEBUG_STALL_PRODUCER 1
+#define FP8MLP_DEBUG_STALL_AUX 2
 int fp8mlp_set_debug_flags(int flags);
 
 /* Static text of a return code. */

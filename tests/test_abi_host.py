@@ -22,11 +22,29 @@ def test_library_exports_every_header_symbol():
         assert hasattr(A, s), f"binding lacks {s}"
 
 
+# the calls the boundary of the block is specified with (forward, backward,
+# W2 cache refresh, amax reduction with the scale update, and their helpers)
+BOUNDARY = ["fp8mlp_mlp_fwd", "fp8mlp_mlp_bwd", "fp8mlp_w2_fp8_cache_refresh", "fp8mlp_amax_reduce_update_scale",
+            "fp8mlp_scale_state_init", "fp8mlp_workspace_size", "fp8mlp_partial_amax_count",
+            "fp8mlp_get_device_status", "fp8mlp_error_string"]
+
+
 def test_header_declares_the_boundary_calls():
     syms = set(A.header_symbols())
-    for s in ["fp8mlp_mlp_fwd", "fp8mlp_mlp_bwd", "fp8mlp_w2_fp8_cache_refresh",
-              "fp8mlp_amax_reduce_update_scale", "fp8mlp_up_proj_fused", "fp8mlp_down_proj_fp8"]:
-        assert s in syms
+    for s in BOUNDARY + ["fp8mlp_up_proj_fused", "fp8mlp_down_proj_fp8", "fp8mlp_bwd_dpre", "fp8mlp_bwd_dx",
+                         "fp8mlp_bwd_dw", "fp8mlp_partial_amax_shape"]:
+        assert s in syms, s
+        assert hasattr(A.lib, s), s
+
+
+def test_partial_amax_count_is_the_shape_product():
+    for M, h in [(0, 3072), (1, 16), (300, 272), (16384, 3072), (49152, 3072), (65536, 4096)]:
+        rb, cb, br, bc = A.fp8mlp_partial_amax_shape(M, h)
+        assert A.fp8mlp_partial_amax_count(M, h) == rb * cb
+        # every block of post is covered
+        assert rb * br >= M and cb * bc >= h
+    assert A.fp8mlp_partial_amax_count(16384, 3072) == 512 * 48
+    assert A.fp8mlp_partial_amax_count(-1, 16) == 0
 
 
 def test_scale_state_layout_is_32_bytes():
@@ -77,7 +95,8 @@ def test_flag_checks():
     assert _rc("fp8mlp_up_proj_fused", 16, 64, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 8, None) == A.ERR_INVALID_ARG
     assert _rc("fp8mlp_mlp_fwd", 16, 64, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
                A.FWD_EVAL_BF16 | A.FWD_CALIBRATE, None) == A.ERR_INVALID_ARG
-    assert _rc("fp8mlp_set_debug_flags", 2) == A.ERR_INVALID_ARG
+    assert _rc("fp8mlp_set_debug_flags", 4) == A.ERR_INVALID_ARG
+    assert _rc("fp8mlp_set_debug_flags", A.DEBUG_STALL_AUX) == 0 and _rc("fp8mlp_set_debug_flags", 0) == 0
     assert _rc("fp8mlp_set_wait_timeout_ns", 0) == A.ERR_INVALID_ARG
 
 

@@ -15,7 +15,7 @@ from fp8_relu_mlp_b200 import _abi as A
 from fp8_relu_mlp_b200 import synth
 from fp8_relu_mlp_b200.block import MLPBlock
 from oracle import ref
-from tests.gpu_util import host_bits, rel_fro
+from tests.gpu_util import host_bits, rel_fro, stack_errors_given_layer_inputs
 from tests.test_gpu_parity import post_within_accumulation_bound
 
 pytestmark = pytest.mark.gpu
@@ -58,7 +58,8 @@ def _forward_checks(blk, P, W, rows, s_o):
     ok, frac = post_within_accumulation_bound(post_g, P["x"], P["W1"], rows=rows)
     assert ok and frac < 1e-2, frac
     q_g = host_bits(blk.post_fp8.index_select(0, idx))
-    # equal wherever post agrees; elsewhere one FP8 step at most
+    # the FP8 copy is the oracle's quantisation of the kernel's own post
+    assert np.array_equal(q_g, ref.quantise_post(post_g, s_o))
     same = post_g == f["post"]
     assert np.array_equal(q_g[same], f["q"][same])
     out_g = ref.bf16_to_f64(host_bits(blk.out.index_select(0, idx)))
@@ -209,8 +210,13 @@ def test_fullsize_fp8_up_overlapped_step_sampled():
     W2q_o, _, s_w2i = ref.w2_cache(P["W2"])
     out_o = ref.down_proj_fp8(ref.quantise_post(post_o, s_o), W2q_o, np.float32(np.float32(1) / s_o), s_w2i)
     assert rel_fro(ref.bf16_to_f64(host_bits(blk.out)[rows]), ref.bf16_to_f64(out_o)) < 2e-2
-    # BF16 backward from the GPU's own post is the straight-through gradient;
-    # the oracle's backward uses its own post (from the e4m3 up-projection)
+    # the BF16 backward of the kernel's own post (the straight-through
+    # gradient of this layer given its inputs) within the gradient bound
+    post_g = host_bits(blk.post)[rows]
+    dPre_g = ref.bwd_dpre(post_g, P["dOut"][rows], P["W2"])
+    assert rel_fro(ref.bf16_to_f64(host_bits(blk.dX)[rows]), ref.bf16_to_f64(ref.bwd_dx(dPre_g, P["W1"]))) < 1e-2
+    # end to end, the oracle's backward of its own post (from its e4m3
+    # up-projection): the FP8 forward's bound
     dPre_o = ref.bwd_dpre(post_o, P["dOut"][rows], P["W2"])
     dX_o = ref.bwd_dx(dPre_o, P["W1"])
     assert rel_fro(ref.bf16_to_f64(host_bits(blk.dX)[rows]), ref.bf16_to_f64(dX_o)) < 2e-2
@@ -259,6 +265,12 @@ def test_stack9_fullsize_sampled_rows(fp8_up):
     else:
         saved, rL = ref.stack_forward(r0[rows], layers, scales)
     dr0, _ = ref.stack_backward(saved, layers, dtop[rows])
+    # each layer given its own inputs: FP8 codes bit for bit, out and the
+    # gradients within the single-kernel bounds
+    e = stack_errors_given_layer_inputs(S, layers, scales, dtop, rows=rows)
+    assert e["q_mismatch"] == 0 and e["out"] < 4e-3, e
+    assert e["dX"] < 1e-2 and e["dr0"] < 1e-2, e
+    # end to end against the oracle's own stack: the FP8 forward's bound
     assert rel_fro(ref.bf16_to_f64(host_bits(S.r[L])[rows]), ref.bf16_to_f64(rL)) < 2e-2
     assert rel_fro(ref.bf16_to_f64(host_bits(S.dr)[rows]), ref.bf16_to_f64(dr0)) < 2e-2
     assert A.fp8mlp_get_device_status() == 0
