@@ -86,6 +86,31 @@ def parse():
 # peaks
 # ---------------------------------------------------------------------------
 
+# the B200's dense datasheet peaks: the step fractions are also reported
+# against these (the measured-peak fractions are the primary ones)
+SPEC_PEAKS = {"bf16_tflops": 2250.0, "fp8_tflops": 4500.0, "hbm_gbs": 8000.0}
+
+
+def roofline_s(work, bf16_tf, fp8_tf, hbm_gbs, keys=None):
+    """Roofline time of a step: the sum over its kernels of the slower of the
+    tensor time (BF16 and FP8 FLOPs at their peaks) and the HBM time."""
+    ks = list(work) if keys is None else keys
+    return sum(max(work[k]["bf16"] / (bf16_tf * 1e12) + work[k]["fp8"] / (fp8_tf * 1e12),
+                   work[k]["bytes"] / (hbm_gbs * 1e9)) for k in ks)
+
+
+def spec_roofline(step_s, roof_fn, fwd_s=None, fwd_fn=None):
+    """The step (and forward) roofline fractions against SPEC_PEAKS;
+    roof_fn(bf16_tf, fp8_tf, hbm_gbs) -> seconds."""
+    P = SPEC_PEAKS
+    r = roof_fn(P["bf16_tflops"], P["fp8_tflops"], P["hbm_gbs"])
+    out = {"roofline_ms": r * 1e3, "frac": r / step_s, "peaks": dict(P, source="B200 dense datasheet")}
+    if fwd_fn is not None:
+        rf = fwd_fn(P["bf16_tflops"], P["fp8_tflops"], P["hbm_gbs"])
+        out.update(fwd_roofline_ms=rf * 1e3, fwd_frac=rf / fwd_s)
+    return out
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -356,7 +381,9 @@ def cpu_baseline(W, seconds, tokens=None, fp8_up=False):
                        if W.name.startswith("ce") else "") +
                       f"{reps} oracle steps of {tokens} tokens of the {W.name} workload "
                       f"(d={W.d}, {'V' if W.name.startswith('ce') else 'h'}={W.h}, {W.layers} layer(s); "
-                      f"the whole {'fwd+bwd' if W.backward else 'forward'} step), {el:.1f} s"}
+                      f"the whole {'fwd+bwd' if W.backward else 'forward'} step), {el:.1f} s; "
+                      f"tokens/s extrapolated from {tokens}-token steps to the workload's {W.M} tokens "
+                      f"(the oracle's work is linear in the tokens)"}
 
 
 def run_reference(a, W, world, rank):
@@ -554,13 +581,13 @@ def run_ours(a, W, world, rank, local_rank):
     peak_dom = fp8_peak if wd["fp8"] else peaks["bf16_tflops"]
     achieved = (wd["bf16"] + wd["fp8"]) / dom_s / 1e12
     traffic = load_traffic(W.name).get(dom)
-    roof_t = 0.0
-    for n, w in work.items():
-        roof_t += max(w["bf16"] / (peaks["bf16_tflops"] * 1e12) + w["fp8"] / (fp8_peak * 1e12),
-                      w["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    roof_t = roofline_s(work, peaks["bf16_tflops"], fp8_peak, peaks["hbm_gbs"])
     fwd_s = avg["up_fused"] + avg["down_fp8"]
-    fwd_roof = sum(work[k]["bf16"] / (peaks["bf16_tflops"] * 1e12) + work[k]["fp8"] / (fp8_peak * 1e12)
-                   for k in ("up_fused", "down_fp8"))
+
+    def fwd_fn(pb, p8, bw):
+        return sum(work[k]["bf16"] / (pb * 1e12) + work[k]["fp8"] / (p8 * 1e12) for k in ("up_fused", "down_fp8"))
+    fwd_roof = fwd_fn(peaks["bf16_tflops"], fp8_peak, peaks["hbm_gbs"])
+    spec = spec_roofline(total_s / a.steps, lambda pb, p8, bw: roofline_s(work, pb, p8, bw), fwd_s, fwd_fn)
 
     e2e = None
     if not a.no_e2e:
@@ -588,7 +615,7 @@ def run_ours(a, W, world, rank, local_rank):
                               "fwd_ms": fwd_s * 1e3, "fwd_roofline_ms": fwd_roof * 1e3,
                               "fwd_frac": fwd_roof / fwd_s, "fwd_tokens_per_s": M / fwd_s,
                               "peaks": {"bf16_tflops": peaks["bf16_tflops"], "fp8_tflops": fp8_peak,
-                                        "hbm_gbs": peaks["hbm_gbs"]}},
+                                        "hbm_gbs": peaks["hbm_gbs"]}, "spec": spec},
             "kernels_ms": breakdown,
             "kernels_ms_note": "median of 5 untimed steps with an event between every kernel",
             "clocks": clocks, "gpu_launches": int(launches), "device_status": status,
@@ -670,10 +697,8 @@ def run_dp(a, W, world, rank, local_rank, blk, flush, dist, peaks, fp8_peak, fp8
     e2e = None
     if not a.no_e2e and P is not None:
         e2e = measure_e2e(a, blk, P, torch, blk.device, None, M, world, dist, step_fn=stepper)
-    roof_t = 0.0
-    for n, w in work.items():
-        roof_t += max(w["bf16"] / (peaks["bf16_tflops"] * 1e12) + w["fp8"] / (fp8_peak * 1e12),
-                      w["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    roof_t = roofline_s(work, peaks["bf16_tflops"], fp8_peak, peaks["hbm_gbs"])
+    spec = spec_roofline(total_s / a.steps, lambda pb, p8, bw: roofline_s(work, pb, p8, bw))
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
@@ -688,7 +713,7 @@ def run_dp(a, W, world, rank, local_rank, blk, flush, dist, peaks, fp8_peak, fp8
                          "traffic": load_traffic(W.name).get("bwd_dw"),
                          "peak_source": f"bf16_tflops burst of {peaks['source']} peaks"},
             "step_roofline": {"roofline_ms": roof_t * 1e3, "measured_ms": total_s / a.steps * 1e3,
-                              "frac": roof_t / (total_s / a.steps)},
+                              "frac": roof_t / (total_s / a.steps), "spec": spec},
             "clocks": clk.summary(), "gpu_launches": int(launches), "device_status": status,
             "launch_mode": "eager",
         }
@@ -784,8 +809,9 @@ def run_fwd(a, W, world, rank, local_rank):
     work = kernel_work(M, d, h)
     up_s = statistics.mean(up_ms) * 1e-3
     achieved = work["up_fused"]["bf16"] / up_s / 1e12
-    roof = sum(max(work[k]["bf16"] / (peaks["bf16_tflops"] * 1e12) + work[k]["fp8"] / (fp8_peak * 1e12),
-                   work[k]["bytes"] / (peaks["hbm_gbs"] * 1e9)) for k in ("up_fused", "down_fp8", "amax_scale"))
+    fwd_keys = ("up_fused", "down_fp8", "amax_scale")
+    roof = roofline_s(work, peaks["bf16_tflops"], fp8_peak, peaks["hbm_gbs"], fwd_keys)
+    spec = spec_roofline(total_s / a.steps, lambda pb, p8, bw: roofline_s(work, pb, p8, bw, fwd_keys))
     e2e = None
     if not a.no_e2e:
         # x in from pinned host memory and out back, every step; copies
@@ -827,7 +853,8 @@ def run_fwd(a, W, world, rank, local_rank):
                          "traffic": load_traffic(W.name).get("up_fused"),
                          "peak_source": "bf16_tflops burst of measured peaks"},
             "step_roofline": {"roofline_ms": roof * 1e3, "measured_ms": total_s / a.steps * 1e3,
-                              "frac": roof / (total_s / a.steps), "peaks": {**peaks, "fp8_tflops": fp8_peak}},
+                              "frac": roof / (total_s / a.steps), "peaks": {**peaks, "fp8_tflops": fp8_peak},
+                              "spec": spec},
             "kernels_ms": {"up_fused": statistics.median(up_ms), "down_fp8": statistics.median(down_ms)},
             "clocks": clk.summary(), "gpu_launches": int(kps * a.steps), "device_status": status,
             "launch_mode": "eager" if graph is None else "cuda_graph",
@@ -939,8 +966,10 @@ def run_linear(a, W, world, rank, local_rank):
     F = 2 * M * K * N
     fwd_s = statistics.mean(fwd_ms) * 1e-3
     achieved = F / fwd_s / 1e12
-    roof = (F / (fp8_peak * 1e12) + 2 * F / (peaks["bf16_tflops"] * 1e12)
-            + (2 * M * K + M * K) / (peaks["hbm_gbs"] * 1e9))
+    def roof_fn(pb, p8, bw):
+        return F / (p8 * 1e12) + 2 * F / (pb * 1e12) + (2 * M * K + M * K) / (bw * 1e9)
+    roof = roof_fn(peaks["bf16_tflops"], fp8_peak, peaks["hbm_gbs"])
+    spec = spec_roofline(total_s / a.steps, roof_fn)
     e2e = None
     if not a.no_e2e:
         # x and the upstream gradient dY in from pinned host memory, y and dX
@@ -979,7 +1008,7 @@ def run_linear(a, W, world, rank, local_rank):
                          "unit": "TFLOP/s", "frac": achieved / fp8_peak,
                          "traffic": load_traffic(W.name).get("linear_fwd_fp8"), "peak_source": fp8_src},
             "step_roofline": {"roofline_ms": roof * 1e3, "measured_ms": total_s / a.steps * 1e3,
-                              "frac": roof / (total_s / a.steps)},
+                              "frac": roof / (total_s / a.steps), "spec": spec},
             "clocks": clk.summary(), "gpu_launches": int(kps * a.steps),
             "launch_mode": "eager" if graph is None else "cuda_graph",
         }
@@ -1231,11 +1260,14 @@ def run_ce(a, W, world, rank, local_rank):
                     "unit": "GB/s", "traffic": load_traffic(W.name).get(dom),
                     "peak_source": f"hbm_gbs of {peaks['source']} peaks"}
     roofline["frac"] = roofline["achieved"] / roofline["peak"]
-    roof_t = sum(max(w["bf16"] / (peaks["bf16_tflops"] * 1e12) + w["fp8"] / (fp8_peak * 1e12),
-                     w["bytes"] / (peaks["hbm_gbs"] * 1e9)) for w in work.values())
+    roof_t = roofline_s(work, peaks["bf16_tflops"], fp8_peak, peaks["hbm_gbs"])
     fwd_s = breakdown["ce_fwd"] * 1e-3
     wf = work["ce_fwd"]
-    fwd_roof = wf["bf16"] / (peaks["bf16_tflops"] * 1e12) + wf["fp8"] / (fp8_peak * 1e12)
+
+    def fwd_fn(pb, p8, bw):
+        return wf["bf16"] / (pb * 1e12) + wf["fp8"] / (p8 * 1e12)
+    fwd_roof = fwd_fn(peaks["bf16_tflops"], fp8_peak, peaks["hbm_gbs"])
+    spec = spec_roofline(total_s / a.steps, lambda pb, p8, bw: roofline_s(work, pb, p8, bw), fwd_s, fwd_fn)
 
     e2e = None
     if not a.no_e2e:
@@ -1289,7 +1321,7 @@ def run_ce(a, W, world, rank, local_rank):
                               "frac": roof_t / (total_s / a.steps), "fwd_ms": fwd_s * 1e3,
                               "fwd_roofline_ms": fwd_roof * 1e3, "fwd_frac": fwd_roof / fwd_s,
                               "peaks": {"bf16_tflops": peaks["bf16_tflops"], "fp8_tflops": fp8_peak,
-                                        "hbm_gbs": peaks["hbm_gbs"]}},
+                                        "hbm_gbs": peaks["hbm_gbs"]}, "spec": spec},
             "kernels_ms": breakdown,
             "kernels_ms_note": "median of 5 untimed steps with an event between every call; ce_fwd includes "
                                "its two small reduction kernels",
@@ -1414,11 +1446,9 @@ def run_stack(a, W, world, rank, local_rank):
         work["up_fused"] = dict(bf16=0, fp8=F, bytes=M * d + h * d + 3 * M * h)
         work["w2_cache"]["bytes"] += 2 * (2 * h * d) + h * d
         norm_bytes += M * d
-    roof_t = 0.0
-    for n, w in work.items():
-        roof_t += max(w["bf16"] / (peaks["bf16_tflops"] * 1e12) + w["fp8"] / (fp8_peak * 1e12),
-                      w["bytes"] / (peaks["hbm_gbs"] * 1e9))
-    roof_t = L * (roof_t + norm_bytes / (peaks["hbm_gbs"] * 1e9)) + 4 * M * d / (peaks["hbm_gbs"] * 1e9)
+    def roof_fn(pb, p8, bw):
+        return L * (roofline_s(work, pb, p8, bw) + norm_bytes / (bw * 1e9)) + 4 * M * d / (bw * 1e9)
+    roof_t = roof_fn(peaks["bf16_tflops"], fp8_peak, peaks["hbm_gbs"])
     dom_s = statistics.mean(dom_ms) * 1e-3
     achieved = work["bwd_dw"]["bf16"] / dom_s / 1e12
     # a step of tens of milliseconds runs under the power cap: the kernel is
@@ -1476,7 +1506,8 @@ def run_stack(a, W, world, rank, local_rank):
             "step_roofline": {"roofline_ms": roof_t * 1e3, "measured_ms": total_s / a.steps * 1e3,
                               "frac": roof_t / (total_s / a.steps),
                               "peaks": {"bf16_tflops": peaks["bf16_tflops"], "fp8_tflops": fp8_peak,
-                                        "hbm_gbs": peaks["hbm_gbs"]}},
+                                        "hbm_gbs": peaks["hbm_gbs"]},
+                              "spec": spec_roofline(total_s / a.steps, roof_fn)},
             "clocks": clk.summary(), "gpu_launches": int(launches), "device_status": status,
             "launch_mode": "eager" if graph is None else "cuda_graph",
         }

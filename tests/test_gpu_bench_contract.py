@@ -47,6 +47,12 @@ def test_bench_line_step16k():
     assert {"sm_mhz", "sm_max_mhz", "reasons"} <= set(clk)
     assert d["gpu_launches"] >= 8 * d["steps"]
     assert d["device_status"] == 0
+    # the step against the measured peaks and against the datasheet peaks
+    sr = d["step_roofline"]
+    assert abs(sr["frac"] - sr["roofline_ms"] / sr["measured_ms"]) < 1e-9
+    sp = sr["spec"]
+    assert sp["peaks"]["bf16_tflops"] == 2250.0 and sp["peaks"]["fp8_tflops"] == 4500.0
+    assert 0 < sp["frac"] < sr["frac"] and 0 < sp["fwd_frac"] < sr["fwd_frac"]
 
 
 @pytest.mark.timeout(900)
