@@ -262,7 +262,13 @@ def _rand_codes(g, shape):
     return c
 
 
-@pytest.mark.parametrize("M,d,h", SHAPES)
+# more e4m3 down-projections: ragged M with an N ending a quarter into its
+# second tile (320 = 256 + 64), K ending inside a partial k-block (1040 =
+# 8 x 128 + 16) over several waves, and the benchmark's M = 16384 (2.59 waves)
+EXTRA_DOWN_SHAPES = [(1000, 320, 512), (4100, 768, 1040), (16384, 768, 3072)]
+
+
+@pytest.mark.parametrize("M,d,h", SHAPES + EXTRA_DOWN_SHAPES)
 def test_down_proj_fp8(M, d, h):
     g = np.random.default_rng(M * 7 + h)
     q = _rand_codes(g, (M, h))
@@ -302,7 +308,7 @@ def test_down_proj_bf16_eval(M, d, h):
 # whole forward, FP8 path, vs the oracle
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("M,d,h", SHAPES)
+@pytest.mark.parametrize("M,d,h", SHAPES + EXTRA_DOWN_SHAPES[:1])
 def test_mlp_fwd_fp8(M, d, h):
     P = synth.make_problem(M, d, h, seed=21)
     W2q_t, s_w, s_wi = ref.w2_cache(P["W2"])
@@ -360,6 +366,30 @@ def test_bwd_dpre(M, d, h):
     # zero post gives exactly zero dPre (relu'(pre) = 0 there)
     assert (ref.bf16_to_f64(got)[ref.bf16_to_f64(post) == 0] == 0).all()
     assert dPre.intact()
+
+
+@pytest.mark.parametrize("M,d,h", [(300, 80, 272), (1000, 768, 3072)])
+def test_bwd_dpre_post_16_byte_aligned(M, d, h):
+    """post at an address that is 16-byte but not 32-byte aligned (the
+    boundary allows any 16-byte aligned pointer): the same bits as from an
+    aligned copy of the same values."""
+    P = synth.make_problem(M, d, h, seed=33)
+    post = _post_like(np.random.default_rng(M + 1), M, h)
+    dOut, W2 = dev_bf16(P["dOut"]), dev_bf16(P["W2"])
+    base = torch.zeros(M * h + 64, dtype=torch.bfloat16, device="cuda")
+    off = next(k for k in range(8, 64, 8) if (base.data_ptr() + 2 * k) % 32 == 16)
+    post_u = base[off:off + M * h].view(M, h)
+    post_u.copy_(dev_bf16(post))
+    assert post_u.data_ptr() % 32 == 16
+    got_u = Guarded((M, h), torch.bfloat16)
+    got_a = Guarded((M, h), torch.bfloat16)
+    A.fp8mlp_bwd_dpre(M, d, h, dOut, W2, post_u, got_u.t)
+    A.fp8mlp_bwd_dpre(M, d, h, dOut, W2, dev_bf16(post), got_a.t)
+    torch.cuda.synchronize()
+    assert torch.equal(got_u.t, got_a.t)
+    want = ref.bwd_dpre(post, P["dOut"], P["W2"])
+    assert rel_fro(ref.bf16_to_f64(host_bits(got_u.t)), ref.bf16_to_f64(want)) < 4e-3
+    assert got_u.intact() and got_a.intact()
 
 
 @pytest.mark.parametrize("M,d,h", SHAPES)
