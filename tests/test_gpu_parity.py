@@ -370,9 +370,9 @@ def test_bwd_dpre(M, d, h):
 
 @pytest.mark.parametrize("M,d,h", [(300, 80, 272), (1000, 768, 3072)])
 def test_bwd_dpre_post_16_byte_aligned(M, d, h):
-    """post at an address that is 16-byte but not 32-byte aligned (the
-    boundary allows any 16-byte aligned pointer): the same bits as from an
-    aligned copy of the same values."""
+    """post, and then dPre too, at an address that is 16-byte but not 32-byte
+    aligned (the boundary allows any 16-byte aligned pointer): the same bits
+    as from aligned buffers holding the same values."""
     P = synth.make_problem(M, d, h, seed=33)
     post = _post_like(np.random.default_rng(M + 1), M, h)
     dOut, W2 = dev_bf16(P["dOut"]), dev_bf16(P["W2"])
@@ -385,8 +385,16 @@ def test_bwd_dpre_post_16_byte_aligned(M, d, h):
     got_a = Guarded((M, h), torch.bfloat16)
     A.fp8mlp_bwd_dpre(M, d, h, dOut, W2, post_u, got_u.t)
     A.fp8mlp_bwd_dpre(M, d, h, dOut, W2, dev_bf16(post), got_a.t)
+    # and dPre itself at such an address, the bytes around it untouched
+    out_base = torch.full((M * h + 64,), 7.0, dtype=torch.bfloat16, device="cuda")
+    off2 = next(k for k in range(8, 64, 8) if (out_base.data_ptr() + 2 * k) % 32 == 16)
+    out_u = out_base[off2:off2 + M * h].view(M, h)
+    assert out_u.data_ptr() % 32 == 16
+    A.fp8mlp_bwd_dpre(M, d, h, dOut, W2, post_u, out_u)
     torch.cuda.synchronize()
     assert torch.equal(got_u.t, got_a.t)
+    assert torch.equal(out_u, got_a.t)
+    assert bool((out_base[:off2] == 7.0).all()) and bool((out_base[off2 + M * h:] == 7.0).all())
     want = ref.bwd_dpre(post, P["dOut"], P["W2"])
     assert rel_fro(ref.bf16_to_f64(host_bits(got_u.t)), ref.bf16_to_f64(want)) < 4e-3
     assert got_u.intact() and got_a.intact()
