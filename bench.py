@@ -781,9 +781,9 @@ def run_fwd(a, W, world, rank, local_rank):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     npa = blk.partial_amax.numel()
 
-    def step(ev=None, bufs=None):
+    def step(ev=None, bufs=None, marks=(0, 1, 2, 3)):
         def mark(i):
-            if ev is not None:
+            if ev is not None and i in marks:
                 ev[i].record()
         xb, ob = bufs if bufs is not None else (blk.x, blk.out)
         mark(0)
@@ -796,21 +796,34 @@ def run_fwd(a, W, world, rank, local_rank):
 
     step()
     torch.cuda.synchronize()
+    # as in the training step: the events between the kernels (which time
+    # the up-projection, the dominant kernel, and the down-projection) are in
+    # every DOM_EVERY-th timed step; the others replay the same calls with
+    # only the start and end events, so that each kernel may start while the
+    # previous one finishes
     ev = [torch.cuda.Event(enable_timing=True, external=not a.eager) for _ in range(4)]
+    ev_p = [torch.cuda.Event(enable_timing=True, external=not a.eager) for _ in range(4)]
     n_cap0 = A.fp8mlp_kernel_launch_count()
-    graph = None
+    graph = graph_p = None
     if not a.eager:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             step(ev)
-    kps = A.fp8mlp_kernel_launch_count() - n_cap0 if graph is not None else 3
+        graph_p = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_p):
+            step(ev_p, marks=(0, 3))
+    kps = (A.fp8mlp_kernel_launch_count() - n_cap0) // 2 if graph is not None else 3
 
-    def run():
-        graph.replay() if graph is not None else step(ev)
+    def run(timed=True):
+        if timed:
+            graph.replay() if graph is not None else step(ev)
+        else:
+            graph_p.replay() if graph_p is not None else step(ev_p, marks=(0, 3))
 
     for _ in range(max(a.warmup, 3)):
-        flush.zero_()
-        run()
+        for t_ in (True, False):
+            flush.zero_()
+            run(t_)
     torch.cuda.synchronize()
     A.fp8mlp_clear_device_status()
     if dist:
@@ -818,13 +831,18 @@ def run_fwd(a, W, world, rank, local_rank):
     torch.cuda.synchronize()
     step_ms, up_ms, down_ms = [], [], []
     with ClockSampler(local_rank) as clk:
-        for _ in range(a.steps):
+        for i in range(a.steps):
             flush.zero_()
-            run()
-            ev[3].synchronize()
-            step_ms.append(ev[0].elapsed_time(ev[3]))
-            up_ms.append(ev[0].elapsed_time(ev[1]))
-            down_ms.append(ev[1].elapsed_time(ev[2]))
+            if i % DOM_EVERY == 0:
+                run(True)
+                ev[3].synchronize()
+                step_ms.append(ev[0].elapsed_time(ev[3]))
+                up_ms.append(ev[0].elapsed_time(ev[1]))
+                down_ms.append(ev[1].elapsed_time(ev[2]))
+            else:
+                run(False)
+                ev_p[3].synchronize()
+                step_ms.append(ev_p[0].elapsed_time(ev_p[3]))
     status = A.fp8mlp_get_device_status()
     total_s = sum(step_ms) * 1e-3
     if dist:
@@ -874,7 +892,9 @@ def run_fwd(a, W, world, rank, local_rank):
             "data": "synthetic (seeded; shapes of the 768-dim GPT-2-small / nanochat MLP)",
             "config": dict(config_of(W), parallelism=f"dp{world} replicas" if world > 1 else "single GPU"),
             "roofline": {"bound": "tensor", "kernel": "up_fused", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "timed_launches": len(up_ms),
+                         "timing": f"CUDA events around the kernel on every {DOM_EVERY}th timed step (the first "
+                                   f"included); the other timed steps replay the same calls without them",
                          "traffic": load_traffic(W.name).get("up_fused"),
                          "peak_source": "bf16_tflops burst of measured peaks"},
             "step_roofline": {"roofline_ms": roof * 1e3, "measured_ms": total_s / a.steps * 1e3,
@@ -939,9 +959,9 @@ def run_linear(a, W, world, rank, local_rank):
     A.fp8mlp_quantize_x(M, K, x, st, xq, pax)
     A.fp8mlp_amax_reduce_update_scale(pax, npx, st)
 
-    def step(ev=None, bufs=None):
+    def step(ev=None, bufs=None, marks=(0, 1, 2, 3)):
         def mark(i):
-            if ev is not None:
+            if ev is not None and i in marks:
                 ev[i].record()
         xb, dYb, yb, dXb = bufs if bufs is not None else (x, dY, y, dX)
         mark(0)
@@ -956,33 +976,51 @@ def run_linear(a, W, world, rank, local_rank):
 
     step()
     torch.cuda.synchronize()
+    # the events around the forward GEMM (the dominant kernel) in every
+    # DOM_EVERY-th timed step; the others replay the same calls with only the
+    # start and end events (see run_ours)
     ev = [torch.cuda.Event(enable_timing=True, external=not a.eager) for _ in range(4)]
+    ev_p = [torch.cuda.Event(enable_timing=True, external=not a.eager) for _ in range(4)]
     n_cap0 = A.fp8mlp_kernel_launch_count()
-    graph = None
+    graph = graph_p = None
     if not a.eager:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             step(ev)
-    kps = A.fp8mlp_kernel_launch_count() - n_cap0
+        graph_p = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_p):
+            step(ev_p, marks=(0, 3))
+        kps = (A.fp8mlp_kernel_launch_count() - n_cap0) // 2
+    else:
+        kps = A.fp8mlp_kernel_launch_count() - n_cap0
 
-    def run():
-        graph.replay() if graph is not None else step(ev)
+    def run(timed=True):
+        if timed:
+            graph.replay() if graph is not None else step(ev)
+        else:
+            graph_p.replay() if graph_p is not None else step(ev_p, marks=(0, 3))
 
     for _ in range(max(a.warmup, 3)):
-        flush.zero_()
-        run()
+        for t_ in (True, False):
+            flush.zero_()
+            run(t_)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     step_ms, fwd_ms = [], []
     with ClockSampler(local_rank) as clk:
-        for _ in range(a.steps):
+        for i in range(a.steps):
             flush.zero_()
-            run()
-            ev[3].synchronize()
-            step_ms.append(ev[0].elapsed_time(ev[3]))
-            fwd_ms.append(ev[1].elapsed_time(ev[2]))
+            if i % DOM_EVERY == 0:
+                run(True)
+                ev[3].synchronize()
+                step_ms.append(ev[0].elapsed_time(ev[3]))
+                fwd_ms.append(ev[1].elapsed_time(ev[2]))
+            else:
+                run(False)
+                ev_p[3].synchronize()
+                step_ms.append(ev_p[0].elapsed_time(ev_p[3]))
     total_s = sum(step_ms) * 1e-3
     if dist:
         t = torch.tensor([total_s], device=dev, dtype=torch.float64)
@@ -1031,7 +1069,10 @@ def run_linear(a, W, world, rank, local_rank):
             "config": dict(config_of(W), K=K, N=N, parallelism=f"dp{world} replicas" if world > 1 else "single GPU"),
             "roofline": {"bound": "tensor", "kernel": "linear_fwd_fp8", "achieved": achieved, "peak": fp8_peak,
                          "unit": "TFLOP/s", "frac": achieved / fp8_peak,
-                         "traffic": load_traffic(W.name).get("linear_fwd_fp8"), "peak_source": fp8_src},
+                         "traffic": load_traffic(W.name).get("linear_fwd_fp8"), "peak_source": fp8_src,
+                         "timed_launches": len(fwd_ms),
+                         "timing": f"CUDA events around the kernel on every {DOM_EVERY}th timed step (the first "
+                                   f"included); the other timed steps replay the same calls without them"},
             "step_roofline": {"roofline_ms": roof * 1e3, "measured_ms": total_s / a.steps * 1e3,
                               "frac": roof / (total_s / a.steps), "spec": spec},
             "clocks": clk.summary(), "gpu_launches": int(kps * a.steps),
