@@ -17,6 +17,11 @@ comes from separate untimed steps.  ``e2e`` repeats the measurement through the 
 with the step's inputs copied in from pinned host memory and its results
 (out, dX) copied back, inside the timed region.
 
+On one GPU the default run (step16k) also runs the forward-only workload
+(fwd16k, M=16384) and the training step at M=49152 (train49k) as child
+processes with the same steps and warm-up, and nests their summaries in the
+line's ``also`` object (``--no-also`` skips them).
+
 Multi-GPU: one process per GPU under torchrun; ``--gpus N`` run without a
 torchrun environment starts the N ranks itself (and ``--gpus N`` under a
 different WORLD_SIZE is an error, so a scaling run cannot silently time one
@@ -80,6 +85,9 @@ def parse():
                     help="with N>1, reduce-scatter dW1/dW2 (each rank keeps h/N rows) instead of all-reducing them")
     ap.add_argument("--replicas", action="store_true",
                     help="with N>1, run independent replicas (no partial-amax / dW all-reduce)")
+    ap.add_argument("--no-also", action="store_true",
+                    help="step16k on one GPU: do not also run the fwd16k and train49k workloads (their summaries "
+                         "go into the line's `also` object)")
     return ap.parse_args()
 
 
@@ -653,6 +661,9 @@ def run_ours(a, W, world, rank, local_rank):
             line["spike_schedule"] = schedule
         if not a.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(W, a.cpu_seconds)
+        if (W.name == "step16k" and world == 1 and not a.no_also and not a.fp8_up and not a.serial
+                and not a.eager and not a.no_pdl):
+            line["also"] = also_workloads(a)
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()
@@ -1656,6 +1667,35 @@ def measure_e2e(a, blk, P, torch, dev, stream, M, world, dist, step_fn=None):
             "overlap": "copies on two streams beside the compute, double-buffered device sets",
             "copy_bound": {"value": cb, "unit": "tokens/s",
                            "note": "the same pinned copies alone, both directions at once (this rank's link)"}}
+
+
+def also_workloads(a):
+    """The other two MLP workloads of the benchmark suite, each run as a
+    child process of this command on the same GPU with the same steps and
+    warm-up (the forward alone at M=16384; the training step at M=49152),
+    summarised for the default line's `also` object."""
+    import subprocess
+    out = {}
+    for wl in ("fwd16k", "train49k"):
+        cmd = [sys.executable, os.path.abspath(__file__), "--workload", wl, "--steps", str(a.steps), "--warmup",
+               str(a.warmup), "--no-cpu-baseline", "--no-also"] + (["--no-e2e"] if a.no_e2e else [])
+        try:
+            r = subprocess.run(cmd, capture_output=True, text=True, timeout=600)
+            lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+            if r.returncode != 0 or not lines:
+                out[wl] = {"error": f"exit {r.returncode}: {r.stderr.strip()[-300:]}"}
+                continue
+            d = json.loads(lines[-1])
+            sr = d.get("step_roofline", {})
+            out[wl] = {"metric": d["metric"], "value": d["value"], "unit": d["unit"], "ms_per_step": d["ms_per_step"],
+                       "steps": d["steps"], "warmup": d["warmup"], "config": d["config"]["workload"],
+                       "step_roofline_frac": sr.get("frac"), "step_roofline_frac_spec": sr.get("spec", {}).get("frac"),
+                       "roofline": d.get("roofline"), "e2e": (d.get("e2e") or {}).get("value"),
+                       "clocks": d.get("clocks"), "gpu_launches": d.get("gpu_launches"),
+                       "device_status": d.get("device_status")}
+        except Exception as ex:  # pragma: no cover
+            out[wl] = {"error": f"{type(ex).__name__}: {ex}"}
+    return out
 
 
 def relaunch(n):

@@ -53,6 +53,13 @@ def test_bench_line_step16k():
     sp = sr["spec"]
     assert sp["peaks"]["bf16_tflops"] == 2250.0 and sp["peaks"]["fp8_tflops"] == 4500.0
     assert 0 < sp["frac"] < sr["frac"] and 0 < sp["fwd_frac"] < sr["fwd_frac"]
+    # the other two MLP workloads, run by the same command
+    for wl, metric_word in (("fwd16k", "fwd tokens/s"), ("train49k", "fwd+bwd tokens/s")):
+        o = d["also"][wl]
+        assert "error" not in o, o
+        assert o["config"].startswith(wl) and metric_word in o["metric"] and o["value"] > 0
+        assert o["steps"] == d["steps"] and o["warmup"] == d["warmup"]
+        assert 0 < o["step_roofline_frac"] < 1.3 and o["device_status"] == 0
 
 
 @pytest.mark.timeout(900)
