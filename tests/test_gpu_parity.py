@@ -192,6 +192,36 @@ def test_amax_reduce_update_scale_bit_exact(n):
     assert g["step"] == o["step"] == 2 and g["flags"] == o["flags"]
 
 
+def test_forward_of_zero_activations_keeps_the_scale():
+    """x = 0: post, its FP8 copy, every partial amax and out are zero; the
+    reduced amax is 0, so the update keeps the previous scale and sets the
+    kept-scale flag (no device status: 0 is finite), as the oracle does."""
+    M, d, h = 300, 128, 512
+    P = synth.make_problem(M, d, h, seed=9)
+    x = torch.zeros(M, d, dtype=torch.bfloat16, device="cuda")
+    W2q_o, _, s_wi = ref.w2_cache(P["W2"])
+    st = _state(2.0, 37.0)
+    rb, cb, _, _ = A.fp8mlp_partial_amax_shape(M, h)
+    post = Guarded((M, h), torch.bfloat16, fill=1.0)
+    q = Guarded((M, h), torch.uint8, fill=7)
+    pa = Guarded((rb, cb), torch.float32, fill=1.0)
+    out = Guarded((M, d), torch.bfloat16, fill=1.0)
+    A.fp8mlp_clear_device_status()
+    A.fp8mlp_mlp_fwd(M, d, h, x, dev_bf16(P["W1"]), dev_u8(W2q_o), dev_f32(np.array([s_wi, 0, 0, 0], np.float32)),
+                     None, st, post.t, q.t, pa.t, out.t, None, 0)
+    A.fp8mlp_amax_reduce_update_scale(pa.t, A.fp8mlp_partial_amax_count(M, h), st)
+    g = _read_state(st)
+    assert A.fp8mlp_get_device_status() == 0
+    assert not host_bits(post.t).any() and not host_bits(q.t).any() and not host_bits(pa.t).any()
+    assert not host_bits(out.t).any()
+    o = ref.scale_update(ref.scale_state_init(2.0, 37.0), ref.reduce_partials(host_bits(pa.t)))
+    for k in ("amax_prev", "scale", "scale_inv"):
+        assert g[k] == o[k], k
+    assert g["flags"] == o["flags"] == ref.FLAG_KEPT_SCALE and g["step"] == o["step"] == 1
+    for t in (post, q, pa, out):
+        assert t.intact()
+
+
 def test_scale_keeps_previous_on_nonfinite_amax():
     A.fp8mlp_clear_device_status()
     st = _state(1.5, 1.0)
@@ -1134,6 +1164,53 @@ def test_fp8_up_forward_normal_inputs(M, d, h):
     # against the exact BF16 network: the FP8 up- and down-projection error
     exact = ref.bf16_to_f64(ref.down_proj_bf16(ref.relu2_post(ref.up_proj(P["x"], P["W1"])), P["W2"]))
     assert rel_fro(ref.bf16_to_f64(host_bits(b.out)), exact) < 8e-2
+
+
+@pytest.mark.parametrize("M,d,h,seed", [(1000, 768, 3072, 124), (16384, 768, 3072, 0)])
+def test_up_proj_fp8_normal_inputs_bit_exact_given_pre(M, d, h, seed):
+    """The e4m3 up-projection on normal inputs.  The x codes and the W1 cache
+    equal the oracle's bit for bit; the kernel's exported pre (the fp32
+    accumulator times fp32(s_x^-1 s_w1^-1)) lies within the fp32 accumulation
+    bound of the exact e4m3 product (itself exact in fp64) plus the rounding
+    of the scaling; given that pre, post, the FP8 copy and the partial amax
+    equal the oracle's bit for bit.  At M=16384 the inputs are the
+    benchmark's own (seed 0)."""
+    P = synth.make_problem(M, d, h, seed=seed)
+    s_x = np.float32(448.0 / 10.0)
+    st_x = _state(2.0, float(s_x))
+    st = _state(2.0, 20.0)
+    x, W1 = dev_bf16(P["x"]), dev_bf16(P["W1"])
+    xq = Guarded((M, d), torch.uint8)
+    pax = torch.zeros(max(1, A.fp8mlp_x_partial_amax_count(M, d)), device="cuda")
+    A.fp8mlp_quantize_x(M, d, x, st_x, xq.t, pax)
+    W1q = Guarded((h, d), torch.uint8)
+    w1inv = torch.zeros(4, device="cuda")
+    ws = torch.empty(A.fp8mlp_workspace_size(0, d, h), dtype=torch.uint8, device="cuda")
+    A.fp8mlp_w1_fp8_cache_refresh(h, d, W1, W1q.t, w1inv, ws)
+    post = Guarded((M, h), torch.bfloat16)
+    q = Guarded((M, h), torch.uint8)
+    rb, cb, _, _ = A.fp8mlp_partial_amax_shape(M, h)
+    pa = Guarded((rb, cb), torch.float32)
+    pre = Guarded((M, h), torch.float32)
+    A.fp8mlp_up_proj_fused_fp8(M, d, h, xq.t, W1q.t, w1inv, st_x, st, post.t, q.t, pa.t, pre.t, 0)
+    torch.cuda.synchronize()
+    for g in (xq, W1q, post, q, pa, pre):
+        assert g.intact()
+    xq_o, _ = ref.quantise_x(P["x"], s_x)
+    W1q_o, _, s_w1i = ref.w1_cache(P["W1"])
+    assert np.array_equal(host_bits(xq.t), xq_o)
+    assert np.array_equal(host_bits(W1q.t), W1q_o)
+    assert np.float32(w1inv[0].item()) == s_w1i
+    comb = np.float32(np.float32(np.float32(1) / s_x) * s_w1i)
+    X, Wd = ref.e4m3_to_f64(xq_o), ref.e4m3_to_f64(W1q_o)
+    exact = (X @ Wd.T) * np.float64(comb)
+    pre_g = host_bits(pre.t).astype(np.float64)
+    bound = d * 2.0 ** -24 * (np.abs(X) @ np.abs(Wd).T) * np.float64(comb) + 2.0 ** -24 * np.abs(pre_g) + 1e-30
+    assert bool((np.abs(pre_g - exact) <= bound).all())
+    pg = host_bits(post.t)
+    assert np.array_equal(pg, ref.relu2_post(host_bits(pre.t)))
+    assert np.array_equal(host_bits(q.t), ref.quantise_post(pg, np.float32(20.0)))
+    assert np.array_equal(host_bits(pa.t), _pa_oracle(pg, M, h))
 
 
 # ---------------------------------------------------------------------------
