@@ -1059,6 +1059,81 @@ def test_data_parallel_step_single_rank():
     assert torch.equal(sharded.dW1_shard, plain.dW1) and torch.equal(sharded.dW2_shard, plain.dW2)
 
 
+def test_token_sharding_on_two_blocks_reproduces_the_whole_batch():
+    """The data-parallel partition on one GPU, without ranks that wait on one
+    another: two blocks hold the two halves of the tokens and run the
+    library's kernels in turn; the two exchanges of the data-parallel step
+    are done between them with plain tensor ops (MAX over the two
+    partial-amax tensors, SUM of the weight gradients).  Against the block
+    that holds the whole batch: the delayed scale after calibration and after
+    the step bit for bit, the rows of post, its FP8 copy, out, dPre and dX
+    bit for bit (each output element's accumulation does not depend on which
+    tile holds its row), and dW = dW(half 0) + dW(half 1) within the fp32
+    rounding of the two partial sums and of their sum."""
+    from fp8_relu_mlp_b200.block import MLPBlock
+    M, d, h = 2048, 768, 3072
+    half = M // 2
+    P = synth.make_problem(M, d, h, seed=92)
+
+    def make(rows):
+        b = MLPBlock(len(range(*rows.indices(M))), d, h)
+        for k in ("x", "W1", "W2", "dOut"):
+            a = P[k][rows] if k in ("x", "dOut") else P[k]
+            getattr(b, k).copy_(MLPBlock.bits_to_bf16(a, b.device))
+        b.refresh_w2_cache()
+        return b
+
+    def calibrate_shared(blocks):
+        for b in blocks:
+            A.fp8mlp_mlp_fwd(b.M, d, h, b.x, b.W1, None, None, None, b.state, b.post, None, b.partial_amax, None,
+                             None, A.FWD_CALIBRATE)
+        exchange_amax(blocks)
+
+    def exchange_amax(blocks):
+        m = blocks[0].partial_amax.clone()
+        for b in blocks[1:]:
+            m = torch.maximum(m, b.partial_amax)
+        for b in blocks:
+            b.partial_amax.copy_(m)
+            b.update_scale()
+
+    whole = make(slice(0, M))
+    whole.calibrate()
+    parts = [make(slice(0, half)), make(slice(half, M))]
+    calibrate_shared(parts)
+    torch.cuda.synchronize()
+    for b in parts:
+        assert torch.equal(b.state, whole.state)
+    whole.forward()
+    whole.backward()
+    whole.update_scale()
+    for b in parts:
+        b.forward()
+        b.backward()
+    exchange_amax(parts)
+    torch.cuda.synchronize()
+    for b in parts:
+        assert torch.equal(b.state, whole.state)
+    for i, b in enumerate(parts):
+        sl = slice(i * half, (i + 1) * half)
+        for k in ("post", "post_fp8", "out", "dPre", "dX"):
+            assert torch.equal(getattr(b, k), getattr(whole, k)[sl]), (i, k)
+    # dW1 = dPre^T x and dW2 = post^T dOut from the kernels' own (identical)
+    # dPre and post: the whole batch's fp32 accumulation and the sum of the
+    # two halves' are each within the recursive-summation bound of the exact
+    # product (the halves' sum adds one rounding, relative 2^-24)
+    X, G = ref.bf16_to_f64(P["x"]), ref.bf16_to_f64(P["dOut"])
+    for k, left in (("dW1", whole.dPre), ("dW2", whole.post)):
+        L = ref.bf16_to_f64(host_bits(left))
+        exact, absprod = L.T @ (X if k == "dW1" else G), np.abs(L).T @ np.abs(X if k == "dW1" else G)
+        got = host_bits(getattr(parts[0], k) + getattr(parts[1], k))
+        for val in (got, host_bits(getattr(whole, k))):
+            ok, nbad = within_accumulation_bound(val, exact, absprod, M, False, extra=2.0 ** -23)
+            assert ok, (k, nbad)
+        assert rel_fro(got, host_bits(getattr(whole, k))) < 1e-5
+    assert A.fp8mlp_get_device_status() == 0
+
+
 # ---------------------------------------------------------------------------
 # FP8 up-projection: x quantiser, W1 cache, e4m3 up-projection
 # ---------------------------------------------------------------------------
