@@ -58,6 +58,7 @@ _SIGS = {
     "fp8mlp_mlp_fwd": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _p],
     "fp8mlp_partial_amax_shape": [_i, _i, _p, _p, _p, _p],
     "fp8mlp_partial_amax_count": [_i, _i],
+    "fp8mlp_mlp_train_step": [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p],
     "fp8mlp_scale_state_init": [_p, _f, _f, _p],
     "fp8mlp_amax_reduce_update_scale": [_p, _i, _p, _p],
     "fp8mlp_w2_fp8_cache_refresh": [_i, _i, _p, _p, _p, _p, _p],
@@ -180,6 +181,13 @@ def fp8mlp_partial_amax_shape(M, h):
     v = [ctypes.c_int() for _ in range(4)]
     _call("fp8mlp_partial_amax_shape", M, h, *[ctypes.addressof(x) for x in v])
     return tuple(x.value for x in v)
+
+
+def fp8mlp_mlp_train_step(M, d, h, x, W1, W2, dOut, W2q_t, w2_scale_inv, st, post, post_fp8, partial_amax, out,
+                          dPre, dX, dW1, dW2, workspace, stream=None):
+    return _call("fp8mlp_mlp_train_step", M, d, h, _ptr(x), _ptr(W1), _ptr(W2), _ptr(dOut), _ptr(W2q_t),
+                 _ptr(w2_scale_inv), _ptr(st), _ptr(post), _ptr(post_fp8), _ptr(partial_amax), _ptr(out), _ptr(dPre),
+                 _ptr(dX), _ptr(dW1), _ptr(dW2), _ptr(workspace), _stream(stream))
 
 
 def fp8mlp_partial_amax_count(M, h):

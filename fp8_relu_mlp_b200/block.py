@@ -176,6 +176,19 @@ class MLPBlock:
         main.wait_stream(side)
         mark(7)
 
+    def train_step_native(self):
+        """``refresh_w2_cache(); train_step()`` as one library call with the
+        schedule of ``train_step_overlapped`` built into the library
+        (``fp8mlp_mlp_train_step``: its own second stream for the cache
+        refresh and the scale update, dPre and dW started in the previous
+        GEMM's last wave); the same results, bit for bit.  BF16 up-projection
+        only."""
+        if self.fp8_up:
+            raise ValueError("the library's training step runs the BF16 up-projection; use train_step_overlapped")
+        A.fp8mlp_mlp_train_step(self.M, self.d, self.h, self.x, self.W1, self.W2, self.dOut, self.W2q_t,
+                                self.w2_scale_inv, self.state, self.post, self.post_fp8, self.partial_amax, self.out,
+                                self.dPre, self.dX, self.dW1, self.dW2, self.workspace, self.stream)
+
     # ------------------------------------------------------------ CUDA graph
     def capture(self, fn):
         """Record the library calls made by ``fn()`` into a CUDA graph and return

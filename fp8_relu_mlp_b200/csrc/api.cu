@@ -796,6 +796,112 @@ int fp8mlp_mlp_bwd(int M, int d, int h, const uint16_t* x, const uint16_t* W1, c
                        stream);
 }
 
+}  // extern "C"
+
+namespace {
+// the second stream and the events of fp8mlp_mlp_train_step, one set per
+// device, created at the first call on it; a call enqueues its whole
+// sequence (event records and waits included) under the device's lock
+struct StepStreams {
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
+};
+StepStreams g_step[kMaxDevices];
+std::mutex g_step_mutex[kMaxDevices];
+
+int step_streams(int dev, StepStreams** out) {
+  StepStreams& ss = g_step[dev];
+  if (ss.side == nullptr) {
+    cudaStream_t side = nullptr;
+    cudaError_t e = cudaStreamCreateWithFlags(&side, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return cuda_fail(e, "train_step: second stream");
+    cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
+    for (int i = 0; i < 4; ++i) {
+      e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+      if (e != cudaSuccess) {
+        for (int j = 0; j < i; ++j) cudaEventDestroy(ev[j]);
+        cudaStreamDestroy(side);
+        return cuda_fail(e, "train_step: events");
+      }
+    }
+    for (int i = 0; i < 4; ++i) ss.ev[i] = ev[i];
+    ss.side = side;
+  }
+  *out = &ss;
+  return FP8MLP_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int fp8mlp_mlp_train_step(int M, int d, int h, const uint16_t* x, const uint16_t* W1, const uint16_t* W2,
+                          const uint16_t* dOut, uint8_t* W2q_t, float* w2_scale_inv, fp8mlp_scale_state* st,
+                          uint16_t* post, uint8_t* post_fp8, float* partial_amax, uint16_t* out, uint16_t* dPre,
+                          uint16_t* dX, float* dW1, float* dW2, void* workspace, fp8mlp_stream_t stream) {
+  g_detail.clear();
+  TRY(check_dims(M, d, h));
+  REQUIRE_PTR(W1);
+  REQUIRE_PTR(W2);
+  REQUIRE_PTR(W2q_t);
+  REQUIRE_PTR(st);
+  REQUIRE_PTR(dW1);
+  REQUIRE_PTR(dW2);
+  REQUIRE_PTR(workspace);
+  if (w2_scale_inv == nullptr || (reinterpret_cast<uintptr_t>(w2_scale_inv) & 3u))
+    return fail(FP8MLP_ERR_INVALID_ARG, "w2_scale_inv is NULL or misaligned");
+  if (M > 0) {
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(dOut);
+    REQUIRE_PTR(post);
+    REQUIRE_PTR(post_fp8);
+    REQUIRE_PTR(out);
+    REQUIRE_PTR(dPre);
+    REQUIRE_PTR(dX);
+    if (partial_amax == nullptr || (reinterpret_cast<uintptr_t>(partial_amax) & 3u))
+      return fail(FP8MLP_ERR_INVALID_ARG, "partial_amax is NULL or misaligned");
+  }
+  DeviceInfo* di = nullptr;
+  TRY(current_device(&di));
+  const int npa = fp8mlp_partial_amax_count(M, h);
+  if (M == 0) {
+    // nothing to overlap: the cache, zero weight gradients, the kept scale
+    TRY(fp8mlp_w2_fp8_cache_refresh(h, d, W2, W2q_t, w2_scale_inv, workspace, stream));
+    TRY(fp8mlp_mlp_bwd(0, d, h, x, W1, W2, post, dOut, dPre, dX, dW1, dW2, stream));
+    return fp8mlp_amax_reduce_update_scale(partial_amax, 0, st, stream);
+  }
+  std::lock_guard<std::mutex> lock(g_step_mutex[di->device]);
+  StepStreams* ss = nullptr;
+  TRY(step_streams(di->device, &ss));
+  cudaStream_t s = stream, side = ss->side;
+#define TRY_CUDA(call, what)                    \
+  do {                                          \
+    const cudaError_t e_ = (call);              \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+  // the W2 cache refresh (from the current W2) beside the up-projection,
+  // which does not read the cache; joined before the down-projection
+  TRY_CUDA(cudaEventRecord(ss->ev[0], s), "train_step: fork");
+  TRY_CUDA(cudaStreamWaitEvent(side, ss->ev[0], 0), "train_step: fork");
+  TRY(fp8mlp_w2_fp8_cache_refresh(h, d, W2, W2q_t, w2_scale_inv, workspace, side));
+  TRY_CUDA(cudaEventRecord(ss->ev[1], side), "train_step: join");
+  TRY(fp8mlp_up_proj_fused(M, d, h, x, W1, st, post, post_fp8, partial_amax, nullptr, 0, s));
+  TRY_CUDA(cudaStreamWaitEvent(s, ss->ev[1], 0), "train_step: join");
+  TRY(fp8mlp_down_proj_fp8(M, d, h, post_fp8, W2q_t, w2_scale_inv, st, out, s));
+  // dPre reads nothing the down-projection writes: it may start in its last wave
+  TRY(fp8mlp_bwd_dpre(M, d, h, dOut, W2, post, dPre, FP8MLP_LAUNCH_OVERLAP_PREVIOUS, s));
+  // the delayed-scale update beside dX and dW, which do not read the scale
+  TRY_CUDA(cudaEventRecord(ss->ev[2], s), "train_step: fork");
+  TRY_CUDA(cudaStreamWaitEvent(side, ss->ev[2], 0), "train_step: fork");
+  TRY(fp8mlp_amax_reduce_update_scale(partial_amax, npa, st, side));
+  TRY_CUDA(cudaEventRecord(ss->ev[3], side), "train_step: join");
+  TRY(fp8mlp_bwd_dx(M, d, h, dPre, W1, dX, s));
+  // dW reads nothing dX writes: it may start in dX's last wave
+  TRY(fp8mlp_bwd_dw(M, d, h, x, dPre, post, dOut, dW1, dW2, FP8MLP_LAUNCH_OVERLAP_PREVIOUS, s));
+  TRY_CUDA(cudaStreamWaitEvent(s, ss->ev[3], 0), "train_step: join");
+#undef TRY_CUDA
+  return FP8MLP_OK;
+}
+
 int fp8mlp_rmsnorm_fwd_quant(int M, int d, const uint16_t* r, uint16_t* x, float* rstd,
                              const fp8mlp_scale_state* st_x, uint8_t* x_fp8, float* row_amax,
                              fp8mlp_stream_t stream) {

@@ -416,6 +416,35 @@ int fp8mlp_mlp_bwd(int M, int d, int h, const uint16_t* x, const uint16_t* W1, c
                    const uint16_t* post, const uint16_t* dOut, uint16_t* dPre, uint16_t* dX, float* dW1,
                    float* dW2, fp8mlp_stream_t stream);
 
+/*
+ * One whole training step of the block, scheduled for the GPU ("A
+ * Retrospective on Our World Records", Main Track: the transposed FP8 W2
+ * cache refreshed after the optimizer update, the fused up-projection, the
+ * FP8 down-projection, the BF16 backward, the partial amax reduced into the
+ * next step's scale).  Results, bit for bit, are those of
+ *   fp8mlp_w2_fp8_cache_refresh (from the current W2, into W2q_t),
+ *   fp8mlp_mlp_fwd (default flags), fp8mlp_mlp_bwd,
+ *   fp8mlp_amax_reduce_update_scale (fp8mlp_partial_amax_count(M, h) entries),
+ * called in that order on `stream`.  The schedule: the cache refresh runs on
+ * a second stream beside the up-projection (which does not read the cache)
+ * and is joined before the down-projection; dPre and dW start while the
+ * GEMM before each finishes its last wave (FP8MLP_LAUNCH_OVERLAP_PREVIOUS);
+ * the scale update runs on the second stream beside dX and dW and is joined
+ * at the end, so work enqueued later on `stream` sees every result.
+ * Buffers and layouts as in those calls; workspace: fp8mlp_workspace_size
+ * (M, d, h) bytes for the cache refresh.  The second stream and its four
+ * events are the library's own, one set per device, created by the first
+ * call on that device: make that call before any stream capture.  A call
+ * enqueues its whole sequence under that device's lock, so calls from
+ * several host threads are safe, but their second-stream work runs one
+ * call after another.  M = 0: the cache is refreshed, dW1 and dW2 are
+ * zeroed and the scale update keeps the scale (amax 0).
+ */
+int fp8mlp_mlp_train_step(int M, int d, int h, const uint16_t* x, const uint16_t* W1, const uint16_t* W2,
+                          const uint16_t* dOut, uint8_t* W2q_t, float* w2_scale_inv, fp8mlp_scale_state* st,
+                          uint16_t* post, uint8_t* post_fp8, float* partial_amax, uint16_t* out, uint16_t* dPre,
+                          uint16_t* dX, float* dW1, float* dW2, void* workspace, fp8mlp_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * Layer stack helpers (RMSNorm without gain, eps = 1e-6; residual add).
  * The pages train 9-layer, 768-dim models with ReLU^2 MLPs ("nanochat

@@ -117,6 +117,21 @@ def test_linear_bwd_checks_before_enqueueing():
     assert A.fp8mlp_linear_bwd_workspace_size(100, 768, 2304) == 0
 
 
+def test_train_step_checks_before_enqueueing():
+    # M, d, h, x, W1, W2, dOut, W2q_t, w2_scale_inv, st, post, post_fp8, pa, out, dPre, dX, dW1, dW2, ws, stream
+    args = [256, 64, 256] + [FAKE] * 16 + [None]
+    for pos in range(3, 19):
+        a = list(args)
+        a[pos] = None
+        assert _rc("fp8mlp_mlp_train_step", *a) == A.ERR_INVALID_ARG, pos
+    a = list(args)
+    a[4] = FAKE + 8          # W1 misaligned
+    assert _rc("fp8mlp_mlp_train_step", *a) == A.ERR_INVALID_ARG
+    a = list(args)
+    a[1] = 72                # d not a multiple of 16
+    assert _rc("fp8mlp_mlp_train_step", *a) == A.ERR_UNSUPPORTED_SHAPE
+
+
 def test_scale_state_init_checks():
     assert _rc("fp8mlp_scale_state_init", FAKE, ctypes.c_float(0.0), ctypes.c_float(1.0), None) == A.ERR_INVALID_ARG
     assert _rc("fp8mlp_scale_state_init", FAKE, ctypes.c_float(2.0), ctypes.c_float(-1.0), None) == A.ERR_INVALID_ARG

@@ -933,6 +933,59 @@ def test_overlapped_step_matches_serial(M, fp8_up):
         assert torch.equal(getattr(e, k), getattr(g, k)), k
 
 
+@pytest.mark.parametrize("M", [1000, 16384])
+def test_native_train_step_matches_serial(M):
+    """fp8mlp_mlp_train_step (the library's own scheduled step: second
+    stream, launch overlap) against refresh_w2_cache + train_step, bit for
+    bit, three steps, eagerly and replayed as a CUDA graph."""
+    from fp8_relu_mlp_b200.block import MLPBlock
+    d, h = 768, 3072
+    P = synth.make_problem(M, d, h, seed=81)
+
+    def make():
+        b = MLPBlock(M, d, h)
+        for k in ("x", "W1", "W2", "dOut"):
+            getattr(b, k).copy_(MLPBlock.bits_to_bf16(P[k], b.device))
+        b.refresh_w2_cache()
+        b.calibrate()
+        return b
+
+    keys = ["post", "post_fp8", "out", "dPre", "dX", "dW1", "dW2", "W2q_t", "w2_scale_inv", "state", "partial_amax"]
+    e, n, g = make(), make(), make()
+    for _ in range(3):
+        e.refresh_w2_cache()
+        e.train_step()
+        n.train_step_native()
+    g.train_step_native()
+    graph = g.capture(g.train_step_native)
+    graph.replay()
+    graph.replay()
+    torch.cuda.synchronize()
+    for k in keys:
+        assert torch.equal(getattr(e, k), getattr(n, k)), k
+        assert torch.equal(getattr(e, k), getattr(g, k)), k
+    assert A.fp8mlp_get_device_status() == 0
+
+
+def test_native_train_step_empty_batch():
+    from fp8_relu_mlp_b200.block import MLPBlock
+    d, h = 128, 512
+    P = synth.make_problem(1, d, h, seed=82)
+    b = MLPBlock(0, d, h)
+    for k in ("W1", "W2"):
+        getattr(b, k).copy_(MLPBlock.bits_to_bf16(P[k], b.device))
+    b.dW1.fill_(1.0)
+    b.dW2.fill_(1.0)
+    before = b.read_state()
+    b.train_step_native()
+    torch.cuda.synchronize()
+    assert not b.dW1.any() and not b.dW2.any()
+    W2q_o, _, s_wi = ref.w2_cache(P["W2"])
+    assert np.array_equal(host_bits(b.W2q_t), W2q_o) and np.float32(b.w2_scale_inv[0].item()) == s_wi
+    after = b.read_state()
+    assert after["scale"] == before["scale"] and after["flags"] & ref.FLAG_KEPT_SCALE and after["step"] == 1
+
+
 def test_host_pipeline_matches_in_place_steps():
     # inputs from pinned host memory and results back to it, with the copies
     # overlapped across two buffer sets: the same step sequence as stepping
