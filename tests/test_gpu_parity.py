@@ -933,13 +933,13 @@ def test_overlapped_step_matches_serial(M, fp8_up):
         assert torch.equal(getattr(e, k), getattr(g, k)), k
 
 
-@pytest.mark.parametrize("M", [1000, 16384])
-def test_native_train_step_matches_serial(M):
+@pytest.mark.parametrize("M,d,h", [(17, 16, 16), (300, 80, 272), (1000, 768, 3072), (16384, 768, 3072)])
+def test_native_train_step_matches_serial(M, d, h):
     """fp8mlp_mlp_train_step (the library's own scheduled step: second
     stream, launch overlap) against refresh_w2_cache + train_step, bit for
-    bit, three steps, eagerly and replayed as a CUDA graph."""
+    bit, three steps, eagerly and replayed as a CUDA graph; ragged shapes
+    down to the smallest d and h."""
     from fp8_relu_mlp_b200.block import MLPBlock
-    d, h = 768, 3072
     P = synth.make_problem(M, d, h, seed=81)
 
     def make():
