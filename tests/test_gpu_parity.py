@@ -1438,3 +1438,54 @@ def test_smoke_entry_point():
     import __graft_entry__
     __graft_entry__.smoke()
     assert A.fp8mlp_get_device_status() == 0
+
+
+# ---------------------------------------------------------------------------
+# a seeded sweep of shapes: ragged tails at every position
+# ---------------------------------------------------------------------------
+
+def _random_shapes(n, seed):
+    g = np.random.default_rng(seed)
+    shapes = []
+    for _ in range(n):
+        M = int(g.integers(1, 2049))
+        d = 16 * int(g.integers(1, 65))    # 16 .. 1024
+        h = 16 * int(g.integers(1, 257))   # 16 .. 4096
+        shapes.append((M, d, h))
+    return shapes
+
+
+@pytest.mark.parametrize("M,d,h", _random_shapes(16, 2026))
+def test_random_shapes_up_projection_and_step(M, d, h):
+    """On grid inputs (every partial sum exact in fp32) the fused
+    up-projection's post, FP8 copy and partial amax equal the oracle's bit
+    for bit; the library's scheduled training step equals the serial calls
+    bit for bit on normal inputs."""
+    from fp8_relu_mlp_b200.block import MLPBlock
+    G = synth.make_problem(M, d, h, seed=M + 7 * d + h, x_dist="grid", w_dist="grid")
+    s = np.float32(448.0 / 37.0)
+    st = _state(2.0, float(s))
+    post, q, pa, _ = _up(M, d, h, dev_bf16(G["x"]), dev_bf16(G["W1"]), st)
+    post_o = ref.relu2_post(ref.up_proj(G["x"], G["W1"]))
+    assert np.array_equal(host_bits(post.t), post_o)
+    assert np.array_equal(host_bits(q.t), ref.quantise_post(post_o, s))
+    assert np.array_equal(host_bits(pa.t), _pa_oracle(post_o, M, h))
+    P = synth.make_problem(M, d, h, seed=M + d + h)
+
+    def make():
+        b = MLPBlock(M, d, h)
+        for k in ("x", "W1", "W2", "dOut"):
+            getattr(b, k).copy_(MLPBlock.bits_to_bf16(P[k], b.device))
+        b.refresh_w2_cache()
+        b.calibrate()
+        return b
+
+    e, n = make(), make()
+    for _ in range(2):
+        e.refresh_w2_cache()
+        e.train_step()
+        n.train_step_native()
+    torch.cuda.synchronize()
+    for k in ("post", "post_fp8", "out", "dPre", "dX", "dW1", "dW2", "W2q_t", "state", "partial_amax"):
+        assert torch.equal(getattr(e, k), getattr(n, k)), k
+    assert A.fp8mlp_get_device_status() == 0
